@@ -1,0 +1,141 @@
+"""CPU oracle for the Gated DeltaNet token mixer -- TEST INFRASTRUCTURE ONLY.
+
+A plain fp64 restatement (C, threads over (sequence, head)) of what the mixer
+computes, used by the tests, the smoke check and the benchmark's CPU baseline.
+The CUDA library never imports or links it, and it shares no code with it.
+
+Functions here only marshal numpy arrays into the C library built from
+``gdn_oracle.c``; see that file's header for the sources each step follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+_F32, _BF16, _F64 = 0, 1, 2
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        vp, i32, f64, i64p = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
+        L.gdn_oracle_recurrence_mut.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32,
+                                                i32, f64, i32, f64, vp, i32, vp, vp, i32, i32]
+        L.gdn_oracle_recurrence_mut.restype = i32
+        L.gdn_oracle_chunked.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32, i32,
+                                         f64, i32, f64, vp, i32, vp, vp, i32, i32]
+        L.gdn_oracle_chunked.restype = i32
+        L.gdn_oracle_conv_silu.argtypes = [vp, i32, vp, i32, i64p, i32, i32, i32, vp, i32, vp,
+                                           i32, i32, i32, i32, f64, vp, i32]
+        L.gdn_oracle_conv_silu.restype = i32
+        _lib = L
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def _arr(a: np.ndarray, kind: str):
+    """(contiguous array, dtype code). kind 'bf16' means uint16 bit patterns."""
+    if kind == "bf16":
+        a = np.ascontiguousarray(a, dtype=np.uint16)
+        return a, _BF16
+    if a.dtype == np.float64:
+        return np.ascontiguousarray(a), _F64
+    return np.ascontiguousarray(a, dtype=np.float32), _F32
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: float = 1.0,
+               qk_l2norm: bool = True, eps: float = 1e-6, threads: Optional[int] = None,
+               want_o: bool = True, mutation: int = 0):
+    """Token-by-token gated delta rule in fp64.
+
+    q,k [T,H,dk], v [T,H,dv] (uint16 bf16 bits when dtype=='bf16', else
+    float), g/beta [T,H], cu_seqlens [N+1], h0 [N,H,dk,dv] or None.
+    Returns (o [T,H,dv] float64 or None, hT [N,H,dk,dv] float64).
+    """
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    q, dt = _arr(q, dtype)
+    k, _ = _arr(k, dtype)
+    v, _ = _arr(v, dtype)
+    g, gdt = _arr(np.asarray(g), "f")
+    beta = np.ascontiguousarray(beta, dtype=g.dtype)
+    h0a, h0dt = (None, _F64) if h0 is None else _arr(np.asarray(h0), "f")
+    hT = np.empty((N, H, dk, dv), np.float64)
+    o = np.empty((T, H, dv), np.float64) if want_o else None
+    rc = lib().gdn_oracle_recurrence_mut(
+        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, dk, dv,
+        float(scale), int(qk_l2norm), float(eps), _ptr(h0a), h0dt, _ptr(hT), _ptr(o),
+        threads or default_threads(), int(mutation))
+    if rc != 0:
+        raise ValueError("oracle recurrence: bad arguments")
+    return o, hT
+
+
+def chunked(q, k, v, g, beta, cu_seqlens, *, dtype: str, chunk: int, h0=None,
+            scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6,
+            threads: Optional[int] = None):
+    """fp64 chunkwise (UT-transform) evaluation of the same recurrence; used
+    only to check that the chunk algebra equals the token loop."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    q, dt = _arr(q, dtype)
+    k, _ = _arr(k, dtype)
+    v, _ = _arr(v, dtype)
+    g, gdt = _arr(np.asarray(g), "f")
+    beta = np.ascontiguousarray(beta, dtype=g.dtype)
+    h0a, h0dt = (None, _F64) if h0 is None else _arr(np.asarray(h0), "f")
+    hT = np.empty((N, H, dk, dv), np.float64)
+    o = np.empty((T, H, dv), np.float64)
+    rc = lib().gdn_oracle_chunked(
+        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, dk, dv,
+        float(scale), int(qk_l2norm), float(eps), _ptr(h0a), h0dt, _ptr(hT), _ptr(o),
+        int(chunk), threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle chunked: bad arguments")
+    return o, hT
+
+
+def conv_silu(x, w, cu_seqlens, *, dtype: str, state_in=None, apply_silu: bool = True,
+              qk_l2norm: bool = False, n_qk: int = 0, head_dim: int = 128, eps: float = 1e-6,
+              threads: Optional[int] = None):
+    """Causal depthwise conv (+SiLU, + per-head L2 norm of the first n_qk
+    channels) over packed sequences, fp64.
+
+    x [T,C], w [C,K], state_in [N,C,K-1] or None (same encoding as x).
+    Returns (y [T,C] float64, state_out [N,C,K-1] float64).
+    """
+    T, C = x.shape
+    K = w.shape[1]
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    x, dt = _arr(x, dtype)
+    w, wdt = _arr(w, dtype)
+    st, sdt = (None, _F64) if state_in is None else _arr(state_in, dtype)
+    y = np.empty((T, C), np.float64)
+    st_out = np.empty((N, C, K - 1), np.float64)
+    rc = lib().gdn_oracle_conv_silu(
+        _ptr(x), dt, _ptr(w), wdt, _ptr(cu), N, C, K, _ptr(st), sdt, _ptr(st_out),
+        int(apply_silu), int(qk_l2norm), int(n_qk), int(head_dim), float(eps), _ptr(y),
+        threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle conv: bad arguments")
+    return y, st_out
