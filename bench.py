@@ -1,0 +1,517 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet token mixer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline workload (one step): chunked gated-delta-rule prefill of 8 sequences x
+16384 tokens, 16 heads, d_k = d_v = 128, bf16 q/k/v, fp32 gates and fp32 final
+state, chunk 64 -- one gdn_prefill call over the packed batch. Inputs stay
+resident in HBM (about 1.1 GB, larger than the 126 MB L2). The same JSON line
+carries two more measured workloads of the same hot path: batched decode
+(256 sequences, 100 in-place steps) and one 0.8B-shaped layer prefill
+(conv + SiLU + L2 norm, then the chunked prefill, T = 4096).
+
+Multi-GPU: one process per GPU (torchrun), each rank runs its own replica of
+the workload (weak scaling, no data-path collective); the step time is the max
+over ranks.
+
+--impl reference times the CPU oracle (fp64, C, host threads) on a bounded
+sample of the same workload; it is the reference arm of this benchmark.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDN prefill tokens/s & % bf16 TC roofline; decode tokens/s & % HBM BW (1×B200)"
+UNIT = "tokens/s"
+H, D, CHUNK = 16, 128, 64
+SEQS, SEQ_LEN = 8, 16384
+# Algorithmic work per (token, head) of the chunked prefill (chunk C, d = 128):
+# five C x C x d products and three C x d x d products, 2 flops per MAC.
+FLOP_PER_TOKEN_HEAD = 10 * CHUNK * D + 6 * D * D          # 180,224
+# q, k, v, o in bf16 plus g, beta in fp32.
+BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 2 + 2 * 4          # 1,032
+STATE_BYTES = D * D * 4                                    # per (sequence, head)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "gated_deltanet_linear_silu_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, sources, units_this_launch: float):
+    """dram bytes per launch from the committed ncu summary, scaled to this
+    launch's units; None when the kernel source changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec or rec.get("source_hash") != source_hash(*sources):
+        return None
+    return rec["dram_bytes_per_unit"] * units_this_launch
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed regions
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.samples, self.proc, self.err = [], None, None
+        self.active = False
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            target = str(device_index)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", target, f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception as e:  # no nvidia-smi
+            self.err = str(e)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if self.active:
+                self.samples.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        sm = [float(s[0]) for s in self.samples if len(s) >= 7 and s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if len(s) >= 7 and s[1].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in self.samples:
+            if len(s) >= 7:
+                for nm, val in zip(names, s[3:7]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (barrier + max over ranks only)
+# ----------------------------------------------------------------------------
+
+class Dist:
+    def __init__(self, want: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+        if self.world != want:
+            raise SystemExit(f"--gpus {want} but WORLD_SIZE={self.world}")
+
+    def init(self):
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(self.local)
+        if self.world > 1:
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(P, tokens: int, n_seq: int):
+    """Oracle over the first `tokens` tokens of the first n_seq sequences, all
+    heads. Returns (token count processed, seconds, threads)."""
+    import numpy as np
+    import oracle
+    qs, ks, vs, gs, bs, cu = [], [], [], [], [], [0]
+    for n in range(n_seq):
+        a = int(P.cu_seqlens[n])
+        b = min(int(P.cu_seqlens[n + 1]), a + tokens)
+        for lst, arr in ((qs, P.q), (ks, P.k), (vs, P.v), (gs, P.g), (bs, P.beta)):
+            lst.append(arr[a:b])
+        cu.append(cu[-1] + (b - a))
+    cat = lambda xs: np.ascontiguousarray(np.concatenate(xs))
+    threads = min(oracle.default_threads(), n_seq * P.H)
+    t0 = time.perf_counter()
+    oracle.recurrence(cat(qs), cat(ks), cat(vs), cat(gs), cat(bs), cu, dtype=P.dtype,
+                      qk_l2norm=P.qk_l2norm, threads=threads, want_o=True)
+    return cu[-1], time.perf_counter() - t0, threads
+
+
+def calibrated_sample(P, target_s: float):
+    """Pick (tokens, n_seq) so one oracle pass takes about target_s seconds."""
+    import oracle
+    n_seq = max(1, min(P.N, oracle.default_threads() // P.H or 1))
+    tok, dt, _ = oracle_sample(P, 512, n_seq)
+    rate = tok / max(dt, 1e-6)  # tokens/s with n_seq sequences in parallel
+    tokens = int(max(256, min(SEQ_LEN, rate * target_s / n_seq)))
+    return tokens, n_seq
+
+
+def run_reference(args, dist: Dist):
+    import gdn_inputs as gi
+    if dist.rank != 0:
+        return
+    P = gi.long_prefill(SEQS, SEQ_LEN, H, D)
+    tokens, n_seq = calibrated_sample(P, 5.0)
+    for _ in range(args.warmup):
+        oracle_sample(P, min(tokens, 1024), n_seq)
+    times, toks, threads = [], 0, 1
+    for _ in range(args.steps):
+        tk, dt, threads = oracle_sample(P, tokens, n_seq)
+        times.append(dt)
+        toks = tk
+    step_s = statistics.mean(times)
+    value = toks / step_s
+    sample = f"first {tokens} tokens of {n_seq} of the 8 sequences, all 16 heads, fp64 token loop"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def config_block(n):
+    return {"workload": "long_prefill_8x16384_h16_d128_bf16", "global_batch": SEQS * n,
+            "seq_len": SEQ_LEN, "heads": H, "head_dim": D, "chunk": CHUNK,
+            "parallelism": f"replicas{n}" if n > 1 else "single",
+            "l2": "inputs larger than L2 (1.1 GB resident per step)"}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def timed(fn, steps, stream):
+    """Run fn `steps` times between two events; returns (total ms, per-call ms)."""
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(steps):
+        fn()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    return evs[0].elapsed_time(evs[-1]), per
+
+
+def bench_prefill(args, dist, pk):
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+
+    dev = torch.device("cuda", dist.local)
+    P = gi.long_prefill(SEQS, SEQ_LEN, H, D)
+    T = P.T_tot
+
+    def pinned(a, dtype):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if dtype == torch.bfloat16
+                             else np.ascontiguousarray(a))
+        t = t.view(dtype) if dtype == torch.bfloat16 else t
+        return t.pin_memory()
+
+    hq, hk, hv = (pinned(a, torch.bfloat16) for a in (P.q, P.k, P.v))
+    hg, hb = pinned(P.g, torch.float32), pinned(P.beta, torch.float32)
+    hcu = torch.from_numpy(P.cu_seqlens.astype(np.int32)).pin_memory()
+    q, k, v, g, beta = (t.to(dev) for t in (hq, hk, hv, hg, hb))
+    cu = hcu.to(dev)
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((SEQS, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(SEQS, T, H, D, D, CHUNK), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, chunk=CHUNK,
+                    algo=args.algo)
+
+    for _ in range(args.warmup):
+        step()
+    gdn.check_device_status(dev)
+    dist.barrier()
+    torch.cuda.synchronize()
+    total_ms, per = timed(step, args.steps, stream)
+    dist.barrier()
+    total_ms = dist.max(total_ms)
+    kernel_ms = dist.max(statistics.mean(per))
+    gdn.check_device_status(dev)
+
+    # end to end: pinned host inputs -> device -> library -> host outputs
+    ho = torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory()
+    hhT = torch.empty((SEQS, H, D, D), dtype=torch.float32).pin_memory()
+    cu_e = torch.empty_like(cu)
+
+    def e2e_step():
+        for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg), (beta, hb), (cu_e, hcu)):
+            dst.copy_(src, non_blocking=True)
+        gdn.prefill(q, k, v, g, beta, cu_e, final_state=hT, out=o, workspace=ws, chunk=CHUNK,
+                    algo=args.algo)
+        ho.copy_(o, non_blocking=True)
+        hhT.copy_(hT, non_blocking=True)
+
+    e2e_step()
+    dist.barrier()
+    torch.cuda.synchronize()
+    e2e_ms, _ = timed(e2e_step, max(1, min(args.steps, 5)), stream)
+    e2e_steps = max(1, min(args.steps, 5))
+    dist.barrier()
+    e2e_ms = dist.max(e2e_ms)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hcu))
+    d2h = ho.numel() * ho.element_size() + hhT.numel() * hhT.element_size()
+    res = {"P": P, "tokens": T, "total_ms": total_ms, "kernel_ms": kernel_ms,
+           "e2e_ms_per_step": e2e_ms / e2e_steps, "h2d": h2d, "d2h": d2h}
+    del q, k, v, g, beta, o, hT, hq, hk, hv, ho, hhT
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode(args, dist, pk):
+    """256 sequences x 16 heads, d=128, 100 in-place steps (one call each)."""
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    N, steps = 256, 100
+    state = torch.from_numpy(gi.decode_state(N, H, D)).to(dev)
+    ins = []
+    for s in range(steps):
+        Dd = gi.decode_step(s, N, H, D)
+        bf = lambda a: torch.from_numpy(a.view("int16")).to(dev).view(torch.bfloat16)
+        ins.append((bf(Dd.q), bf(Dd.k), bf(Dd.v), torch.from_numpy(Dd.g).to(dev),
+                    torch.from_numpy(Dd.beta).to(dev)))
+    o = torch.empty((N, H, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    it = iter(range(10 ** 9))
+
+    def step():
+        i = next(it) % steps
+        gdn.decode_step(*ins[i], state, out=o)
+
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    total_ms, per = timed(step, steps, stream)
+    total_ms = dist.max(total_ms)
+    step_ms = total_ms / steps
+    bytes_step = 2 * N * H * STATE_BYTES + N * H * (4 * D * 2 + 8)
+    return {"value": N / (step_ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": step_ms,
+            "workload": "decode_256x16_d128_100steps",
+            "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": profiled_traffic("decode_step_kernel", ["decode.cu"], N * H),
+                         "algorithmic_bytes": bytes_step},
+            "gpu_launches": steps}
+
+
+def bench_layer(args, dist, pk):
+    """0.8B-shaped layer prefill: conv + SiLU + L2 norm, then chunked prefill."""
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    Lw = gi.layer_0p8b()
+    T = Lw.T_tot
+    bf = lambda a: torch.from_numpy(a.view("int16")).to(dev).view(torch.bfloat16)
+    x, w = bf(Lw.mixed_qkv), bf(Lw.conv_w)
+    g, beta = torch.from_numpy(Lw.g).to(dev), torch.from_numpy(Lw.beta).to(dev)
+    cu = torch.from_numpy(Lw.cu_seqlens).to(dev)
+    y = torch.empty_like(x)
+    st = torch.empty((1, Lw.C, 3), dtype=torch.bfloat16, device=dev)
+    q = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    o = torch.empty_like(q)
+    hT = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(1, T, H, D, D, CHUNK), dtype=torch.uint8, device=dev)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def conv():
+        gdn.conv_silu(x, w, cu, conv_state_out=st, out=y, n_qk_channels=2 * H * D, head_dim=D)
+
+    def layer():
+        conv()
+        qkv = y.view(T, 3, H, D)
+        q.copy_(qkv[:, 0]); k.copy_(qkv[:, 1]); v.copy_(qkv[:, 2])
+        gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, qk_l2norm=False)
+
+    conv_ms, layer_ms = [], []
+    for rep in range(8):
+        for fn, acc in ((conv, conv_ms), (layer, layer_ms)):
+            flush.fill_(rep & 0xFF)  # L2 flush: the layer's inputs fit in L2
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            torch.cuda.synchronize()
+            if rep >= 3:
+                acc.append(s.elapsed_time(e))
+    cms, lms = statistics.median(conv_ms), statistics.median(layer_ms)
+    conv_bytes = 2 * T * Lw.C * 2 + Lw.C * 4 * 2
+    return {"value": T / (lms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": lms,
+            "workload": "layer_0p8b_T4096_conv_then_prefill",
+            "note": "layer time includes three torch copies splitting [q|k|v] for the prefill",
+            "conv": {"ms": cms, "roofline": {
+                "bound": "hbm", "achieved": conv_bytes / (cms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": conv_bytes / (cms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                "traffic": profiled_traffic("conv_silu_kernel", ["conv_silu.cu"], T),
+                "algorithmic_bytes": conv_bytes}}}
+
+
+def run_ours(args, dist: Dist):
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    gdn.lib()  # fail loudly if the library is missing
+    pk = peaks()
+    clocks = ClockSampler(dist.local)
+
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        import gdn_inputs as gi
+        P = gi.long_prefill(SEQS, SEQ_LEN, H, D)
+        tokens, n_seq = calibrated_sample(P, 15.0)
+        tok, dt, threads = oracle_sample(P, tokens, n_seq)
+        cpu = {"value": tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"first {tokens} tokens of {n_seq} of the 8 sequences, all 16 heads "
+                         f"({tok} tokens, {dt:.1f} s, fp64 token loop)"}
+        del P
+
+    clocks.active = True
+    pre = bench_prefill(args, dist, pk)
+    extras = {}
+    if not args.no_extras:
+        extras["decode"] = bench_decode(args, dist, pk)
+        extras["layer"] = bench_layer(args, dist, pk)
+    clocks.active = False
+    clk = clocks.stop()
+
+    tokens_all = pre["tokens"] * dist.world
+    ms_per_step = pre["total_ms"] / args.steps
+    kernel_s = pre["kernel_ms"] * 1e-3
+    th = pre["tokens"] * H
+    flops = th * FLOP_PER_TOKEN_HEAD
+    bytes_alg = th * BYTES_PER_TOKEN_HEAD + SEQS * H * STATE_BYTES
+    hbm_ach = bytes_alg / kernel_s / 1e9
+    tc_ach = flops / kernel_s / 1e12
+    algo = gdn.selected_algo("bf16", D, D, CHUNK, args.algo)
+    tc_used = algo == "tensor"
+    line = {
+        "metric": METRIC, "value": tokens_all / (ms_per_step * 1e-3), "unit": UNIT,
+        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if tc_used else "f32", "data": "synthetic",
+        "config": config_block(dist.world),
+        "roofline": {"bound": "hbm", "achieved": hbm_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": hbm_ach / pk["hbm_gbs"],
+                     "traffic": profiled_traffic("prefill", ["prefill_simt.cu", "prefill_tc.cu"],
+                                                 th),
+                     "kernel": "gdn_prefill (schedule + chunk kernel), CUDA events per call",
+                     "algorithmic_bytes": bytes_alg, "peak_source": pk["source"]},
+        "tc_roofline": {"achieved": tc_ach, "unit": "TFLOP/s", "peak": pk["bf16_tflops"],
+                        "frac": tc_ach / pk["bf16_tflops"],
+                        "frac_sustained": tc_ach / pk["bf16_tflops_sustained"]
+                        if pk.get("bf16_tflops_sustained") else None,
+                        "algorithmic_flops": flops},
+        "e2e": {"value": tokens_all / (pre["e2e_ms_per_step"] * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"]},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+        "algo": algo,
+    }
+    if cpu:
+        line["cpu_baseline"] = cpu
+    line.update(extras)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--no-extras", action="store_true", help="headline workload only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    dist = Dist(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    dist.init()
+    try:
+        run_ours(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

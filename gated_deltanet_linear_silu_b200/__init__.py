@@ -1,0 +1,203 @@
+"""Gated DeltaNet token mixer on B200 (sm_100a): Python binding of libgdn.so.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/gdn.h. PyTorch supplies device
+memory and the current stream. There is no CPU fallback: if libgdn.so has not
+been built (``python -m gated_deltanet_linear_silu_b200.build``) every call
+raises.
+
+Operations (the Qwen3.5 linear-attention layer's token mixer):
+  conv_silu     causal depthwise conv1d (k <= 4) + SiLU over [q | k | v]
+                channels, optional per-head L2 norm of q and k, conv state.
+  prefill       chunked gated delta rule over packed sequences (cu_seqlens),
+                optional initial state, fp32 final state.
+  decode_step   one token per sequence, fp32 state updated in place.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_F32, GDN_BF16 = 0, 1
+ALGOS = {"auto": 0, "simt": 1, "tensor": 2}
+STATUS = {0: "GDN_OK", 1: "GDN_ERR_INVALID_ARG", 2: "GDN_ERR_UNSUPPORTED",
+          3: "GDN_ERR_WORKSPACE", 4: "GDN_ERR_CUDA", 5: "GDN_ERR_TIMEOUT"}
+
+_lib = None
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m gated_deltanet_linear_silu_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                                 ctypes.c_size_t)
+        L.gdn_conv_silu.argtypes = [vp, i32, vp, vp, i32, i64, i32, i32, vp, vp, i32, i32, i32, f32,
+                                    vp, vp]
+        L.gdn_conv_silu.restype = i32
+        L.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
+        L.gdn_prefill_workspace_size.restype = sz
+        L.gdn_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32, f32, i32,
+                                  f32, i32, vp, vp, vp, vp, sz, i32, vp]
+        L.gdn_prefill.restype = i32
+        L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, i32, f32,
+                                      vp, vp]
+        L.gdn_decode_step.restype = i32
+        L.gdn_status_string.argtypes = [i32]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_check_device_status.argtypes = [vp]
+        L.gdn_check_device_status.restype = i32
+        L.gdn_prefill_selected_algo.argtypes = [i32, i32, i32, i32, i32]
+        L.gdn_prefill_selected_algo.restype = i32
+        L.gdn_version.argtypes = []
+        L.gdn_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise GDNError(status, what)
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def conv_silu(x: torch.Tensor, w: torch.Tensor, cu_seqlens: torch.Tensor, *,
+              conv_state: Optional[torch.Tensor] = None, conv_state_out: Optional[torch.Tensor] = None,
+              return_state: bool = True, qk_l2norm: bool = True, n_qk_channels: Optional[int] = None,
+              head_dim: int = 128, eps: float = 1e-6, out: Optional[torch.Tensor] = None
+              ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """y = SiLU(causal depthwise conv(x)) (+ L2 norm of the first n_qk_channels
+    per head). x [T, C], w [C, K], cu_seqlens int32 [N+1] on the device,
+    conv_state [N, C, K-1] or None. Returns (y, conv_state_out)."""
+    T, C = x.shape
+    K = w.shape[1]
+    N = cu_seqlens.shape[0] - 1
+    if n_qk_channels is None:
+        n_qk_channels = 2 * (C // 3)
+    y = torch.empty_like(x) if out is None else out
+    st_out = conv_state_out
+    if st_out is None and return_state:
+        st_out = torch.empty((N, C, K - 1), dtype=x.dtype, device=x.device)
+    _cuda(x, w, cu_seqlens, conv_state, st_out, y)
+    st = lib().gdn_conv_silu(_ptr(x), _dtype_code(x), _ptr(w), _ptr(cu_seqlens), N, T, C, K,
+                             _ptr(conv_state), _ptr(st_out), int(qk_l2norm), int(n_qk_channels),
+                             int(head_dim), float(eps), _ptr(y), _stream(x.device))
+    _check(st, "gdn_conv_silu")
+    return y, st_out
+
+
+def prefill_workspace_size(N: int, T_tot: int, H: int, dk: int, dv: int, chunk: int = 64) -> int:
+    return int(lib().gdn_prefill_workspace_size(N, T_tot, H, dk, dv, chunk))
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+            cu_seqlens: torch.Tensor, *, initial_state: Optional[torch.Tensor] = None,
+            output_final_state: bool = True, final_state: Optional[torch.Tensor] = None,
+            scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6, chunk: int = 64,
+            cu_seqlens_host: Optional[torch.Tensor] = None, algo: str = "auto",
+            workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None
+            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked gated delta rule. q,k [T,H,dk], v [T,H,dv] (bf16 or fp32),
+    g,beta [T,H] fp32, cu_seqlens int32 [N+1] (device). Returns (o, hT);
+    final_state may be initial_state itself for an in-place update."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device) if out is None else out
+    hT = final_state
+    if hT is None and output_final_state:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    ws_bytes = prefill_workspace_size(N, T, H, dk, dv, chunk)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _cuda(q, k, v, g, beta, cu_seqlens, initial_state, hT, o, workspace)
+    host_cu = None
+    if cu_seqlens_host is not None:
+        host_cu = cu_seqlens_host.to(torch.int32).contiguous()
+    st = lib().gdn_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+        None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, dk, dv,
+        float(scale), int(qk_l2norm), float(eps), int(chunk), _ptr(initial_state), _ptr(hT),
+        _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
+    _check(st, "gdn_prefill")
+    return o, hT
+
+
+def selected_algo(dtype: str, dk: int, dv: int, chunk: int = 64, algo: str = "auto") -> str:
+    """Name of the prefill kernel ("simt" or "tensor") that would run; raises
+    if the combination is unsupported."""
+    code = lib().gdn_prefill_selected_algo(GDN_BF16 if dtype == "bf16" else GDN_F32, dk, dv,
+                                            chunk, ALGOS[algo])
+    if code < 0:
+        raise GDNError(2, "gdn_prefill_selected_algo")
+    return {1: "simt", 2: "tensor"}[code]
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                beta: torch.Tensor, state: torch.Tensor, *, scale: float = 1.0,
+                qk_l2norm: bool = True, eps: float = 1e-6, out: Optional[torch.Tensor] = None
+                ) -> torch.Tensor:
+    """One recurrent token per sequence. q,k [N,H,dk], v [N,H,dv], g,beta
+    [N,H] fp32, state [N,H,dk,dv] fp32 updated in place. Returns o [N,H,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device) if out is None else out
+    _cuda(q, k, v, g, beta, state, o)
+    st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta),
+                               _ptr(state), N, H, dk, dv, float(scale), int(qk_l2norm), float(eps),
+                               _ptr(o), _stream(q.device))
+    _check(st, "gdn_decode_step")
+    return o
+
+
+def check_device_status(device: Optional[torch.device] = None) -> None:
+    """Synchronise and raise if a kernel skipped work (bad cu_seqlens, timeout)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _check(lib().gdn_check_device_status(_stream(dev)), "device status")
+
+
+def state_bytes(n_layers: int, heads: int, dk: int, dv: int, elem_bytes: int = 4) -> int:
+    """Bytes of recurrent state for n_layers mixer layers (independent of length)."""
+    return n_layers * heads * dk * dv * elem_bytes
+
+
+def conv_channels(key_heads: int, key_head_dim: int, value_heads: int, value_head_dim: int) -> int:
+    """Channels of the fused conv input: q and k (key_dim each) then v."""
+    return 2 * key_heads * key_head_dim + value_heads * value_head_dim

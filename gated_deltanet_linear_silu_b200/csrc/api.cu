@@ -1,0 +1,188 @@
+// C ABI of libgdn (declared in include/gdn.h): argument validation on the
+// host, workspace carving, kernel dispatch. No allocation, no host sync except
+// in gdn_check_device_status.
+#include <mutex>
+
+#include "../../include/gdn.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace gdn {
+size_t prefill_simt_smem_bytes(int chunk, int dk, int dv);
+}
+
+namespace {
+
+// Device status word: kernels set it (first error wins) when they skip work.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+std::mutex g_status_mu;
+
+// Address of the status word on the current device (looked up once per device).
+int* status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_dim_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
+bool dtype_ok(gdn_dtype_t t) { return t == GDN_F32 || t == GDN_BF16; }
+
+gdn_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+gdn_status_t check_host_seqlens(const int32_t* cu, int N, int64_t T_tot) {
+    if (!cu) return GDN_OK;
+    if (cu[0] != 0 || cu[N] != T_tot) return GDN_ERR_INVALID_ARG;
+    for (int n = 0; n < N; ++n)
+        if (cu[n + 1] < cu[n]) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_version(void) { return 100; }  // 0.1.0
+
+const char* gdn_status_string(gdn_status_t s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
+    }
+    return "GDN_ERR_UNKNOWN";
+}
+
+gdn_status_t gdn_check_device_status(void* stream) {
+    int* p = status_ptr();
+    if (!p) return GDN_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int word = 0;
+    if (cudaMemcpyAsync(&word, p, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyAsync(p, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return GDN_ERR_CUDA;
+    }
+    if (word == gdn::kStatusBadSeqlens) return GDN_ERR_INVALID_ARG;
+    if (word == gdn::kStatusTimeout) return GDN_ERR_TIMEOUT;
+    return word == 0 ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_conv_silu(const void* x, gdn_dtype_t dtype, const void* w,
+                           const int32_t* cu_seqlens, int N, int64_t T_tot, int C, int K,
+                           const void* conv_state_in, void* conv_state_out, int qk_l2norm,
+                           int n_qk_channels, int head_dim, float eps, void* y, void* stream) {
+    if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || C <= 0 || K < 1) return GDN_ERR_INVALID_ARG;
+    if (N == 0 && T_tot > 0) return GDN_ERR_INVALID_ARG;
+    if (N > 0 && !cu_seqlens) return GDN_ERR_INVALID_ARG;
+    if (T_tot > 0 && (!x || !y || !w)) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(w)) return GDN_ERR_INVALID_ARG;
+    if (K > 4 || C % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    if (qk_l2norm) {
+        if (!(head_dim == 16 || head_dim == 32 || head_dim == 64 || head_dim == 128))
+            return GDN_ERR_UNSUPPORTED;
+        if (n_qk_channels < 0 || n_qk_channels % head_dim != 0 || n_qk_channels > C || !(eps >= 0.f))
+            return GDN_ERR_INVALID_ARG;
+    }
+    if (x == y) return GDN_ERR_INVALID_ARG;
+    if (N == 0) return GDN_OK;
+    gdn::ConvArgs a{x, dtype == GDN_BF16, w, cu_seqlens, N, T_tot, C, K, conv_state_in,
+                    conv_state_out, qk_l2norm, n_qk_channels, head_dim, eps, y, status_ptr()};
+    if (!a.status) return GDN_ERR_CUDA;
+    return from_cuda(gdn::launch_conv_silu(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, int chunk) {
+    (void)T_tot; (void)H; (void)dk; (void)dv; (void)chunk;
+    return gdn::prefill_workspace_layout(N < 0 ? 0 : N).total;
+}
+
+gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                         const float* g, const float* beta, const int32_t* cu_seqlens,
+                         const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int dk,
+                         int dv, float scale, int qk_l2norm, float eps, int chunk, const float* h0,
+                         float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
+                         void* stream) {
+    if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+    if (N == 0 && T_tot > 0) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (!(chunk == 16 || chunk == 32 || chunk == 64)) return GDN_ERR_UNSUPPORTED;
+    if (!(algo == GDN_ALGO_AUTO || algo == GDN_ALGO_SIMT || algo == GDN_ALGO_TENSOR))
+        return GDN_ERR_INVALID_ARG;
+    if (N > 0 && !cu_seqlens) return GDN_ERR_INVALID_ARG;
+    if (T_tot > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(h0) ||
+        !aligned16(hT))
+        return GDN_ERR_INVALID_ARG;
+    if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)N * H * 2 >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    if (T_tot >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;  // cu_seqlens is int32
+    if (gdn_status_t st = check_host_seqlens(cu_seqlens_host, N, T_tot)) return st;
+    if (N == 0) return GDN_OK;
+    const gdn::WorkspaceLayout wl = gdn::prefill_workspace_layout(N);
+    if (!workspace || ws_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GDN_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    gdn::PrefillArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, dk, dv,
+                       scale, qk_l2norm, eps, chunk, h0, hT, o,
+                       reinterpret_cast<int32_t*>(ws + wl.order_off),
+                       reinterpret_cast<int32_t*>(ws + wl.counter_off), status_ptr()};
+    if (!a.status) return GDN_ERR_CUDA;
+    const bool tc_ok = gdn::prefill_tc_supported(a);
+    if (algo == GDN_ALGO_TENSOR && !tc_ok) return GDN_ERR_UNSUPPORTED;
+    const bool use_tc = tc_ok && algo != GDN_ALGO_SIMT;
+    if (!use_tc && gdn::prefill_simt_smem_bytes(chunk, dk, dv) > 227 * 1024) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = gdn::launch_prefill_schedule(a, s);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    e = use_tc ? gdn::launch_prefill_tc(a, s) : gdn::launch_prefill_simt(a, s);
+    return from_cuda(e);
+}
+
+int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_algo_t algo) {
+    if (!dtype_ok(dtype) || !head_dim_ok(dk) || !head_dim_ok(dv)) return -1;
+    if (!(chunk == 16 || chunk == 32 || chunk == 64)) return -1;
+    gdn::PrefillArgs a{};
+    a.is_bf16 = dtype == GDN_BF16;
+    a.dk = dk;
+    a.dv = dv;
+    a.chunk = chunk;
+    const bool tc_ok = gdn::prefill_tc_supported(a);
+    if (algo == GDN_ALGO_TENSOR) return tc_ok ? GDN_ALGO_TENSOR : -1;
+    if (algo == GDN_ALGO_SIMT || !tc_ok)
+        return gdn::prefill_simt_smem_bytes(chunk, dk, dv) <= 227 * 1024 ? GDN_ALGO_SIMT : -1;
+    return GDN_ALGO_TENSOR;
+}
+
+gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                             const float* g, const float* beta, float* state, int N, int H, int dk,
+                             int dv, float scale, int qk_l2norm, float eps, void* o, void* stream) {
+    if (!dtype_ok(dtype) || N < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (N == 0) return GDN_OK;
+    if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(state))
+        return GDN_ERR_INVALID_ARG;
+    if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, dk, dv, scale, qk_l2norm, eps, o};
+    return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+// Internal launcher declarations of libgdn (host side). Arguments are
+// validated by the C-ABI layer (api.cu) before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct ConvArgs {
+    const void* x;
+    int is_bf16;
+    const void* w;
+    const int32_t* cu;
+    int N;
+    int64_t T_tot;
+    int C, K;
+    const void* state_in;
+    void* state_out;
+    int qk_l2norm, n_qk, head_dim;
+    float eps;
+    void* y;
+    int* status;
+};
+cudaError_t launch_conv_silu(const ConvArgs& a, cudaStream_t s);
+
+struct DecodeArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    int is_bf16;
+    const float* g;
+    const float* beta;
+    float* state;
+    int N, H, dk, dv;
+    float scale;
+    int qk_l2norm;
+    float eps;
+    void* o;
+};
+cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
+
+struct PrefillArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    int is_bf16;
+    const float* g;
+    const float* beta;
+    const int32_t* cu;
+    int N;
+    int64_t T_tot;
+    int H, dk, dv;
+    float scale;
+    int qk_l2norm;
+    float eps;
+    int chunk;
+    const float* h0;
+    float* hT;
+    void* o;
+    // Workspace carve-up (see prefill_workspace_layout).
+    int32_t* order;    // [N] sequences, longest first
+    int32_t* counter;  // [1] work counter of the persistent kernels
+    int* status;
+};
+
+struct WorkspaceLayout {
+    size_t counter_off, order_off, total;
+};
+WorkspaceLayout prefill_workspace_layout(int N);
+
+// Builds the longest-first schedule and zeroes the work counter.
+cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
+bool prefill_tc_supported(const PrefillArgs& a);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+
+}  // namespace gdn

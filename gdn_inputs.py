@@ -34,7 +34,9 @@ beta and g = log(alpha) as given.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import os
 from typing import Optional
 
 import numpy as np
@@ -223,10 +225,14 @@ def _packed(workload: int, name: str, lengths, H: int, d: int, g_scale: float,
     v = np.empty_like(q)
     beta = np.empty((T_tot, H), np.float32)
     g = np.empty_like(beta)
-    for n, T in enumerate(lengths):
-        s = sequence_tensors(workload, n, int(T), H, d, g_scale)
+
+    def fill(n):  # numpy releases the GIL while drawing, so sequences fill in parallel
+        s = sequence_tensors(workload, n, int(lengths[n]), H, d, g_scale)
         a, b = int(cu[n]), int(cu[n + 1])
         q[a:b], k[a:b], v[a:b], beta[a:b], g[a:b] = s["q"], s["k"], s["v"], s["beta"], s["g"]
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(len(lengths))))
     return Prefill(name, q, k, v, g, beta, cu.astype(np.int32), h0, "bf16", H, d, d)
 
 

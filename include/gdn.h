@@ -1,0 +1,192 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the Gated DeltaNet token mixer on NVIDIA B200
+ * (sm_100a). Three operations, as the Qwen3.5 linear-attention layer uses
+ * them:
+ *
+ *   gdn_conv_silu    causal depthwise conv1d + SiLU over the fused q/k/v
+ *                    channels, optional per-head L2 norm of q and k, with a
+ *                    rolling conv state.
+ *   gdn_prefill      chunked gated delta rule over packed variable-length
+ *                    sequences, optional initial state, fp32 final state.
+ *   gdn_decode_step  one recurrent token per sequence, state updated in place.
+ *
+ * Sources (page title, section):
+ *   [R] "Qwen3.5-MoE source walkthrough", 4.3 Qwen3_5MoeGatedDeltaNet: the
+ *       recurrent rule. With the state S stored as [d_k, d_v]:
+ *         S <- exp(g_t) S;  m = S^T k_t;  delta = beta_t (v_t - m);
+ *         S <- S + k_t delta^T;  o_t = S^T q_t.
+ *   [P] same page, 8.2 (linear_attention cache update): multi-token calls go
+ *       through the chunked kernel and return (output, last recurrent state);
+ *       single-token calls use the recurrent kernel and the conv update; the
+ *       conv and recurrent states are carried between calls.
+ *   [C] "7.6 Qwen3.5: linear-attention hybrid", 7.6.2: depthwise causal
+ *       Conv1d, kernel 4, padding 3, over conv_dim = 2*key_dim + value_dim
+ *       channels; L2 normalisation of q and k before the recurrence.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     contiguous, 16-byte aligned. The library never allocates or frees.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
+ *     asynchronous on it. Argument errors are detected on the host and
+ *     returned synchronously; nothing is launched in that case.
+ *   - A launch failure returns GDN_ERR_CUDA (the CUDA error is left for the
+ *     caller to query with cudaGetLastError()).
+ *   - Problems that only the device can see (a cu_seqlens array that is not
+ *     monotone, a bounded wait that ran out) set a device status word and the
+ *     affected work is skipped; gdn_check_device_status() reports and clears it.
+ *   - No call aborts, exits, traps or asserts on the device.
+ *   - dtype applies to q/k/v/o (and x/w/y for the conv). Gates g, beta and the
+ *     recurrent states are always fp32. Arithmetic is fp32 throughout.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or cu_seqlens */
+    GDN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. head dim 80) */
+    GDN_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required */
+    GDN_ERR_CUDA = 4,         /* a CUDA launch or query failed */
+    GDN_ERR_TIMEOUT = 5       /* a bounded device-side wait ran out */
+} gdn_status_t;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype_t;
+
+/* Which prefill kernel runs. AUTO picks the tcgen05 tensor-core kernel for
+ * bf16 with d_k = d_v = 128 and chunk 64, and the fp32 CUDA-core kernel
+ * otherwise. SIMT forces the CUDA-core kernel (any supported shape).
+ * TENSOR forces the tensor-core kernel (GDN_ERR_UNSUPPORTED if the shape is
+ * not one it handles). */
+typedef enum { GDN_ALGO_AUTO = 0, GDN_ALGO_SIMT = 1, GDN_ALGO_TENSOR = 2 } gdn_algo_t;
+
+/*
+ * Causal depthwise conv1d + SiLU (+ per-head L2 norm of q and k). [C], [P]
+ *
+ *   y[t, c] = SiLU( sum_{j=0}^{K-1} w[c, j] * x~[t - (K-1) + j, c] )
+ *
+ * where x~ is the sequence's own input, preceded by its conv state (or by
+ * zeros when conv_state_in is NULL); sequences never mix. This is PyTorch
+ * Conv1d(groups=C, padding=K-1) cross-correlation truncated to the first T
+ * outputs. When qk_l2norm is set, the first n_qk_channels channels (q then k)
+ * are then divided, per token and per group of head_dim channels, by
+ * sqrt(sum of squares + eps).
+ *
+ *   x               [T_tot, C]     dtype   packed inputs (channels [q | k | v],
+ *                                          head-major inside each block)
+ *   w               [C, K]         dtype   conv taps
+ *   cu_seqlens      [N+1]          int32   device prefix offsets, cu[0] = 0,
+ *                                          cu[N] = T_tot, non-decreasing
+ *   conv_state_in   [N, C, K-1]    dtype   nullable: the K-1 inputs preceding
+ *                                          each sequence, oldest first
+ *   conv_state_out  [N, C, K-1]    dtype   nullable: the K-1 latest inputs of
+ *                                          each sequence (state_in's columns
+ *                                          fill in when T < K-1); may alias
+ *                                          conv_state_in (in-place update)
+ *   y               [T_tot, C]     dtype   output; must not overlap x
+ * Supported: 1 <= K <= 4; C a multiple of 8; when qk_l2norm, head_dim in
+ * {16, 32, 64, 128} and n_qk_channels a multiple of head_dim, <= C.
+ */
+GDN_API gdn_status_t gdn_conv_silu(const void* x, gdn_dtype_t dtype, const void* w,
+                           const int32_t* cu_seqlens, int N, int64_t T_tot, int C, int K,
+                           const void* conv_state_in, void* conv_state_out,
+                           int qk_l2norm, int n_qk_channels, int head_dim, float eps,
+                           void* y, void* stream);
+
+/*
+ * Bytes of device workspace gdn_prefill needs for this problem (a multiple of
+ * 256; never 0). The workspace holds the work schedule (sequences ordered
+ * longest first) and a work counter; it is rewritten by every call.
+ */
+GDN_API size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, int chunk);
+
+/*
+ * Chunked gated delta rule over packed sequences. [R], [P]
+ *
+ * For each sequence n (tokens cu[n] .. cu[n+1]-1) and head h, starting from
+ * S = h0[n, h] (zeros when h0 is NULL), every token t applies
+ *   q^ = scale * L2(q_t), k^ = L2(k_t)  (L2(x) = x / sqrt(sum x^2 + eps) when
+ *                                        qk_l2norm, else identity)
+ *   S <- exp(g_t) S;  delta = beta_t (v_t - S^T k^);  S <- S + k^ delta^T;
+ *   o_t = S^T q^
+ * and the final S is written to hT[n, h]. The kernels evaluate this in chunks
+ * of `chunk` tokens (cumulative decay, UT transform with a unit lower
+ * triangular solve, inter-chunk state passing); the result equals the token
+ * loop up to rounding.
+ *
+ *   q, k            [T_tot, H, dk]  dtype
+ *   v               [T_tot, H, dv]  dtype
+ *   g, beta         [T_tot, H]      fp32    g = log(alpha) <= 0 expected
+ *   cu_seqlens      [N+1]           int32   device prefix offsets
+ *   cu_seqlens_host [N+1]           int32   nullable host copy; when given it
+ *                                           is validated on the host
+ *   h0              [N, H, dk, dv]  fp32    nullable initial state
+ *   hT              [N, H, dk, dv]  fp32    nullable final state; may alias h0
+ *   o               [T_tot, H, dv]  dtype   output
+ *   workspace       ws_bytes >= gdn_prefill_workspace_size(...)
+ * A sequence of length 0 writes hT = h0 (or zeros) and no output.
+ * Supported: dk, dv in {16, 32, ..., 128}; chunk in {16, 32, 64}.
+ * Except for hT == h0, no two buffers may overlap.
+ */
+GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                         const float* g, const float* beta,
+                         const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                         int N, int64_t T_tot, int H, int dk, int dv,
+                         float scale, int qk_l2norm, float eps, int chunk,
+                         const float* h0, float* hT, void* o,
+                         void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream);
+
+/*
+ * The prefill kernel gdn_prefill would run for these arguments:
+ * GDN_ALGO_SIMT or GDN_ALGO_TENSOR, or -1 if the combination is unsupported.
+ */
+GDN_API int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_algo_t algo);
+
+/*
+ * One recurrent step for N independent sequences (one token each). [R], [P]
+ * Same per-token rule as gdn_prefill; `state` is read and overwritten in
+ * place with the post-token state.
+ *
+ *   q, k     [N, H, dk]       dtype
+ *   v        [N, H, dv]       dtype
+ *   g, beta  [N, H]           fp32
+ *   state    [N, H, dk, dv]   fp32   in/out
+ *   o        [N, H, dv]       dtype
+ * Supported: dk, dv in {16, 32, ..., 128}.
+ */
+GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                             const float* g, const float* beta, float* state,
+                             int N, int H, int dk, int dv, float scale, int qk_l2norm,
+                             float eps, void* o, void* stream);
+
+/* Static, human-readable name of a status code. */
+GDN_API const char* gdn_status_string(gdn_status_t status);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when they skip work they cannot do safely. Returns GDN_OK,
+ * GDN_ERR_INVALID_ARG (a device-side cu_seqlens check failed),
+ * GDN_ERR_TIMEOUT (a bounded wait ran out) or GDN_ERR_CUDA.
+ */
+GDN_API gdn_status_t gdn_check_device_status(void* stream);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+GDN_API int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

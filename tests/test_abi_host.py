@@ -1,0 +1,156 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/gdn.h declares, and rejects bad arguments before
+touching a device."""
+import ctypes
+import json
+import os
+import re
+import subprocess
+
+import pytest
+
+import gated_deltanet_linear_silu_b200 as gdn
+from gated_deltanet_linear_silu_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gdn.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"GDN_API\s+[\w\s\*]+?\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ["gdn_conv_silu", "gdn_prefill", "gdn_prefill_workspace_size",
+                     "gdn_decode_step", "gdn_status_string", "gdn_check_device_status"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", gdn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)$", out, re.M))
+    missing = [s for s in declared_symbols() if s not in exported]
+    assert not missing, missing
+    for s in declared_symbols():
+        assert hasattr(L, s)
+    # internal symbols stay hidden
+    assert all(s.startswith("gdn_") for s in exported)
+
+
+def test_status_strings(L):
+    for code, name in gdn.STATUS.items():
+        assert L.gdn_status_string(code).decode() == name
+    assert L.gdn_status_string(99).decode() == "GDN_ERR_UNKNOWN"
+    assert L.gdn_version() >= 100
+
+
+def test_workspace_size_is_aligned_and_grows(L):
+    a = L.gdn_prefill_workspace_size(1, 10, 16, 128, 128, 64)
+    b = L.gdn_prefill_workspace_size(10000, 10, 16, 128, 128, 64)
+    assert a > 0 and a % 256 == 0 and b % 256 == 0 and b > a
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails first
+
+
+def _prefill(L, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, g=FAKE, beta=FAKE, cu=FAKE, cu_host=None, N=1,
+                T=64, H=2, dk=128, dv=128, scale=1.0, l2=1, eps=1e-6, chunk=64, h0=None, hT=None,
+                o=FAKE, ws=FAKE, ws_bytes=1 << 20, algo=0, stream=None)
+    args.update(kw)
+    return L.gdn_prefill(*args.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=7), 1), (dict(N=-1), 1), (dict(H=0), 1), (dict(N=0, T=5), 1),
+    (dict(dk=80 + 1), 2), (dict(dv=144), 2), (dict(chunk=48), 2), (dict(algo=9), 1),
+    (dict(q=None), 1), (dict(o=ctypes.c_void_p((1 << 20) + 4)), 1), (dict(cu=None), 1),
+    (dict(ws=None), 3), (dict(ws_bytes=16), 3), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), 3),
+    (dict(eps=float("nan")), 1),
+])
+def test_prefill_rejects_bad_arguments(L, kw, expect):
+    assert _prefill(L, **kw) == expect
+
+
+def test_prefill_host_seqlens_checked(L):
+    bad = [(0, 30, 20), (1, 64, 64), (0, 10, 70)]  # decreasing / not starting at 0 / != T
+    for cu in bad:
+        arr = (ctypes.c_int32 * 3)(*cu)
+        assert _prefill(L, N=2, cu_host=ctypes.cast(arr, ctypes.c_void_p)) == 1
+
+
+def test_prefill_empty_batch_is_noop(L):
+    assert _prefill(L, N=0, T=0, q=None, k=None, v=None, o=None, cu=None) == 0
+
+
+def _conv(L, **kw):
+    args = dict(x=FAKE, dt=1, w=FAKE, cu=FAKE, N=1, T=16, C=6144, K=4, si=None, so=None, l2=1,
+                nqk=4096, hd=128, eps=1e-6, y=ctypes.c_void_p(1 << 21), stream=None)
+    args.update(kw)
+    return L.gdn_conv_silu(*args.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=3), 1), (dict(K=5), 2), (dict(K=0), 1), (dict(C=6145), 2), (dict(hd=96), 2),
+    (dict(nqk=100), 1), (dict(nqk=8192), 1), (dict(y=FAKE), 1), (dict(x=None), 1),
+    (dict(N=0, T=3), 1),
+])
+def test_conv_rejects_bad_arguments(L, kw, expect):
+    assert _conv(L, **kw) == expect
+
+
+def _decode(L, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, g=FAKE, beta=FAKE, state=FAKE, N=4, H=2, dk=128,
+                dv=128, scale=1.0, l2=1, eps=1e-6, o=FAKE, stream=None)
+    args.update(kw)
+    return L.gdn_decode_step(*args.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=2), 1), (dict(dk=8), 2), (dict(dv=130), 2), (dict(state=None), 1),
+    (dict(state=ctypes.c_void_p((1 << 20) + 8)), 1), (dict(H=-1), 1),
+])
+def test_decode_rejects_bad_arguments(L, kw, expect):
+    assert _decode(L, **kw) == expect
+
+
+def test_decode_empty_batch_is_noop(L):
+    assert _decode(L, N=0, q=None, k=None, v=None, state=None, o=None) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(gdn, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        gdn.lib()
+
+
+def test_sizing_helpers_match_printed_figures():
+    d = json.load(open(os.path.join(ROOT, "tests", "golden", "pages_sizing.json")))
+    for c in d["cases"]:
+        b = gdn.state_bytes(c["layers"], c["heads"], c["dk"], c["dv"], c["elem_bytes"])
+        mb = b / (1e6 if c["mb_is_1e6"] else 2 ** 20)
+        assert abs(mb - c["printed_mb"]) <= 0.05 * c["printed_mb"], (c["source"], mb)
+    cd = d["conv_dim"]
+    assert gdn.conv_channels(cd["key_heads"], cd["key_head_dim"], cd["value_heads"],
+                             cd["value_head_dim"]) == cd["conv_dim"]
+
+
+def test_product_path_does_not_import_oracle():
+    """The binding and build script never reach the oracle."""
+    pkg = os.path.join(ROOT, "gated_deltanet_linear_silu_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "gdn_oracle" not in text, f

@@ -1,0 +1,282 @@
+"""GPU parity: the CUDA path against the CPU oracle on the same seeded bytes,
+element by element at sizes the oracle finishes in seconds (several chunks,
+ragged tails, empty sequences), and on sampled (sequence, head) units at the
+full workload sizes. Tolerances (max-abs-normalised error): 1e-4 for fp32
+inputs, 2e-2 for bf16 inputs with fp32 accumulation."""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+import gated_deltanet_linear_silu_b200 as gdn
+import gdn_inputs as gi
+import oracle
+from gpu_util import (DEV, TOL_BF16, TOL_F32, dev_tensor, err, host, oracle_unit, prefill_gpu,
+                      prefill_oracle, tol)
+
+ALGOS = ["auto", "simt"]
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(DEV)
+
+
+# ----------------------------------------------------------------------------
+# prefill
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("chunk", [64, 32, 16])
+def test_tiny_fp32_workload(chunk):
+    P = gi.tiny_fp32()
+    o, hT = prefill_gpu(P, chunk=chunk)
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_F32
+    assert err(hT, h_ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_bf16_ragged_with_state(algo):
+    P = gi.random_prefill(1, [1, 63, 64, 65, 0, 200, 130, 3], H=3, dk=128, dv=128, with_h0=True)
+    o, hT = prefill_gpu(P, algo=algo)
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_BF16
+    assert err(hT, h_ref) <= TOL_BF16
+    n_empty = 4
+    assert np.array_equal(hT[n_empty], P.h0[n_empty])  # empty sequence passes its state through
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (64, 128), (128, 64), (32, 96), (48, 80), (128, 128)])
+def test_prefill_fp32_shapes(dk, dv):
+    P = gi.random_prefill(2, [70, 5, 129], H=2, dk=dk, dv=dv, dtype="f32", with_h0=True, chunk=32,
+                          scale=0.5)
+    o, hT = prefill_gpu(P)
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_F32
+    assert err(hT, h_ref) <= TOL_F32
+
+
+def test_prefill_without_l2norm_and_strong_decay():
+    P = gi.random_prefill(3, [150, 64], H=2, dk=64, dv=64, dtype="f32", g_scale=10.0,
+                          qk_l2norm=False)
+    P.q = (P.q / np.linalg.norm(P.q, axis=-1, keepdims=True)).astype(np.float32)
+    P.k = (P.k / np.linalg.norm(P.k, axis=-1, keepdims=True)).astype(np.float32)
+    o, hT = prefill_gpu(P)
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_F32 and err(hT, h_ref) <= TOL_F32
+
+
+def test_chunk_sizes_agree():
+    P = gi.random_prefill(4, [100, 37], H=2, dk=32, dv=32, dtype="f32", with_h0=True)
+    outs = [prefill_gpu(P, chunk=c) for c in (16, 32, 64)]
+    for o, hT in outs[1:]:
+        assert err(o, outs[0][0]) <= TOL_F32 and err(hT, outs[0][1]) <= TOL_F32
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_split_and_resume_equals_one_call(algo):
+    T, m = 300, 117
+    P = gi.random_prefill(5, [T], H=2, dk=128, dv=128, with_h0=True)
+    o_all, h_all = prefill_gpu(P, algo=algo)
+    A = gi.random_prefill(5, [T], H=2, dk=128, dv=128, with_h0=True)
+    for name in ("q", "k", "v", "g", "beta"):
+        setattr(A, name, getattr(P, name)[:m])
+    A.cu_seqlens = np.array([0, m], np.int32)
+    o1, h1 = prefill_gpu(A, algo=algo)
+    B = gi.random_prefill(5, [T], H=2, dk=128, dv=128)
+    for name in ("q", "k", "v", "g", "beta"):
+        setattr(B, name, getattr(P, name)[m:])
+    B.cu_seqlens = np.array([0, T - m], np.int32)
+    o2, h2 = prefill_gpu(B, algo=algo, h0=h1)
+    assert err(np.concatenate([o1, o2]), o_all) <= 1e-3
+    assert err(h2, h_all) <= 1e-3
+
+
+def test_varlen_packing_equals_separate_calls():
+    P = gi.random_prefill(6, [33, 0, 97, 64], H=2, dk=64, dv=64, dtype="f32", with_h0=True)
+    o, hT = prefill_gpu(P)
+    for n in range(P.N):
+        a, b = P.cu_seqlens[n], P.cu_seqlens[n + 1]
+        Q = gi.random_prefill(6, [b - a], H=2, dk=64, dv=64, dtype="f32")
+        for name in ("q", "k", "v", "g", "beta"):
+            setattr(Q, name, getattr(P, name)[a:b])
+        Q.h0 = P.h0[n:n + 1]
+        on, hn = prefill_gpu(Q)
+        if b > a:
+            assert err(o[a:b], on) <= 1e-6
+        assert err(hT[n:n + 1], hn) <= 1e-6
+
+
+def test_decode_steps_equal_prefill():
+    T = 40
+    P = gi.random_prefill(7, [T, T], H=2, dk=64, dv=32, dtype="f32", with_h0=True)
+    o_p, h_p = prefill_gpu(P)
+    state = dev_tensor(P.h0, "f32").clone()
+    idx = np.array([0, T])
+    for t in range(T):
+        rows = idx + t
+        args = [dev_tensor(getattr(P, nm)[rows], "f32") for nm in ("q", "k", "v", "g", "beta")]
+        o_t = gdn.decode_step(*args, state, scale=P.scale)
+        assert err(host(o_t), o_p[rows]) <= TOL_F32
+    assert err(host(state), h_p) <= TOL_F32
+
+
+# ----------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind,dk,dv", [("f32", 16, 16), ("f32", 128, 128), ("bf16", 128, 128),
+                                        ("f32", 48, 80), ("bf16", 64, 128)])
+def test_decode_step_matches_oracle(kind, dk, dv):
+    r = np.random.default_rng(8)
+    N, H = 5, 3
+    q, k = r.normal(size=(N, H, dk)).astype(np.float32), r.normal(size=(N, H, dk)).astype(np.float32)
+    v = r.normal(size=(N, H, dv)).astype(np.float32)
+    if kind == "bf16":
+        q, k, v = gi.to_bf16_bits(q), gi.to_bf16_bits(k), gi.to_bf16_bits(v)
+    g = -np.abs(r.normal(size=(N, H))).astype(np.float32)
+    beta = r.uniform(size=(N, H)).astype(np.float32)
+    s0 = r.normal(0, 0.1, size=(N, H, dk, dv)).astype(np.float32)
+    state = dev_tensor(s0, "f32")
+    o = gdn.decode_step(dev_tensor(q, kind), dev_tensor(k, kind), dev_tensor(v, kind),
+                        dev_tensor(g, "f32"), dev_tensor(beta, "f32"), state, scale=0.9)
+    o_ref, s_ref = oracle.recurrence(q, k, v, g, beta, np.arange(N + 1), dtype=kind, h0=s0,
+                                     scale=0.9)
+    assert err(host(o), o_ref) <= tol(kind)
+    assert err(host(state), s_ref) <= TOL_F32  # the state never passes through bf16
+
+
+def test_decode_workload_full_100_steps():
+    """256 sequences x 16 heads, d=128, 100 in-place steps; every output of
+    every step and the final state against the oracle's own trajectory."""
+    N, H, d = 256, 16, 128
+    s0 = gi.decode_state(N, H, d)
+    state = dev_tensor(s0, "f32")
+    ref_state = s0.astype(np.float64)
+    worst_o = 0.0
+    for step in range(100):
+        D = gi.decode_step(step, N, H, d)
+        o = gdn.decode_step(dev_tensor(D.q, "bf16"), dev_tensor(D.k, "bf16"), dev_tensor(D.v, "bf16"),
+                            dev_tensor(D.g, "f32"), dev_tensor(D.beta, "f32"), state)
+        o_ref, ref_state = oracle.recurrence(D.q, D.k, D.v, D.g, D.beta, np.arange(N + 1),
+                                             dtype="bf16", h0=ref_state)
+        worst_o = max(worst_o, err(host(o), o_ref))
+    assert worst_o <= TOL_BF16
+    assert err(host(state), ref_state) <= TOL_BF16
+
+
+# ----------------------------------------------------------------------------
+# conv
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+@pytest.mark.parametrize("with_state", [False, True])
+@pytest.mark.parametrize("K", [4, 3, 1])
+def test_conv_matches_oracle(kind, with_state, K):
+    lens = [5, 1, 0, 2, 40, 33, 70]
+    H, d = 2, 128
+    C = 3 * H * d
+    x, w, cu, st = gi.random_mixed(9, lens, C, K=K, dtype=kind, with_state=with_state)
+    y, st_out = gdn.conv_silu(dev_tensor(x, kind), dev_tensor(w, kind),
+                              torch.from_numpy(cu).to(DEV),
+                              conv_state=None if st is None else dev_tensor(st, kind),
+                              n_qk_channels=2 * H * d, head_dim=d)
+    gdn.check_device_status(DEV)
+    y_ref, st_ref = oracle.conv_silu(x, w, cu, dtype=kind, state_in=st, qk_l2norm=True,
+                                     n_qk=2 * H * d, head_dim=d)
+    assert err(host(y), y_ref) <= (1e-2 if kind == "bf16" else 1e-5)
+    if K > 1:
+        assert np.array_equal(host(st_out), st_ref.astype(np.float32))  # a pure copy: bit exact
+
+
+def test_conv_state_in_place_and_continuation():
+    C, K = 384, 4
+    x, w, cu, st = gi.random_mixed(10, [50], C, K=K, dtype="f32", with_state=True)
+    st_d = dev_tensor(st, "f32")
+    xd, wd = dev_tensor(x, "f32"), dev_tensor(w, "f32")
+    y_all, _ = gdn.conv_silu(xd, wd, torch.tensor([0, 50], dtype=torch.int32, device=DEV),
+                             conv_state=st_d.clone(), qk_l2norm=False)
+    m = 23
+    s = st_d.clone()
+    y1, _ = gdn.conv_silu(xd[:m].contiguous(), wd, torch.tensor([0, m], dtype=torch.int32, device=DEV),
+                          conv_state=s, conv_state_out=s, qk_l2norm=False)
+    y2, _ = gdn.conv_silu(xd[m:].contiguous(), wd, torch.tensor([0, 50 - m], dtype=torch.int32,
+                                                                device=DEV),
+                          conv_state=s, conv_state_out=s, qk_l2norm=False)
+    assert err(host(torch.cat([y1, y2])), host(y_all)) <= 1e-6
+    assert np.array_equal(host(s)[0], x[-3:].T)
+
+
+# ----------------------------------------------------------------------------
+# full-size workloads
+# ----------------------------------------------------------------------------
+
+def test_layer_0p8b_conv_then_prefill():
+    """One 0.8B-shaped layer: T=4096, 16 heads of 128, conv + SiLU + L2 norm,
+    chunked prefill (chunk 64), fp32 final state; every element checked."""
+    Lw = gi.layer_0p8b()
+    T, H, d = Lw.T_tot, Lw.H, Lw.dk
+    cu = torch.from_numpy(Lw.cu_seqlens).to(DEV)
+    y, _ = gdn.conv_silu(dev_tensor(Lw.mixed_qkv, "bf16"), dev_tensor(Lw.conv_w, "bf16"), cu,
+                         n_qk_channels=2 * H * d, head_dim=d)
+    qkv = y.view(T, 3, H, d)
+    q, k, v = (qkv[:, i].contiguous() for i in range(3))
+    o, hT = gdn.prefill(q, k, v, dev_tensor(Lw.g, "f32"), dev_tensor(Lw.beta, "f32"), cu,
+                        qk_l2norm=False)
+    gdn.check_device_status(DEV)
+    y_ref, _ = oracle.conv_silu(Lw.mixed_qkv, Lw.conv_w, Lw.cu_seqlens, dtype="bf16",
+                                qk_l2norm=True, n_qk=2 * H * d, head_dim=d)
+    assert err(host(y), y_ref) <= 1e-2
+    yr = y_ref.reshape(T, 3, H, d)
+    o_ref, h_ref = oracle.recurrence(yr[:, 0], yr[:, 1], yr[:, 2], Lw.g, Lw.beta, Lw.cu_seqlens,
+                                     dtype="f64", qk_l2norm=False)
+    assert err(host(o), o_ref) <= TOL_BF16
+    assert err(host(hT), h_ref) <= TOL_BF16
+
+
+def _sampled_check(P, units):
+    o, hT = prefill_gpu(P)
+    assert np.isfinite(o).all() and np.isfinite(hT).all()
+    worst = 0.0
+    for n, h in units:
+        a, b = int(P.cu_seqlens[n]), int(P.cu_seqlens[n + 1])
+        o_ref, h_ref = oracle_unit(P, n, h)
+        worst = max(worst, err(o[a:b, h], o_ref), err(hT[n, h], h_ref))
+    assert worst <= TOL_BF16, worst
+
+
+def test_long_prefill_full_size_sampled():
+    P = gi.long_prefill()
+    _sampled_check(P, [(0, 0), (3, 7), (7, 15)])
+
+
+def test_varlen_full_size_sampled():
+    P = gi.varlen()
+    lens = np.diff(P.cu_seqlens)
+    longest, shortest = int(np.argmax(lens)), int(np.argmin(lens))
+    _sampled_check(P, [(longest, 0), (shortest, 5), (17, 11)])
+
+
+# ----------------------------------------------------------------------------
+# device-side argument checks
+# ----------------------------------------------------------------------------
+
+def test_bad_device_seqlens_reported_not_faulted():
+    P = gi.random_prefill(11, [64, 64], H=1, dk=32, dv=32, dtype="f32")
+    bad = torch.tensor([0, 100, 64], dtype=torch.int32, device=DEV)  # decreasing, no host copy
+    q, k, v = (dev_tensor(a, "f32") for a in (P.q, P.k, P.v))
+    g, beta = dev_tensor(P.g, "f32"), dev_tensor(P.beta, "f32")
+    gdn.prefill(q, k, v, g, beta, bad)
+    with pytest.raises(gdn.GDNError, match="INVALID_ARG"):
+        gdn.check_device_status(DEV)
+    x = torch.zeros((128, 384), dtype=torch.float32, device=DEV)
+    gdn.conv_silu(x, torch.zeros((384, 4), device=DEV), bad, qk_l2norm=False)
+    with pytest.raises(gdn.GDNError, match="INVALID_ARG"):
+        gdn.check_device_status(DEV)
+    # the context is still usable
+    o, hT = prefill_gpu(P)
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_F32
