@@ -63,6 +63,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_check_device_status.argtypes = [vp]
         L.gdn_check_device_status.restype = i32
+        L.gdn_prefill_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                          f32, i32, f32, i32, vp, vp, vp, i32, vp]
+        L.gdn_prefill_noalloc.restype = i32
+        L.gdn_prefill_noalloc_max_scratch.argtypes = []
+        L.gdn_prefill_noalloc_max_scratch.restype = sz
         L.gdn_prefill_selected_algo.argtypes = [i32, i32, i32, i32, i32]
         L.gdn_prefill_selected_algo.restype = i32
         L.gdn_version.argtypes = []
@@ -158,6 +163,25 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
         _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill")
     return o, hT
+
+
+def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                    beta: torch.Tensor, cu_seqlens: torch.Tensor, *,
+                    initial_state: Optional[torch.Tensor] = None, final_state: torch.Tensor,
+                    out: torch.Tensor, scale: float = 1.0, qk_l2norm: bool = True,
+                    eps: float = 1e-6, chunk: int = 64, algo: str = "auto") -> None:
+    """gdn_prefill_noalloc: prefill with the library's fixed scratch array
+    instead of a workspace; the caller passes every output buffer, so nothing
+    is allocated."""
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    _cuda(q, k, v, g, beta, cu_seqlens, initial_state, final_state, out)
+    st = lib().gdn_prefill_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens), None,
+        N, T, H, dk, dv, float(scale), int(qk_l2norm), float(eps), int(chunk),
+        _ptr(initial_state), _ptr(final_state), _ptr(out), ALGOS[algo], _stream(q.device))
+    _check(st, "gdn_prefill_noalloc")
 
 
 def selected_algo(dtype: str, dk: int, dv: int, chunk: int = 64, algo: str = "auto") -> str:

@@ -149,6 +149,38 @@ GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gd
                          void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream);
 
 /*
+ * gdn_prefill without a caller-supplied workspace. There is no counterpart of
+ * this call in the paper: it exists for callers that cannot allocate device
+ * memory where they run the mixer -- a runtime whose memory planner reserved
+ * the whole device arena at start-up, or a serving loop that must not call
+ * cudaMalloc/cudaFree (which can synchronise the device) once it is running.
+ *
+ * Arguments and results are those of gdn_prefill minus workspace/ws_bytes.
+ * The scratch gdn_prefill keeps in the workspace lives instead in one fixed
+ * array in device global memory, gdn_prefill_noalloc_max_scratch() bytes
+ * (64 KiB: schedules of up to 16320 sequences), which every GPU that loads the
+ * library holds until the process exits. Problems that need more scratch than
+ * that return GDN_ERR_WORKSPACE before anything is launched. The call itself
+ * allocates nothing.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls on a device share the array and it keeps the last call's
+ * contents (each call resets what must start at zero): calls whose kernels
+ * overlap on the GPU race on it, so order them on one stream.
+ */
+GDN_API gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v,
+                                         gdn_dtype_t dtype, const float* g, const float* beta,
+                                         const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
+                                         int N, int64_t T_tot, int H, int dk, int dv,
+                                         float scale, int qk_l2norm, float eps, int chunk,
+                                         const float* h0, float* hT, void* o, gdn_algo_t algo,
+                                         void* stream);
+
+/* Size in bytes of the fixed scratch array behind gdn_prefill_noalloc. */
+GDN_API size_t gdn_prefill_noalloc_max_scratch(void);
+
+/*
  * The prefill kernel gdn_prefill would run for these arguments:
  * GDN_ALGO_SIMT or GDN_ALGO_TENSOR, or -1 if the combination is unsupported.
  */
