@@ -15,7 +15,7 @@ import oracle
 from gpu_util import (DEV, TOL_BF16, TOL_F32, dev_tensor, err, host, oracle_unit, prefill_gpu,
                       prefill_oracle, tol)
 
-ALGOS = ["auto", "simt"]
+ALGOS = ["auto", "simt", "tensor"]
 
 
 @pytest.fixture(autouse=True, scope="module")
@@ -91,8 +91,10 @@ def test_split_and_resume_equals_one_call(algo):
         setattr(B, name, getattr(P, name)[m:])
     B.cu_seqlens = np.array([0, T - m], np.int32)
     o2, h2 = prefill_gpu(B, algo=algo, h0=h1)
-    assert err(np.concatenate([o1, o2]), o_all) <= 1e-3
-    assert err(h2, h_all) <= 1e-3
+    # Moving the chunk boundary changes which values the tensor-core path
+    # rounds to bf16 (2^-9 relative per operand): half the bf16 tolerance.
+    assert err(np.concatenate([o1, o2]), o_all) <= TOL_BF16 / 2
+    assert err(h2, h_all) <= TOL_BF16 / 2
 
 
 def test_varlen_packing_equals_separate_calls():
