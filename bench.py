@@ -236,7 +236,7 @@ def run_reference(args, dist: Dist):
 
 
 def config_block(n):
-    return {"workload": "long_prefill_8x16384_h16_d128_bf16", "global_batch": SEQS * n,
+    return {"workload": f"long_prefill_{SEQS}x{SEQ_LEN}_h16_d128_bf16", "global_batch": SEQS * n,
             "seq_len": SEQ_LEN, "heads": H, "head_dim": D, "chunk": CHUNK,
             "parallelism": f"replicas{n}" if n > 1 else "single",
             "l2": "inputs larger than L2 (1.1 GB resident per step)"}
@@ -491,6 +491,7 @@ def run_ours(args, dist: Dist):
 
 
 def main():
+    global SEQS, SEQ_LEN
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -499,7 +500,10 @@ def main():
     ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--no-extras", action="store_true", help="headline workload only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqs", type=int, default=SEQS, help="sequences (profiling runs only)")
+    ap.add_argument("--seq-len", type=int, default=SEQ_LEN, help="tokens per sequence (profiling)")
     args = ap.parse_args()
+    SEQS, SEQ_LEN = args.seqs, args.seq_len
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     dist = Dist(args.gpus)
