@@ -163,6 +163,7 @@ int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_
     a.dk = dk;
     a.dv = dv;
     a.chunk = chunk;
+    a.T_tot = 1;
     const bool tc_ok = gdn::prefill_tc_supported(a);
     if (algo == GDN_ALGO_TENSOR) return tc_ok ? GDN_ALGO_TENSOR : -1;
     if (algo == GDN_ALGO_SIMT || !tc_ok)

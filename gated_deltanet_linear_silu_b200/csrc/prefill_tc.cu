@@ -61,8 +61,10 @@ constexpr uint32_t kOffUT = kOffWT + 16384;       // U^T bf16 [128 dv][64 tok] K
 constexpr uint32_t kOffP = kOffUT + 16384;        // P bf16 [64 r][64 j] K-major
 constexpr uint32_t kOffT1 = kOffP + 8192;         // T1^T bf16 [64 m][64 r] MN-major
 constexpr uint32_t kOffT2 = kOffT1 + 8192;        // T2^T bf16
-constexpr uint32_t kOffA = kOffT2 + 8192;         // A fp32 [64][64]
-constexpr uint32_t kOffVec = kOffA + 16384;       // gamma, beta, rq, rk: 4 x 64 fp32
+constexpr int kLdA = 68;                          // padded fp32 row stride (272 B)
+constexpr uint32_t kOffA = kOffT2 + 8192;         // A fp32 [64][kLdA] (later also Y)
+constexpr uint32_t kOffTf = kOffA + 64 * kLdA * 4;  // T fp32 [64][kLdA]
+constexpr uint32_t kOffVec = kOffTf + 64 * kLdA * 4;  // gamma, beta, rq, rk: 4 x 64 fp32
 constexpr uint32_t kOffBar = kOffVec + 1024;      // mbarriers
 constexpr uint32_t kOffMisc = kOffBar + 64;       // tmem base, abort flag, scan carry
 constexpr uint32_t kSmemBytes = kOffMisc + 64;
@@ -92,7 +94,7 @@ __device__ __forceinline__ void unpack_bf16(uint32_t w, float& lo, float& hi) {
 }
 
 // Write 64 fp32 values as one 128-byte bf16 row of a 128B-swizzled tile.
-__device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float* v) {
+__device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float (&v)[64]) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         uint4 u;
@@ -105,7 +107,8 @@ __device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float*
 }
 
 // Same, with every value multiplied by f.
-__device__ __forceinline__ void store_row64_scaled(uint8_t* tile, int row, const float* v, float f) {
+__device__ __forceinline__ void store_row64_scaled(uint8_t* tile, int row, const float (&v)[64],
+                                                   float f) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         uint4 u;
@@ -121,7 +124,7 @@ __device__ __forceinline__ void store_row64_scaled(uint8_t* tile, int row, const
 __device__ __forceinline__ void scale_row(uint8_t* tile, int row, float f) {
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        uint4* p = reinterpret_cast<uint4*>(tile + row * 128 + c * 16);
+        uint4* p = reinterpret_cast<uint4*>(tile + sw128_off(row, c));  // spreads banks
         uint4 u = *p;
         float a, b;
         unpack_bf16(u.x, a, b); u.x = pack_bf16(a * f, b * f);
@@ -137,7 +140,7 @@ __device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
     float s = 0.f;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const uint4 u = *reinterpret_cast<const uint4*>(tile + row * 128 + c * 16);
+        const uint4 u = *reinterpret_cast<const uint4*>(tile + sw128_off(row, c));
         float a, b;
         unpack_bf16(u.x, a, b); s = fmaf(a, a, s); s = fmaf(b, b, s);
         unpack_bf16(u.y, a, b); s = fmaf(a, a, s); s = fmaf(b, b, s);
@@ -194,7 +197,6 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     const int H = a.H;
     const int64_t total = (int64_t)a.N * H;
 
-    uint8_t* stage[2] = {sm, sm + kStageBytes};
     uint8_t* sSA = sm + kOffSA;
     uint8_t* sWT = sm + kOffWT;
     uint8_t* sUT = sm + kOffUT;
@@ -202,6 +204,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     uint8_t* sT1 = sm + kOffT1;
     uint8_t* sT2 = sm + kOffT2;
     float* sA = reinterpret_cast<float*>(sm + kOffA);
+    float* sT = reinterpret_cast<float*>(sm + kOffTf);
     float* gam = reinterpret_cast<float*>(sm + kOffVec);
     float* bet = gam + 64;
     float* rq = gam + 128;
@@ -229,10 +232,11 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     const uint32_t tmem = *tmem_base_p;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lane quarter
 
-    uint32_t full_phase[2] = {0, 0};
+    uint32_t full_phase = 0;  // bit s: expected parity of full[s]
     uint32_t mma_phase = 0;
     int cur = 0;              // stage of the chunk being processed
-    bool inflight[2] = {false, false};
+    uint32_t inflight = 0;    // bit s: TMA issued into stage s, not yet consumed
+    auto stage = [&](int i) { return sm + i * kStageBytes; };
     bool aborted = false;
 
     // Bounded wait by every thread; all threads agree on the outcome.
@@ -258,11 +262,19 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         const int64_t base = ((int64_t)U.n * H + U.h) * kD * kD;
         for (int i = tid; i < kD * kD; i += kThreads) a.hT[base + i] = a.h0 ? a.h0[base + i] : 0.f;
     }
-    if (tid == 0 && u < total) {
+    // Gates of the next chunk, prefetched one chunk ahead (threads 0..63, row = tid).
+    float g_next = 0.f, b_next = 0.f;
+    if (u < total) {
         Unit U;
         load_unit(a, u, U);
-        issue_tiles(stage[0], &full[0], &map_q, &map_k, &map_v, U.h, U.start);
-        inflight[0] = true;
+        if (tid == 0) {
+            issue_tiles(stage(0), &full[0], &map_q, &map_k, &map_v, U.h, U.start);
+            inflight |= 1u;
+        }
+        if (tid < 64 && U.start + tid < U.end) {
+            g_next = a.g[(U.start + tid) * H + U.h];
+            b_next = a.beta[(U.start + tid) * H + U.h];
+        }
     }
 
     while (u < total && !aborted) {
@@ -298,34 +310,48 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         for (int64_t c0 = U.start; c0 < U.end && !aborted; c0 += kC) {
             const int L = (U.end - c0 < kC) ? (int)(U.end - c0) : kC;
             const bool last = c0 + kC >= U.end;
-            uint8_t* st = stage[cur];
+            uint8_t* st = stage(cur);
 
-            // ---- prefetch the next chunk (this unit or the next one) into the other stage
-            if (tid == 0) {
-                int64_t nu = u, nc0 = c0 + kC;
+            // ---- prefetch the next chunk (this unit or the next one): tiles into
+            // the other stage by TMA, gates into registers
+            const float g_cur = g_next, b_cur = b_next;
+            {
+                int64_t nu = u, nc0 = c0 + kC, nend = U.end;
+                int nh = U.h;
                 if (last) {
                     nu = next_nonempty(a, u + gridDim.x, total);
-                    Unit N2;
-                    if (nu < total) { load_unit(a, nu, N2); nc0 = N2.start; }
+                    if (nu < total) {
+                        Unit N2;
+                        load_unit(a, nu, N2);
+                        nc0 = N2.start;
+                        nend = N2.end;
+                        nh = N2.h;
+                    }
                 }
                 if (nu < total) {
-                    Unit N2;
-                    load_unit(a, nu, N2);
-                    issue_tiles(stage[cur ^ 1], &full[cur ^ 1], &map_q, &map_k, &map_v, N2.h, nc0);
-                    inflight[cur ^ 1] = true;
+                    if (tid == 0) {
+                        issue_tiles(stage(cur ^ 1), &full[cur ^ 1], &map_q, &map_k, &map_v, nh, nc0);
+                        inflight |= 1u << (cur ^ 1);
+                    }
+                    g_next = 0.f;
+                    b_next = 0.f;
+                    if (tid < 64 && nc0 + tid < nend) {
+                        g_next = a.g[(nc0 + tid) * H + nh];
+                        b_next = a.beta[(nc0 + tid) * H + nh];
+                    }
                 }
             }
-            if (!wait_all(&full[cur], full_phase[cur])) { aborted = true; break; }
-            full_phase[cur] ^= 1;
-            inflight[cur] = false;
+            if (!wait_all(&full[cur], (full_phase >> cur) & 1u)) { aborted = true; break; }
+            full_phase ^= 1u << cur;
+            inflight &= ~(1u << cur);
 
             // ---- per-row scalars: gates, cumulative decay, L2 norms
             if (tid < 64) {
                 const int r = tid;
                 float g = 0.f, b = 0.f, fq = 0.f;
                 if (r < L) {
-                    g = a.g[(c0 + r) * H + U.h];
-                    b = a.beta[(c0 + r) * H + U.h];
+                    g = g_cur;
+                    b = b_cur;
                     const float ss = row_sumsq(st + kQb0, r) + row_sumsq(st + kQb1, r);
                     fq = (a.qk_l2norm ? 1.f / sqrtf(ss + a.eps) : 1.f) * a.scale;
                 }
@@ -384,7 +410,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 } else {
                     const int r = tid - 64;
                     const float gr = gam[r], fr = bet[r] * rk[r];
-                    float4* Ar = reinterpret_cast<float4*>(sA + r * 64);
+                    float4* Ar = reinterpret_cast<float4*>(sA + r * kLdA);
 #pragma unroll
                     for (int q4 = 0; q4 < 16; ++q4) {
                         float4 o;
@@ -401,33 +427,84 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             tc_fence_before();
             __syncthreads();
 
-            // ---- solve T = (I + A)^-1 (column j per thread, tid < 64); Q -> Q~ (tid >= 64)
+            // ---- solve T = (I + A)^-1 in 32x32 blocks. Diagonal blocks by forward
+            // substitution (one column per thread, tid < 64) while tid >= 64 turn
+            // Q into Q~; then T_10 = -T_11 (A_10 T_00).
             if (tid < 64) {
-                const int j = tid;
-                float x[64];
+                const int b = tid >> 5, c = tid & 31, o = 32 * b;
+                float x[32];
 #pragma unroll
-                for (int r = 0; r < 64; ++r) {
-                    float s0 = (r == j) ? 1.f : 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-                    const float4* Ar = reinterpret_cast<const float4*>(sA + r * 64);
+                for (int r = 0; r < 32; ++r) {
+                    float s0 = (r == c) ? 1.f : 0.f, s1 = 0.f;
+                    const float* Ar = sA + (o + r) * kLdA + o;
 #pragma unroll
                     for (int m4 = 0; m4 < r / 4; ++m4) {
-                        const float4 av = Ar[m4];
+                        const float4 av = *reinterpret_cast<const float4*>(Ar + 4 * m4);
                         s0 = fmaf(-av.x, x[4 * m4 + 0], s0);
                         s1 = fmaf(-av.y, x[4 * m4 + 1], s1);
-                        s2 = fmaf(-av.z, x[4 * m4 + 2], s2);
-                        s3 = fmaf(-av.w, x[4 * m4 + 3], s3);
+                        s0 = fmaf(-av.z, x[4 * m4 + 2], s0);
+                        s1 = fmaf(-av.w, x[4 * m4 + 3], s1);
                     }
 #pragma unroll
-                    for (int m = (r / 4) * 4; m < r; ++m) s0 = fmaf(-sA[r * 64 + m], x[m], s0);
-                    x[r] = (s0 + s1) + (s2 + s3);
+                    for (int m = (r / 4) * 4; m < r; ++m) s0 = fmaf(-Ar[m], x[m], s0);
+                    x[r] = s0 + s1;
                 }
-                store_row64_scaled(sT1, j, x, bet[j] * expf(gam[j]) * rk[j]);
-                store_row64_scaled(sT2, j, x, bet[j]);
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    sT[(o + r) * kLdA + o + c] = x[r];
+                    if (b == 1) sT[r * kLdA + 32 + c] = 0.f;  // upper-right block of T
+                }
             } else {
                 const int r = tid - 64;
                 const float f = expf(gam[r]) * rq[r];
                 scale_row(st + kQb0, r, f);
                 scale_row(st + kQb1, r, f);
+            }
+            __syncthreads();
+            {
+                // Y = A_10 T_00 : thread -> 2 rows x 4 columns of the 32x32 block
+                const int r0 = 2 * (tid >> 3), c0b = 4 * (tid & 7);
+                float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
+                for (int m = 0; m < 32; ++m) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(sT + m * kLdA + c0b);
+                    const float a0 = sA[(32 + r0) * kLdA + m], a1 = sA[(33 + r0) * kLdA + m];
+                    y[0][0] = fmaf(a0, t4.x, y[0][0]); y[0][1] = fmaf(a0, t4.y, y[0][1]);
+                    y[0][2] = fmaf(a0, t4.z, y[0][2]); y[0][3] = fmaf(a0, t4.w, y[0][3]);
+                    y[1][0] = fmaf(a1, t4.x, y[1][0]); y[1][1] = fmaf(a1, t4.y, y[1][1]);
+                    y[1][2] = fmaf(a1, t4.z, y[1][2]); y[1][3] = fmaf(a1, t4.w, y[1][3]);
+                }
+                __syncthreads();  // everyone done reading A_10
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    *reinterpret_cast<float4*>(sA + (32 + r0 + i) * kLdA + c0b) =
+                        make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+                __syncthreads();
+                // T_10 = -T_11 Y  (Y now in A's lower-left block)
+                float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 8
+                for (int m = 0; m < 32; ++m) {
+                    const float4 y4 = *reinterpret_cast<const float4*>(sA + (32 + m) * kLdA + c0b);
+                    const float t0 = sT[(32 + r0) * kLdA + 32 + m], t1 = sT[(33 + r0) * kLdA + 32 + m];
+                    z[0][0] = fmaf(t0, y4.x, z[0][0]); z[0][1] = fmaf(t0, y4.y, z[0][1]);
+                    z[0][2] = fmaf(t0, y4.z, z[0][2]); z[0][3] = fmaf(t0, y4.w, z[0][3]);
+                    z[1][0] = fmaf(t1, y4.x, z[1][0]); z[1][1] = fmaf(t1, y4.y, z[1][1]);
+                    z[1][2] = fmaf(t1, y4.z, z[1][2]); z[1][3] = fmaf(t1, y4.w, z[1][3]);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    *reinterpret_cast<float4*>(sT + (32 + r0 + i) * kLdA + c0b) =
+                        make_float4(-z[i][0], -z[i][1], -z[i][2], -z[i][3]);
+            }
+            __syncthreads();
+            // T1^T, T2^T rows (row m = column m of T) as bf16 MN-major B operands
+            if (tid < 64) {
+                const int j = tid;
+                float x[64];
+#pragma unroll
+                for (int r = 0; r < 64; ++r) x[r] = sT[r * kLdA + j];
+                store_row64_scaled(sT1, j, x, bet[j] * expf(gam[j]) * rk[j]);
+                store_row64_scaled(sT2, j, x, bet[j]);
             }
             fence_proxy_async();
             tc_fence_before();
@@ -538,7 +615,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     tmem_wait_ld();
                     store_row64(sSA + hh * 16384, j, v);
                     if (last && a.hT) {
-#pragma unroll 8
+#pragma unroll
                         for (int e = 0; e < 64; ++e) a.hT[sbase + (int64_t)(64 * hh + e) * kD + j] = v[e];
                     }
                 }
@@ -560,7 +637,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     // ---- drain TMA copies still in flight (bounded), free TMEM
     if (tid == 0) {
         for (int s = 0; s < 2; ++s)
-            if (inflight[s]) mbar_wait(&full[s], full_phase[s], kWaitNs);
+            if ((inflight >> s) & 1u) mbar_wait(&full[s], (full_phase >> s) & 1u, kWaitNs);
     }
     tc_fence_before();
     __syncthreads();
