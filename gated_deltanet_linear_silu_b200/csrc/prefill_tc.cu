@@ -26,8 +26,9 @@
 // epilogues, so the MMAs read the raw bf16 input tiles that TMA brings in
 // (128-byte swizzle). The solve for T runs on CUDA cores in fp32.
 //
-// This version runs the phases of a chunk in lock-step across one 128-thread
-// CTA per SM (thread t owns TMEM lane t); thread 0 issues TMA and MMAs. The
+// This version runs the phases of a chunk in lock-step across one 256-thread
+// CTA per SM (two warps per TMEM lane quarter, each taking half of the
+// columns); thread 0 issues TMA and MMAs. The
 // next chunk's tiles are prefetched by TMA during the current chunk.
 // Every wait is bounded: on timeout the kernel records GDN timeout status,
 // drains its TMA copies, frees TMEM and returns.
@@ -47,7 +48,7 @@ using namespace tc;
 
 constexpr int kC = 64;          // chunk
 constexpr int kD = 128;         // head dim (dk = dv)
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
 // Shared memory map (bytes from a 1024-aligned base).
@@ -117,6 +118,21 @@ __device__ __forceinline__ void store_row64_scaled(uint8_t* tile, int row, const
         u.z = pack_bf16(v[8 * c + 4] * f, v[8 * c + 5] * f);
         u.w = pack_bf16(v[8 * c + 6] * f, v[8 * c + 7] * f);
         *reinterpret_cast<uint4*>(tile + sw128_off(row, c)) = u;
+    }
+}
+
+// Write 32 fp32 values (times f) as columns [32*half, 32*half + 32) of one
+// 128-byte bf16 row of a swizzled tile.
+__device__ __forceinline__ void store_half_row(uint8_t* tile, int row, int half, const float (&v)[32],
+                                               float f) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 u;
+        u.x = pack_bf16(v[8 * c + 0] * f, v[8 * c + 1] * f);
+        u.y = pack_bf16(v[8 * c + 2] * f, v[8 * c + 3] * f);
+        u.z = pack_bf16(v[8 * c + 4] * f, v[8 * c + 5] * f);
+        u.w = pack_bf16(v[8 * c + 6] * f, v[8 * c + 7] * f);
+        *reinterpret_cast<uint4*>(tile + sw128_off(row, 4 * half + c)) = u;
     }
 }
 
@@ -194,6 +210,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const PrefillArgs& a = P.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // Two warps share each TMEM lane quarter and split the columns in halves.
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = 32 * quarter + lane;  // TMEM lane owned by this thread
     const int H = a.H;
     const int64_t total = (int64_t)a.N * H;
 
@@ -230,7 +249,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_p;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lane quarter
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;  // this warp's TMEM lane quarter
 
     uint32_t full_phase = 0;  // bit s: expected parity of full[s]
     uint32_t mma_phase = 0;
@@ -282,26 +301,21 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         load_unit(a, u, U);
         const int64_t sbase = ((int64_t)U.n * H + U.h) * kD * kD;
 
-        // ---- initial state: R_S (fp32) and S^T (bf16 A operand); thread = dv lane j
+        // ---- initial state: R_S (fp32) and S^T (bf16 A operand). Thread (row j =
+        // dv index, half) owns dk columns [64*half, 64*half + 64).
         {
-            const int j = tid;
-            float v[32];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    v[e] = a.h0 ? a.h0[sbase + (int64_t)(32 * cc + e) * kD + j] : 0.f;
-                tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
-            }
-        }
-        tmem_wait_st();  // then read the state back to build its bf16 copy
-        {
+            const int j = row;
             float v[64];
-            for (int hh = 0; hh < 2; ++hh) {
-                tmem_ld64(tmem + lane_off + kRS + 64 * hh, v);
-                tmem_wait_ld();
-                store_row64(sSA + hh * 16384, tid, v);
-            }
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+                v[e] = a.h0 ? a.h0[sbase + (int64_t)(64 * half + e) * kD + j] : 0.f;
+            float w0[32], w1[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) { w0[e] = v[e]; w1[e] = v[32 + e]; }
+            tmem_st32(tmem + lane_off + kRS + 64 * half, w0);
+            tmem_st32(tmem + lane_off + kRS + 64 * half + 32, w1);
+            store_row64(sSA + half * 16384, j, v);
+            tmem_wait_st();
         }
         fence_proxy_async();
         tc_fence_before();
@@ -365,7 +379,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 bet[r] = b;
                 rq[r] = fq;
                 gam[r] = x;  // warp 1 adds warp 0's total below
-            } else {
+            } else if (tid < 128) {
                 const int r = tid - 64;
                 float fk = 0.f;
                 if (r < L) {
@@ -395,32 +409,40 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             mma_phase ^= 1;
             tc_fence_after();
 
-            // ---- epilogue a: P rows (tid < 64) and A rows (tid >= 64)
+            // ---- epilogue a: P rows (lanes < 64) and A rows (lanes >= 64); each
+            // thread takes 32 of the 64 columns. Branch-free: every element is
+            // computed (exponent clamped at 0 so the masked-out upper triangle
+            // cannot overflow), then selected.
             {
-                float x[64];
-                tmem_ld64(tmem + lane_off + kRA, x);
+                float x[32];
+                tmem_ld32(tmem + lane_off + kRA + 32 * half, x);
                 tmem_wait_ld();
-                if (tid < 64) {
-                    const int r = tid;
+                const int j0 = 32 * half;
+                if (row < 64) {
+                    const int r = row;
                     const float gr = gam[r], fr = rq[r];
 #pragma unroll
-                    for (int j = 0; j < 64; ++j)
-                        x[j] = (j <= r) ? expf(gr - gam[j]) * fr * rk[j] * x[j] : 0.f;
-                    store_row64(sP, r, x);
-                } else {
-                    const int r = tid - 64;
-                    const float gr = gam[r], fr = bet[r] * rk[r];
-                    float4* Ar = reinterpret_cast<float4*>(sA + r * kLdA);
-#pragma unroll
-                    for (int q4 = 0; q4 < 16; ++q4) {
-                        float4 o;
-                        const int j = 4 * q4;
-                        o.x = (j + 0 < r) ? expf(gr - gam[j + 0]) * fr * rk[j + 0] * x[j + 0] : 0.f;
-                        o.y = (j + 1 < r) ? expf(gr - gam[j + 1]) * fr * rk[j + 1] * x[j + 1] : 0.f;
-                        o.z = (j + 2 < r) ? expf(gr - gam[j + 2]) * fr * rk[j + 2] * x[j + 2] : 0.f;
-                        o.w = (j + 3 < r) ? expf(gr - gam[j + 3]) * fr * rk[j + 3] * x[j + 3] : 0.f;
-                        Ar[q4] = o;
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = j0 + e;
+                        const float ex = __expf(fminf(gr - gam[j], 0.f));
+                        const float val = ex * (fr * rk[j]) * x[e];
+                        x[e] = (j <= r) ? val : 0.f;
                     }
+                    store_half_row(sP, r, half, x, 1.f);
+                } else {
+                    const int r = row - 64;
+                    const float gr = gam[r], fr = bet[r] * rk[r];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = j0 + e;
+                        const float ex = __expf(fminf(gr - gam[j], 0.f));
+                        const float val = ex * (fr * rk[j]) * x[e];
+                        x[e] = (j < r) ? val : 0.f;
+                    }
+                    float4* Ar = reinterpret_cast<float4*>(sA + r * kLdA + j0);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        Ar[q4] = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
                 }
             }
             fence_proxy_async();
@@ -428,8 +450,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             __syncthreads();
 
             // ---- solve T = (I + A)^-1 in 32x32 blocks. Diagonal blocks by forward
-            // substitution (one column per thread, tid < 64) while tid >= 64 turn
-            // Q into Q~; then T_10 = -T_11 (A_10 T_00).
+            // substitution (one column per thread, tid < 64) while tid 64..191 turn
+            // Q into Q~; then T_10 = -T_11 (A_10 T_00) on all threads.
             if (tid < 64) {
                 const int b = tid >> 5, c = tid & 31, o = 32 * b;
                 float x[32];
@@ -454,57 +476,47 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     sT[(o + r) * kLdA + o + c] = x[r];
                     if (b == 1) sT[r * kLdA + 32 + c] = 0.f;  // upper-right block of T
                 }
-            } else {
-                const int r = tid - 64;
-                const float f = expf(gam[r]) * rq[r];
-                scale_row(st + kQb0, r, f);
-                scale_row(st + kQb1, r, f);
+            } else if (tid < 192) {
+                const int rr = tid - 64, r = rr & 63;
+                scale_row(st + ((rr >> 6) ? kQb1 : kQb0), r, expf(gam[r]) * rq[r]);
             }
             __syncthreads();
             {
-                // Y = A_10 T_00 : thread -> 2 rows x 4 columns of the 32x32 block
-                const int r0 = 2 * (tid >> 3), c0b = 4 * (tid & 7);
-                float y[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                // Y = A_10 T_00 ; thread -> 2 rows x 2 columns of the 32x32 block
+                const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
+                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
                 for (int m = 0; m < 32; ++m) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(sT + m * kLdA + c0b);
+                    const float2 t2 = *reinterpret_cast<const float2*>(sT + m * kLdA + c0b);
                     const float a0 = sA[(32 + r0) * kLdA + m], a1 = sA[(33 + r0) * kLdA + m];
-                    y[0][0] = fmaf(a0, t4.x, y[0][0]); y[0][1] = fmaf(a0, t4.y, y[0][1]);
-                    y[0][2] = fmaf(a0, t4.z, y[0][2]); y[0][3] = fmaf(a0, t4.w, y[0][3]);
-                    y[1][0] = fmaf(a1, t4.x, y[1][0]); y[1][1] = fmaf(a1, t4.y, y[1][1]);
-                    y[1][2] = fmaf(a1, t4.z, y[1][2]); y[1][3] = fmaf(a1, t4.w, y[1][3]);
+                    y00 = fmaf(a0, t2.x, y00); y01 = fmaf(a0, t2.y, y01);
+                    y10 = fmaf(a1, t2.x, y10); y11 = fmaf(a1, t2.y, y11);
                 }
                 __syncthreads();  // everyone done reading A_10
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-                    *reinterpret_cast<float4*>(sA + (32 + r0 + i) * kLdA + c0b) =
-                        make_float4(y[i][0], y[i][1], y[i][2], y[i][3]);
+                *reinterpret_cast<float2*>(sA + (32 + r0) * kLdA + c0b) = make_float2(y00, y01);
+                *reinterpret_cast<float2*>(sA + (33 + r0) * kLdA + c0b) = make_float2(y10, y11);
                 __syncthreads();
                 // T_10 = -T_11 Y  (Y now in A's lower-left block)
-                float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
 #pragma unroll 8
                 for (int m = 0; m < 32; ++m) {
-                    const float4 y4 = *reinterpret_cast<const float4*>(sA + (32 + m) * kLdA + c0b);
+                    const float2 y2 = *reinterpret_cast<const float2*>(sA + (32 + m) * kLdA + c0b);
                     const float t0 = sT[(32 + r0) * kLdA + 32 + m], t1 = sT[(33 + r0) * kLdA + 32 + m];
-                    z[0][0] = fmaf(t0, y4.x, z[0][0]); z[0][1] = fmaf(t0, y4.y, z[0][1]);
-                    z[0][2] = fmaf(t0, y4.z, z[0][2]); z[0][3] = fmaf(t0, y4.w, z[0][3]);
-                    z[1][0] = fmaf(t1, y4.x, z[1][0]); z[1][1] = fmaf(t1, y4.y, z[1][1]);
-                    z[1][2] = fmaf(t1, y4.z, z[1][2]); z[1][3] = fmaf(t1, y4.w, z[1][3]);
+                    z00 = fmaf(t0, y2.x, z00); z01 = fmaf(t0, y2.y, z01);
+                    z10 = fmaf(t1, y2.x, z10); z11 = fmaf(t1, y2.y, z11);
                 }
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-                    *reinterpret_cast<float4*>(sT + (32 + r0 + i) * kLdA + c0b) =
-                        make_float4(-z[i][0], -z[i][1], -z[i][2], -z[i][3]);
+                *reinterpret_cast<float2*>(sT + (32 + r0) * kLdA + c0b) = make_float2(-z00, -z01);
+                *reinterpret_cast<float2*>(sT + (33 + r0) * kLdA + c0b) = make_float2(-z10, -z11);
             }
             __syncthreads();
             // T1^T, T2^T rows (row m = column m of T) as bf16 MN-major B operands
-            if (tid < 64) {
-                const int j = tid;
+            if (tid < 128) {
+                const int j = tid & 63;
                 float x[64];
 #pragma unroll
                 for (int r = 0; r < 64; ++r) x[r] = sT[r * kLdA + j];
-                store_row64_scaled(sT1, j, x, bet[j] * expf(gam[j]) * rk[j]);
-                store_row64_scaled(sT2, j, x, bet[j]);
+                if (tid < 64) store_row64_scaled(sT1, j, x, bet[j] * expf(gam[j]) * rk[j]);
+                else store_row64_scaled(sT2, j, x, bet[j]);
             }
             fence_proxy_async();
             tc_fence_before();
@@ -529,15 +541,16 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             mma_phase ^= 1;
             tc_fence_after();
 
-            // ---- epilogue w: -W^T rows (lane = dk i); K -> K~ in place
+            // ---- epilogue w: -W^T rows (lane = dk i, 32 columns each); K -> K~ in place
             {
-                float x[64];
-                tmem_ld64(tmem + lane_off + kRW, x);
+                float x[32];
+                tmem_ld32(tmem + lane_off + kRW + 32 * half, x);
                 tmem_wait_ld();
-                store_row64_scaled(sWT, tid, x, -1.f);
-                const int r = tid & 63;
-                const float f = expf(gL - gam[r]) * rk[r];
-                scale_row(st + (tid < 64 ? kKb0 : kKb1), r, f);
+                store_half_row(sWT, row, half, x, -1.f);
+                if (tid < 128) {
+                    const int r = tid & 63;
+                    scale_row(st + (tid < 64 ? kKb0 : kKb1), r, expf(gL - gam[r]) * rk[r]);
+                }
             }
             fence_proxy_async();
             tc_fence_before();
@@ -563,13 +576,13 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             {
                 const float eL = expf(gL);
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = 0; cc < 2; ++cc) {
                     float v[32];
-                    tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
+                    tmem_ld32(tmem + lane_off + kRS + 64 * half + 32 * cc, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] *= eL;
-                    tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
+                    tmem_st32(tmem + lane_off + kRS + 64 * half + 32 * cc, v);
                 }
                 tmem_wait_st();
             }
@@ -577,12 +590,12 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             mma_phase ^= 1;
             tc_fence_after();
 
-            // ---- epilogue U: U^T rows (lane = dv j) as bf16 A operand
+            // ---- epilogue U: U^T rows (lane = dv j, 32 tokens each) as bf16 A operand
             {
-                float x[64];
-                tmem_ld64(tmem + lane_off + kRU, x);
+                float x[32];
+                tmem_ld32(tmem + lane_off + kRU + 32 * half, x);
                 tmem_wait_ld();
-                store_row64(sUT, tid, x);
+                store_half_row(sUT, row, half, x, 1.f);
             }
             fence_proxy_async();
             tc_fence_before();
@@ -607,24 +620,36 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
 
             // ---- epilogue S and O
             {
-                const int j = tid;
+                const int j = row;
                 float v[64];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    tmem_ld64(tmem + lane_off + kRS + 64 * hh, v);
-                    tmem_wait_ld();
-                    store_row64(sSA + hh * 16384, j, v);
-                    if (last && a.hT) {
-#pragma unroll
-                        for (int e = 0; e < 64; ++e) a.hT[sbase + (int64_t)(64 * hh + e) * kD + j] = v[e];
-                    }
-                }
-                tmem_ld64(tmem + lane_off + kRO, v);
+                tmem_ld64(tmem + lane_off + kRS + 64 * half, v);
                 tmem_wait_ld();
+                store_row64(sSA + half * 16384, j, v);
+                if (last && a.hT) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) a.hT[sbase + (int64_t)(64 * half + e) * kD + j] = v[e];
+                }
+                // O^T column j, tokens [32*half, 32*half+32) -> O tile [64 tokens][128]
+                // bf16 staged in this stage's V region (V is dead after MMA_b), then
+                // written out as coalesced 16-byte rows, only the L valid tokens.
+                float x[32];
+                tmem_ld32(tmem + lane_off + kRO + 32 * half, x);
+                tmem_wait_ld();
+                uint16_t* ostage = reinterpret_cast<uint16_t*>(st + kVb0);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ostage[(32 * half + e) * kD + j] = f32_to_bf16(x[e]);
+            }
+            __syncthreads();
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(st + kVb0);
                 uint16_t* o = static_cast<uint16_t*>(a.o);
 #pragma unroll
-                for (int r = 0; r < 64; ++r)
-                    if (r < L) o[((c0 + r) * H + U.h) * kD + j] = f32_to_bf16(v[r]);
+                for (int i = 0; i < 4; ++i) {
+                    const int vid = tid + kThreads * i;  // 16-byte vector id
+                    const int r = vid >> 4, c16 = vid & 15;
+                    if (r < L)
+                        *reinterpret_cast<uint4*>(o + ((c0 + r) * H + U.h) * kD + 8 * c16) = src[vid];
+                }
             }
             fence_proxy_async();
             tc_fence_before();
