@@ -449,14 +449,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             tc_fence_before();
             __syncthreads();
 
-            // ---- solve T = (I + A)^-1 in 32x32 blocks. Diagonal blocks by forward
-            // substitution (one column per thread, tid < 64) while tid 64..191 turn
-            // Q into Q~; then T_10 = -T_11 (A_10 T_00) on all threads.
+            // ---- solve T = (I + A)^-1 by blocks: 16x16 diagonal inverses by forward
+            // substitution (one column per thread, tid < 64), merged to 32x32
+            // (T_10 = -T_11 A_10 T_00), then to 64x64 below. Meanwhile tid 64..191
+            // turn Q into Q~ and tid 192..255 clear the upper-right 32x32 block.
             if (tid < 64) {
-                const int b = tid >> 5, c = tid & 31, o = 32 * b;
-                float x[32];
+                const int o = 16 * (tid >> 4), c = tid & 15;
+                float x[16];
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
+                for (int r = 0; r < 16; ++r) {
                     float s0 = (r == c) ? 1.f : 0.f, s1 = 0.f;
                     const float* Ar = sA + (o + r) * kLdA + o;
 #pragma unroll
@@ -471,14 +472,44 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     for (int m = (r / 4) * 4; m < r; ++m) s0 = fmaf(-Ar[m], x[m], s0);
                     x[r] = s0 + s1;
                 }
+                const bool left = ((tid >> 4) & 1) == 0;  // block 0 or 2: clear its right neighbour
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
+                for (int r = 0; r < 16; ++r) {
                     sT[(o + r) * kLdA + o + c] = x[r];
-                    if (b == 1) sT[r * kLdA + 32 + c] = 0.f;  // upper-right block of T
+                    if (left) sT[(o + r) * kLdA + o + 16 + c] = 0.f;
                 }
             } else if (tid < 192) {
                 const int rr = tid - 64, r = rr & 63;
                 scale_row(st + ((rr >> 6) ? kQb1 : kQb0), r, expf(gam[r]) * rq[r]);
+            } else {
+                for (int e = tid - 192; e < 32 * 32; e += 64) sT[(e >> 5) * kLdA + 32 + (e & 31)] = 0.f;
+            }
+            __syncthreads();
+            {
+                // 16 -> 32: for the pairs of diagonal blocks at offset o = 0 and 32,
+                // Y = A_10 T_00 then T_10 = -T_11 Y; thread -> 1 row x 2 columns.
+                const int o = 32 * (tid >> 7), idx = tid & 127;
+                const int r = idx >> 3, cc = 2 * (idx & 7);
+                float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float2 t2 = *reinterpret_cast<const float2*>(sT + (o + m) * kLdA + o + cc);
+                    const float av = sA[(o + 16 + r) * kLdA + o + m];
+                    y0 = fmaf(av, t2.x, y0);
+                    y1 = fmaf(av, t2.y, y1);
+                }
+                __syncthreads();  // A_10 blocks fully read
+                *reinterpret_cast<float2*>(sA + (o + 16 + r) * kLdA + o + cc) = make_float2(y0, y1);
+                __syncthreads();
+                float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float2 y2 = *reinterpret_cast<const float2*>(sA + (o + 16 + m) * kLdA + o + cc);
+                    const float tv = sT[(o + 16 + r) * kLdA + o + 16 + m];
+                    z0 = fmaf(tv, y2.x, z0);
+                    z1 = fmaf(tv, y2.y, z1);
+                }
+                *reinterpret_cast<float2*>(sT + (o + 16 + r) * kLdA + o + cc) = make_float2(-z0, -z1);
             }
             __syncthreads();
             {
