@@ -26,12 +26,20 @@
 // epilogues, so the MMAs read the raw bf16 input tiles that TMA brings in
 // (128-byte swizzle). The solve for T runs on CUDA cores in fp32.
 //
-// This version runs the phases of a chunk in lock-step across one 256-thread
-// CTA per SM (two warps per TMEM lane quarter, each taking half of the
-// columns); thread 0 issues TMA and MMAs. The
-// next chunk's tiles are prefetched by TMA during the current chunk.
-// Every wait is bounded: on timeout the kernel records GDN timeout status,
-// drains its TMA copies, frees TMEM and returns.
+// Warp specialisation (one CTA of 12 warps per SM, persistent over units):
+//   warps 0-7   prep group: everything that does not depend on the state --
+//               gates, norms, [Q;K]K^T, P, A, the triangular solve, W^T, U~^T,
+//               Q~ and K~ -- for chunk c+1 ...
+//   warps 8-11  state group: ... while these run the state chain of chunk c
+//               (U, the state update, O) with the state resident in TMEM. When
+//               the state group is done with a stage of the two-stage ring it
+//               refills it (TMA for the q/k/v tiles, plain loads for the gates)
+//               with the chunk two ahead.
+// The groups hand off through mbarriers; TMEM holds double-buffered U~/U
+// and O regions so the prep of c+1 never waits for the epilogues of c.
+// Every wait is bounded: on timeout the kernel records the timeout status,
+// all groups leave their loops, MMAs and TMA copies are drained (bounded),
+// TMEM is freed and the kernel returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -48,32 +56,38 @@ using namespace tc;
 
 constexpr int kC = 64;          // chunk
 constexpr int kD = 128;         // head dim (dk = dv)
-constexpr int kThreads = 256;
+constexpr int kPrepThreads = 256;
+constexpr int kStateThreads = 128;
+constexpr int kThreads = kPrepThreads + kStateThreads;
+constexpr int kStateWarp0 = kPrepThreads / 32;               // 8
+constexpr int kBarPrep = 1, kBarState = 2;                   // named barrier ids
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
 // Shared memory map (bytes from a 1024-aligned base).
 constexpr uint32_t kBox = 8192;                   // 64 rows x 128 B (64 bf16)
 constexpr uint32_t kQb0 = 0, kKb0 = kBox, kQb1 = 2 * kBox, kKb1 = 3 * kBox;
 constexpr uint32_t kVb0 = 4 * kBox, kVb1 = 5 * kBox;
-constexpr uint32_t kStageBytes = 6 * kBox;        // 48 KB: Q, K, V tiles
-constexpr uint32_t kOffSA = 2 * kStageBytes;      // S^T bf16, 2 x [128 dv][64 dk] K-major
+constexpr uint32_t kStageBytes = 6 * kBox;        // 48 KB: Q, K, V tiles (V later holds O)
+constexpr uint32_t kOffVec = 2 * kStageBytes;     // per stage: g, beta, gamma, bet, rq, rk (6 x 64 fp32)
+constexpr uint32_t kVecBytes = 2048;
+constexpr uint32_t kOffSA = kOffVec + 2 * kVecBytes;  // S^T bf16, 2 x [128 dv][64 dk] K-major
 constexpr uint32_t kOffWT = kOffSA + 32768;       // -W^T bf16 [128 dk][64 tok] MN-major
 constexpr uint32_t kOffUT = kOffWT + 16384;       // U^T bf16 [128 dv][64 tok] K-major
-constexpr uint32_t kOffP = kOffUT + 16384;        // P bf16 [64 r][64 j] K-major
-constexpr uint32_t kOffT1 = kOffP + 8192;         // T1^T bf16 [64 m][64 r] MN-major
-constexpr uint32_t kOffT2 = kOffT1 + 8192;        // T2^T bf16
+constexpr uint32_t kOffP = kOffUT + 16384;        // P bf16 [64 r][64 j] K-major, per stage
 constexpr int kLdA = 68;                          // padded fp32 row stride (272 B)
-constexpr uint32_t kOffA = kOffT2 + 8192;         // A fp32 [64][kLdA] (later also Y)
+constexpr uint32_t kOffA = kOffP + 2 * 8192;      // A fp32 [64][kLdA]; after the solve T1^T, T2^T
+constexpr uint32_t kOffT1 = kOffA, kOffT2 = kOffA + 8192;
 constexpr uint32_t kOffTf = kOffA + 64 * kLdA * 4;  // T fp32 [64][kLdA]
-constexpr uint32_t kOffVec = kOffTf + 64 * kLdA * 4;  // gamma, beta, rq, rk: 4 x 64 fp32
-constexpr uint32_t kOffBar = kOffVec + 1024;      // mbarriers
-constexpr uint32_t kOffMisc = kOffBar + 64;       // tmem base, abort flag, scan carry
+constexpr uint32_t kOffBar = kOffTf + 64 * kLdA * 4;  // mbarriers
+constexpr uint32_t kOffMisc = kOffBar + 128;      // tmem base, abort flag, scan carry
 constexpr uint32_t kSmemBytes = kOffMisc + 64;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kOffA % 1024 == 0 && kOffSA % 1024 == 0 && kOffP % 1024 == 0, "swizzle alignment");
 
 // TMEM columns (fp32, 128 lanes).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kRS = 0, kRU = 128, kRO = 192, kRA = 256, kRW = 320;
+constexpr uint32_t kRS = 0, kRO = 128, kRU = 256, kRA = 384, kRW = 448;  // R_O, R_U: 2 x 64
 
 constexpr uint32_t kIdescA = idesc_bf16(128, 64, 0, 0);    // [Q;K] K^T
 constexpr uint32_t kIdescMN = idesc_bf16(128, 64, 1, 1);   // K^T T1^T, V^T T2^T
@@ -92,33 +106,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ void unpack_bf16(uint32_t w, float& lo, float& hi) {
     lo = __uint_as_float(w << 16);
     hi = __uint_as_float(w & 0xFFFF0000u);
-}
-
-// Write 64 fp32 values as one 128-byte bf16 row of a 128B-swizzled tile.
-__device__ __forceinline__ void store_row64(uint8_t* tile, int row, const float (&v)[64]) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = pack_bf16(v[8 * c + 0], v[8 * c + 1]);
-        u.y = pack_bf16(v[8 * c + 2], v[8 * c + 3]);
-        u.z = pack_bf16(v[8 * c + 4], v[8 * c + 5]);
-        u.w = pack_bf16(v[8 * c + 6], v[8 * c + 7]);
-        *reinterpret_cast<uint4*>(tile + sw128_off(row, c)) = u;
-    }
-}
-
-// Same, with every value multiplied by f.
-__device__ __forceinline__ void store_row64_scaled(uint8_t* tile, int row, const float (&v)[64],
-                                                   float f) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint4 u;
-        u.x = pack_bf16(v[8 * c + 0] * f, v[8 * c + 1] * f);
-        u.y = pack_bf16(v[8 * c + 2] * f, v[8 * c + 3] * f);
-        u.z = pack_bf16(v[8 * c + 4] * f, v[8 * c + 5] * f);
-        u.w = pack_bf16(v[8 * c + 6] * f, v[8 * c + 7] * f);
-        *reinterpret_cast<uint4*>(tile + sw128_off(row, c)) = u;
-    }
 }
 
 // Write 32 fp32 values (times f) as columns [32*half, 32*half + 32) of one
@@ -202,185 +189,186 @@ __device__ __forceinline__ void issue_tiles(uint8_t* stage, uint64_t* bar, const
     tma_load_3d(stage + kVb1, mv, bar, 64, h, t);
 }
 
+
+// Named barrier over `count` threads (warp multiple) with an OR-reduction.
+__device__ __forceinline__ bool group_any(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void group_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// The CTA's work list: chunks of its units (u = blockIdx.x + k * gridDim.x,
+// non-empty ones), in order. Every group walks the same list.
+struct Item {
+    int64_t u;
+    Unit U;
+    int64_t c0;
+    int L;
+    bool first, last;
+};
+
+__device__ __forceinline__ bool item_first(const PrefillArgs& a, int64_t total, Item& it) {
+    it.u = next_nonempty(a, blockIdx.x, total);
+    if (it.u >= total) return false;
+    load_unit(a, it.u, it.U);
+    it.c0 = it.U.start;
+    it.first = true;
+    it.L = (int)((it.U.end - it.c0 < kC) ? it.U.end - it.c0 : kC);
+    it.last = it.c0 + kC >= it.U.end;
+    return true;
+}
+
+__device__ __forceinline__ bool item_next(const PrefillArgs& a, int64_t total, Item& it) {
+    it.c0 += kC;
+    it.first = false;
+    if (it.c0 >= it.U.end) {
+        it.u = next_nonempty(a, it.u + gridDim.x, total);
+        if (it.u >= total) return false;
+        load_unit(a, it.u, it.U);
+        it.c0 = it.U.start;
+        it.first = true;
+    }
+    it.L = (int)((it.U.end - it.c0 < kC) ? it.U.end - it.c0 : kC);
+    it.last = it.c0 + kC >= it.U.end;
+    return true;
+}
+
+// Bounded wait that also gives up once another group has aborted.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
+                                                   volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitNs) return false;
+    }
+    return true;
+}
+
+struct Smem {
+    uint8_t* base;
+    __device__ uint8_t* stage(int s) const { return base + s * kStageBytes; }
+    __device__ float* vec(int s) const { return reinterpret_cast<float*>(base + kOffVec + s * kVecBytes); }
+    // vec layout: [0,64) g raw, [64,128) beta raw, [128,192) gamma, [192,256) beta,
+    // [256,320) rq, [320,384) rk
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap map_q,
                   const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the shared-window address (swizzle atoms, TMA).
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const Smem S{sm};
     const PrefillArgs& a = P.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // Two warps share each TMEM lane quarter and split the columns in halves.
-    const int quarter = warp & 3, half = warp >> 2;
-    const int row = 32 * quarter + lane;  // TMEM lane owned by this thread
     const int H = a.H;
     const int64_t total = (int64_t)a.N * H;
 
     uint8_t* sSA = sm + kOffSA;
     uint8_t* sWT = sm + kOffWT;
     uint8_t* sUT = sm + kOffUT;
-    uint8_t* sP = sm + kOffP;
     uint8_t* sT1 = sm + kOffT1;
     uint8_t* sT2 = sm + kOffT2;
     float* sA = reinterpret_cast<float*>(sm + kOffA);
     float* sT = reinterpret_cast<float*>(sm + kOffTf);
-    float* gam = reinterpret_cast<float*>(sm + kOffVec);
-    float* bet = gam + 64;
-    float* rq = gam + 128;
-    float* rk = gam + 192;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [2]
-    uint64_t* mbar = full + 2;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
+    uint64_t* full = bars + 0;      // [2] tiles + gates of a stage landed (state -> prep)
+    uint64_t* pdone = bars + 4;     // [2] prep -> state        (count 1)
+    uint64_t* pa_bar = bars + 6;    // prep MMA completions
+    uint64_t* u_bar = bars + 7;     // state MMA1 (U) completion
+    uint64_t* s_bar = bars + 8;     // state MMA2 (S) completion
+    uint64_t* o_bar = bars + 9;     // state MMA2 (O) completion
+    uint64_t* wt_free = bars + 10;  // state MMA1 done reading -W^T
+    uint64_t* drain_p = bars + 11;  // exit: all prep MMAs done
+    uint64_t* drain_s = bars + 12;  // exit: all state MMAs done
     uint32_t* tmem_base_p = reinterpret_cast<uint32_t*>(sm + kOffMisc);
-    int* abort_flag = reinterpret_cast<int*>(sm + kOffMisc + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
     float* carry = reinterpret_cast<float*>(sm + kOffMisc + 8);
 
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
-        mbar_init(mbar, 1);
+        mbar_init(&pdone[0], 1);
+        mbar_init(&pdone[1], 1);
+        mbar_init(pa_bar, 1);
+        mbar_init(u_bar, 1);
+        mbar_init(s_bar, 1);
+        mbar_init(o_bar, 1);
+        mbar_init(wt_free, 1);
+        mbar_init(drain_p, 1);
+        mbar_init(drain_s, 1);
         fence_mbar_init();
         *abort_flag = 0;
-        prefetch_tmap(&map_q);
-        prefetch_tmap(&map_k);
-        prefetch_tmap(&map_v);
     }
     if (warp == 0) tmem_alloc(tmem_base_p, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_p;
-    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;  // this warp's TMEM lane quarter
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lane quarter
 
-    uint32_t full_phase = 0;  // bit s: expected parity of full[s]
-    uint32_t mma_phase = 0;
-    int cur = 0;              // stage of the chunk being processed
-    uint32_t inflight = 0;    // bit s: TMA issued into stage s, not yet consumed
-    auto stage = [&](int i) { return sm + i * kStageBytes; };
-    bool aborted = false;
-
-    // Bounded wait by every thread; all threads agree on the outcome.
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-        const bool ok = mbar_wait(bar, parity, kWaitNs);
-        const int bad = __syncthreads_or(!ok);
-        if (bad && tid == 0) {
-            *abort_flag = 1;
-            set_status(a.status, kStatusTimeout);
-        }
-        return !bad;
+    auto abort_now = [&](int code) {
+        *abort_flag = 1;
+        set_status(a.status, code);
     };
 
-    int64_t u = next_nonempty(a, blockIdx.x, total);
-    // Units with no tokens on this CTA's stride still need hT = h0.
-    for (int64_t e = blockIdx.x; e < total; e += gridDim.x) {
-        Unit U;
-        if (!load_unit(a, e, U)) {
-            if (tid == 0) set_status(a.status, kStatusBadSeqlens);
-            continue;
-        }
-        if (U.end > U.start || !a.hT) continue;
-        const int64_t base = ((int64_t)U.n * H + U.h) * kD * kD;
-        for (int i = tid; i < kD * kD; i += kThreads) a.hT[base + i] = a.h0 ? a.h0[base + i] : 0.f;
-    }
-    // Gates of the next chunk, prefetched one chunk ahead (threads 0..63, row = tid).
-    float g_next = 0.f, b_next = 0.f;
-    if (u < total) {
-        Unit U;
-        load_unit(a, u, U);
-        if (tid == 0) {
-            issue_tiles(stage(0), &full[0], &map_q, &map_k, &map_v, U.h, U.start);
-            inflight |= 1u;
-        }
-        if (tid < 64 && U.start + tid < U.end) {
-            g_next = a.g[(U.start + tid) * H + U.h];
-            b_next = a.beta[(U.start + tid) * H + U.h];
-        }
-    }
-
-    while (u < total && !aborted) {
-        Unit U;
-        load_unit(a, u, U);
-        const int64_t sbase = ((int64_t)U.n * H + U.h) * kD * kD;
-
-        // ---- initial state: R_S (fp32) and S^T (bf16 A operand). Thread (row j =
-        // dv index, half) owns dk columns [64*half, 64*half + 64).
-        {
-            const int j = row;
-            float v[64];
-#pragma unroll
-            for (int e = 0; e < 64; ++e)
-                v[e] = a.h0 ? a.h0[sbase + (int64_t)(64 * half + e) * kD + j] : 0.f;
-            float w0[32], w1[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) { w0[e] = v[e]; w1[e] = v[32 + e]; }
-            tmem_st32(tmem + lane_off + kRS + 64 * half, w0);
-            tmem_st32(tmem + lane_off + kRS + 64 * half + 32, w1);
-            store_row64(sSA + half * 16384, j, v);
-            tmem_wait_st();
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-
-        for (int64_t c0 = U.start; c0 < U.end && !aborted; c0 += kC) {
-            const int L = (U.end - c0 < kC) ? (int)(U.end - c0) : kC;
-            const bool last = c0 + kC >= U.end;
-            uint8_t* st = stage(cur);
-
-            // ---- prefetch the next chunk (this unit or the next one): tiles into
-            // the other stage by TMA, gates into registers
-            const float g_cur = g_next, b_cur = b_next;
+    if (warp < kStateWarp0) {
+        // ================================================================ prep
+        const int ptid = tid;  // 0..255
+        const int half = warp >> 2;
+        const int row = 32 * (warp & 3) + lane;  // TMEM lane owned by this thread
+        uint32_t pa_phase = 0;
+        Item it;
+        bool have = item_first(a, total, it);
+        for (int i = 0; have; ++i, have = item_next(a, total, it)) {
+            const int s = i & 1, ns = i >> 1;
+            const int L = it.L;
+            uint8_t* st = S.stage(s);
+            float* vec = S.vec(s);
+            float* gam = vec + 128;
+            float* bet = vec + 192;
+            float* rq = vec + 256;
+            float* rk = vec + 320;
+            uint8_t* sP = sm + kOffP + s * 8192;
             {
-                int64_t nu = u, nc0 = c0 + kC, nend = U.end;
-                int nh = U.h;
-                if (last) {
-                    nu = next_nonempty(a, u + gridDim.x, total);
-                    if (nu < total) {
-                        Unit N2;
-                        load_unit(a, nu, N2);
-                        nc0 = N2.start;
-                        nend = N2.end;
-                        nh = N2.h;
-                    }
-                }
-                if (nu < total) {
-                    if (tid == 0) {
-                        issue_tiles(stage(cur ^ 1), &full[cur ^ 1], &map_q, &map_k, &map_v, nh, nc0);
-                        inflight |= 1u << (cur ^ 1);
-                    }
-                    g_next = 0.f;
-                    b_next = 0.f;
-                    if (tid < 64 && nc0 + tid < nend) {
-                        g_next = a.g[(nc0 + tid) * H + nh];
-                        b_next = a.beta[(nc0 + tid) * H + nh];
-                    }
+                const bool ok = mbar_wait_or_abort(&full[s], ns & 1, abort_flag);
+                if (group_any(kBarPrep, kPrepThreads, !ok)) {
+                    if (ptid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                    break;
                 }
             }
-            if (!wait_all(&full[cur], (full_phase >> cur) & 1u)) { aborted = true; break; }
-            full_phase ^= 1u << cur;
-            inflight &= ~(1u << cur);
 
-            // ---- per-row scalars: gates, cumulative decay, L2 norms
-            if (tid < 64) {
-                const int r = tid;
-                float g = 0.f, b = 0.f, fq = 0.f;
+            // ---- per-row scalars: cumulative decay, L2 norms (q: tid < 64, k: 64..127)
+            if (ptid < 64) {
+                const int r = ptid;
+                float fq = 0.f;
                 if (r < L) {
-                    g = g_cur;
-                    b = b_cur;
                     const float ss = row_sumsq(st + kQb0, r) + row_sumsq(st + kQb1, r);
                     fq = (a.qk_l2norm ? 1.f / sqrtf(ss + a.eps) : 1.f) * a.scale;
                 }
-                float x = g;  // inclusive scan over the 64 rows (two warps)
+                float x = vec[r];  // g (0 past L); inclusive scan over 64 rows (two warps)
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, x, o);
                     if (lane >= o) x += y;
                 }
-                if (tid == 31) *carry = x;
-                bet[r] = b;
+                if (ptid == 31) *carry = x;
+                bet[r] = vec[64 + r];
                 rq[r] = fq;
-                gam[r] = x;  // warp 1 adds warp 0's total below
-            } else if (tid < 128) {
-                const int r = tid - 64;
+                gam[r] = x;
+            } else if (ptid < 128) {
+                const int r = ptid - 64;
                 float fk = 0.f;
                 if (r < L) {
                     const float ss = row_sumsq(st + kKb0, r) + row_sumsq(st + kKb1, r);
@@ -388,13 +376,13 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
                 rk[r] = fk;
             }
-            __syncthreads();
-            if (tid >= 32 && tid < 64) gam[tid] += *carry;
-            __syncthreads();
+            group_sync(kBarPrep, kPrepThreads);
+            if (ptid >= 32 && ptid < 64) gam[ptid] += *carry;
+            group_sync(kBarPrep, kPrepThreads);
             const float gL = gam[63];
 
-            // ---- MMA_a: [Q;K] K^T -> R_A
-            if (tid == 0) {
+            // ---- [Q;K] K^T -> R_A
+            if (ptid == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
@@ -403,16 +391,21 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     mma_bf16(tmem + kRA, sw128_desc(smem_u32(st + qo), 16, 1024),
                              sw128_desc(smem_u32(st + ko), 16, 1024), kIdescA, k > 0);
                 }
-                mma_commit(mbar);
+                mma_commit(pa_bar);
             }
-            if (!wait_all(mbar, mma_phase)) { aborted = true; break; }
-            mma_phase ^= 1;
+            {
+                const bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag);
+                if (group_any(kBarPrep, kPrepThreads, !ok)) {
+                    if (ptid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                    break;
+                }
+                pa_phase ^= 1;
+            }
             tc_fence_after();
 
-            // ---- epilogue a: P rows (lanes < 64) and A rows (lanes >= 64); each
-            // thread takes 32 of the 64 columns. Branch-free: every element is
-            // computed (exponent clamped at 0 so the masked-out upper triangle
-            // cannot overflow), then selected.
+            // ---- P rows (lanes < 64) and A rows (lanes >= 64), 32 columns per
+            // thread. Branch-free: every element is computed (exponent clamped
+            // at 0 so the masked-out upper triangle cannot overflow), then selected.
             {
                 float x[32];
                 tmem_ld32(tmem + lane_off + kRA + 32 * half, x);
@@ -447,14 +440,14 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             }
             fence_proxy_async();
             tc_fence_before();
-            __syncthreads();
+            group_sync(kBarPrep, kPrepThreads);
 
             // ---- solve T = (I + A)^-1 by blocks: 16x16 diagonal inverses by forward
-            // substitution (one column per thread, tid < 64), merged to 32x32
-            // (T_10 = -T_11 A_10 T_00), then to 64x64 below. Meanwhile tid 64..191
-            // turn Q into Q~ and tid 192..255 clear the upper-right 32x32 block.
-            if (tid < 64) {
-                const int o = 16 * (tid >> 4), c = tid & 15;
+            // substitution (one column per thread, ptid < 64), merged to 32x32
+            // (T_10 = -T_11 A_10 T_00), then to 64x64. Meanwhile ptid 64..191
+            // turn Q into Q~ and ptid 192..255 clear the upper-right 32x32 block.
+            if (ptid < 64) {
+                const int o = 16 * (ptid >> 4), c = ptid & 15;
                 float x[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
@@ -472,23 +465,22 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     for (int m = (r / 4) * 4; m < r; ++m) s0 = fmaf(-Ar[m], x[m], s0);
                     x[r] = s0 + s1;
                 }
-                const bool left = ((tid >> 4) & 1) == 0;  // block 0 or 2: clear its right neighbour
+                const bool left = ((ptid >> 4) & 1) == 0;  // blocks 0 and 2 clear their right neighbour
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     sT[(o + r) * kLdA + o + c] = x[r];
                     if (left) sT[(o + r) * kLdA + o + 16 + c] = 0.f;
                 }
-            } else if (tid < 192) {
-                const int rr = tid - 64, r = rr & 63;
+            } else if (ptid < 192) {
+                const int rr = ptid - 64, r = rr & 63;
                 scale_row(st + ((rr >> 6) ? kQb1 : kQb0), r, expf(gam[r]) * rq[r]);
             } else {
-                for (int e = tid - 192; e < 32 * 32; e += 64) sT[(e >> 5) * kLdA + 32 + (e & 31)] = 0.f;
+                for (int e = ptid - 192; e < 32 * 32; e += 64) sT[(e >> 5) * kLdA + 32 + (e & 31)] = 0.f;
             }
-            __syncthreads();
+            group_sync(kBarPrep, kPrepThreads);
             {
-                // 16 -> 32: for the pairs of diagonal blocks at offset o = 0 and 32,
-                // Y = A_10 T_00 then T_10 = -T_11 Y; thread -> 1 row x 2 columns.
-                const int o = 32 * (tid >> 7), idx = tid & 127;
+                // 16 -> 32 for the block pairs at o = 0 and 32: thread -> 1 row x 2 columns
+                const int o = 32 * (ptid >> 7), idx = ptid & 127;
                 const int r = idx >> 3, cc = 2 * (idx & 7);
                 float y0 = 0.f, y1 = 0.f;
 #pragma unroll
@@ -498,9 +490,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     y0 = fmaf(av, t2.x, y0);
                     y1 = fmaf(av, t2.y, y1);
                 }
-                __syncthreads();  // A_10 blocks fully read
+                group_sync(kBarPrep, kPrepThreads);  // A_10 blocks fully read
                 *reinterpret_cast<float2*>(sA + (o + 16 + r) * kLdA + o + cc) = make_float2(y0, y1);
-                __syncthreads();
+                group_sync(kBarPrep, kPrepThreads);
                 float z0 = 0.f, z1 = 0.f;
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
@@ -511,10 +503,10 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
                 *reinterpret_cast<float2*>(sT + (o + 16 + r) * kLdA + o + cc) = make_float2(-z0, -z1);
             }
-            __syncthreads();
+            group_sync(kBarPrep, kPrepThreads);
             {
-                // Y = A_10 T_00 ; thread -> 2 rows x 2 columns of the 32x32 block
-                const int r0 = 2 * (tid >> 4), c0b = 2 * (tid & 15);
+                // 32 -> 64: Y = A_10 T_00 then T_10 = -T_11 Y; thread -> 2 rows x 2 columns
+                const int r0 = 2 * (ptid >> 4), c0b = 2 * (ptid & 15);
                 float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
                 for (int m = 0; m < 32; ++m) {
@@ -523,11 +515,10 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     y00 = fmaf(a0, t2.x, y00); y01 = fmaf(a0, t2.y, y01);
                     y10 = fmaf(a1, t2.x, y10); y11 = fmaf(a1, t2.y, y11);
                 }
-                __syncthreads();  // everyone done reading A_10
+                group_sync(kBarPrep, kPrepThreads);  // A_10 fully read
                 *reinterpret_cast<float2*>(sA + (32 + r0) * kLdA + c0b) = make_float2(y00, y01);
                 *reinterpret_cast<float2*>(sA + (33 + r0) * kLdA + c0b) = make_float2(y10, y11);
-                __syncthreads();
-                // T_10 = -T_11 Y  (Y now in A's lower-left block)
+                group_sync(kBarPrep, kPrepThreads);
                 float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
 #pragma unroll 8
                 for (int m = 0; m < 32; ++m) {
@@ -539,162 +530,309 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 *reinterpret_cast<float2*>(sT + (32 + r0) * kLdA + c0b) = make_float2(-z00, -z01);
                 *reinterpret_cast<float2*>(sT + (33 + r0) * kLdA + c0b) = make_float2(-z10, -z11);
             }
-            __syncthreads();
-            // T1^T, T2^T rows (row m = column m of T) as bf16 MN-major B operands
-            if (tid < 128) {
-                const int j = tid & 63;
-                float x[64];
+            group_sync(kBarPrep, kPrepThreads);
+            // T1^T, T2^T rows (row m = column m of T) as bf16 MN-major B operands,
+            // written over A (dead by now)
+            {
+                // thread -> (tile, row j, half): 32 values of row j of T1^T or T2^T
+                const int j = ptid & 63, hf = (ptid >> 6) & 1, which = ptid >> 7;
+                float x[32];
 #pragma unroll
-                for (int r = 0; r < 64; ++r) x[r] = sT[r * kLdA + j];
-                if (tid < 64) store_row64_scaled(sT1, j, x, bet[j] * expf(gam[j]) * rk[j]);
-                else store_row64_scaled(sT2, j, x, bet[j]);
+                for (int r = 0; r < 32; ++r) x[r] = sT[(32 * hf + r) * kLdA + j];
+                const float f = which == 0 ? bet[j] * expf(gam[j]) * rk[j] : bet[j];
+                store_half_row(which == 0 ? sT1 : sT2, j, hf, x, f);
             }
             fence_proxy_async();
             tc_fence_before();
-            __syncthreads();
+            group_sync(kBarPrep, kPrepThreads);
 
-            // ---- MMA_w: W^T = K^T T1^T -> R_W ;  MMA_b: U~^T = V^T T2^T -> R_U
-            if (tid == 0) {
+            // ---- W^T = K^T T1^T -> R_W ;  U~^T = V^T T2^T -> R_U[s]
+            if (ptid == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
+                for (int k = 0; k < 4; ++k)
                     mma_bf16(tmem + kRW, sw128_desc(smem_u32(st + kKb0 + 2048 * k), kKb1 - kKb0, 1024),
                              sw128_desc(smem_u32(sT1 + 2048 * k), 8192, 1024), kIdescMN, k > 0);
-                }
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    mma_bf16(tmem + kRU, sw128_desc(smem_u32(st + kVb0 + 2048 * k), kVb1 - kVb0, 1024),
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem + kRU + 64 * s, sw128_desc(smem_u32(st + kVb0 + 2048 * k), kVb1 - kVb0, 1024),
                              sw128_desc(smem_u32(sT2 + 2048 * k), 8192, 1024), kIdescMN, k > 0);
-                }
-                mma_commit(mbar);
+                mma_commit(pa_bar);
             }
-            if (!wait_all(mbar, mma_phase)) { aborted = true; break; }
-            mma_phase ^= 1;
+            {
+                bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag);
+                // -W^T is about to be overwritten: the state group's MMA1 of the
+                // previous chunk must be done reading it.
+                if (ok && i > 0) ok = mbar_wait_or_abort(wt_free, (i - 1) & 1, abort_flag);
+                if (group_any(kBarPrep, kPrepThreads, !ok)) {
+                    if (ptid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                    break;
+                }
+                pa_phase ^= 1;
+            }
             tc_fence_after();
 
-            // ---- epilogue w: -W^T rows (lane = dk i, 32 columns each); K -> K~ in place
+            // ---- -W^T rows (lane = dk i, 32 columns each); K -> K~ in place
             {
                 float x[32];
                 tmem_ld32(tmem + lane_off + kRW + 32 * half, x);
                 tmem_wait_ld();
                 store_half_row(sWT, row, half, x, -1.f);
-                if (tid < 128) {
-                    const int r = tid & 63;
-                    scale_row(st + (tid < 64 ? kKb0 : kKb1), r, expf(gL - gam[r]) * rk[r]);
+                if (ptid < 128) {
+                    const int r = ptid & 63;
+                    scale_row(st + (ptid < 64 ? kKb0 : kKb1), r, expf(gL - gam[r]) * rk[r]);
                 }
             }
             fence_proxy_async();
             tc_fence_before();
-            __syncthreads();
-
-            // ---- MMA1: U^T += S^T (-W^T) (R_U) ; O^T = S^T Q~^T (R_O)
-            if (tid == 0) {
-                tc_fence_after();
+            group_sync(kBarPrep, kPrepThreads);
+            if (ptid == 0) mbar_arrive(&pdone[s]);
+        }
+        // drain this issuer's MMAs before TMEM is freed
+        if (ptid == 0) {
+            mma_commit(drain_p);
+            mbar_wait(drain_p, 0, kWaitNs / 4);
+        }
+    } else {
+        // ================================================================ state
+        const int stid = tid - kPrepThreads;  // 0..127 = TMEM lane = dv index j
+        const int j = stid;
+        uint32_t ph = 0;  // parity of u_bar / s_bar / o_bar (one completion each per chunk)
+        // Units with no tokens on this CTA's stride still need hT = h0.
+        for (int64_t e = blockIdx.x; e < total; e += gridDim.x) {
+            Unit U;
+            if (!load_unit(a, e, U)) {
+                if (stid == 0) set_status(a.status, kStatusBadSeqlens);
+                continue;
+            }
+            if (U.end > U.start || !a.hT) continue;
+            const int64_t base = ((int64_t)U.n * H + U.h) * kD * kD;
+            for (int x = stid; x < kD * kD; x += kStateThreads) a.hT[base + x] = a.h0 ? a.h0[base + x] : 0.f;
+        }
+        // Fill stage s with item `f`: gates by threads 0..63, then the leader
+        // arms the stage barrier and issues the six TMA tile loads.
+        uint32_t issued = 0, issued_par = 0;  // for the bounded drain at exit
+        auto fill = [&](const Item& f, int s, int use) {
+            float* v = S.vec(s);
+            if (stid < 64) {
+                const int r = stid;
+                float g = 0.f, b = 0.f;
+                if (r < f.L) {
+                    g = a.g[(f.c0 + r) * H + f.U.h];
+                    b = a.beta[(f.c0 + r) * H + f.U.h];
+                }
+                v[r] = g;
+                v[64 + r] = b;
+            }
+            group_sync(kBarState, kStateThreads);
+            if (stid == 0) {
+                issue_tiles(S.stage(s), &full[s], &map_q, &map_k, &map_v, f.U.h, f.c0);
+                issued |= 1u << s;
+                issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(use & 1) << s);
+            }
+        };
+        if (stid == 0) {
+            prefetch_tmap(&map_q);
+            prefetch_tmap(&map_k);
+            prefetch_tmap(&map_v);
+        }
+        Item it, ahead;
+        bool have = item_first(a, total, it);
+        bool have_ahead = have;
+        if (have) {
+            ahead = it;
+            fill(ahead, 0, 0);
+            have_ahead = item_next(a, total, ahead);
+            if (have_ahead) {
+                fill(ahead, 1, 0);
+                have_ahead = item_next(a, total, ahead);  // ahead = item 2
+            }
+        }
+        bool drained = true;
+        for (int i = 0; have; ++i, have = item_next(a, total, it)) {
+            const int s = i & 1, ns = i >> 1;
+            const int L = it.L;
+            const int64_t c0 = it.c0;
+            uint8_t* st = S.stage(s);
+            const float* vec = S.vec(s);
+            const int64_t sbase = ((int64_t)it.U.n * H + it.U.h) * kD * kD;
+            if (it.first) {
+                // initial state: R_S (fp32) and S^T (bf16 A operand); thread = dv lane j
+                const float* h0p = a.h0 ? a.h0 + sbase + j : nullptr;  // column j of S
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float v[32];
+                    if (h0p) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = h0p[(32 * cc + e) * kD];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                    }
+                    tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
+                }
+                tmem_wait_st();
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
+                    tmem_wait_ld();
+                    store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                group_sync(kBarState, kStateThreads);
+            }
+            {
+                const bool ok = mbar_wait_or_abort(&pdone[s], ns & 1, abort_flag);
+                if (group_any(kBarState, kStateThreads, !ok)) {
+                    if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                    break;
+                }
+            }
+            tc_fence_after();
+            drained = false;
+            // ---- MMA1: U^T += S^T (-W^T) (R_U[s]) ; O^T = S^T Q~^T (R_O[s])
+            if (stid == 0) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint64_t sa = sw128_desc(smem_u32(sSA + (k >> 2) * 16384 + 32 * (k & 3)), 16, 1024);
-                    mma_bf16(tmem + kRU, sa, sw128_desc(smem_u32(sWT + 2048 * k), 8192, 1024), kIdescSW, 1);
+                    mma_bf16(tmem + kRU + 64 * s, sa, sw128_desc(smem_u32(sWT + 2048 * k), 8192, 1024),
+                             kIdescSW, 1);
                 }
+                mma_commit(u_bar);
+                mma_commit(wt_free);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint64_t sa = sw128_desc(smem_u32(sSA + (k >> 2) * 16384 + 32 * (k & 3)), 16, 1024);
                     const uint32_t qo = (k < 4 ? kQb0 : kQb1) + 32 * (k & 3);
-                    mma_bf16(tmem + kRO, sa, sw128_desc(smem_u32(st + qo), 16, 1024), kIdescSQ, k > 0);
+                    mma_bf16(tmem + kRO + 64 * s, sa, sw128_desc(smem_u32(st + qo), 16, 1024), kIdescSQ,
+                             k > 0);
                 }
-                mma_commit(mbar);
             }
             // R_S <- e^{gamma_L} R_S while MMA1 runs (MMA1 does not touch R_S)
             {
-                const float eL = expf(gL);
+                const float eL = expf(vec[128 + 63]);
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
+                for (int cc = 0; cc < 4; ++cc) {
                     float v[32];
-                    tmem_ld32(tmem + lane_off + kRS + 64 * half + 32 * cc, v);
+                    tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] *= eL;
-                    tmem_st32(tmem + lane_off + kRS + 64 * half + 32 * cc, v);
+                    tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
                 }
                 tmem_wait_st();
             }
-            if (!wait_all(mbar, mma_phase)) { aborted = true; break; }
-            mma_phase ^= 1;
-            tc_fence_after();
-
-            // ---- epilogue U: U^T rows (lane = dv j, 32 tokens each) as bf16 A operand
             {
+                const bool ok = mbar_wait_or_abort(u_bar, ph, abort_flag);
+                if (group_any(kBarState, kStateThreads, !ok)) {
+                    if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                    break;
+                }
+            }
+            tc_fence_after();
+            // ---- U^T row j (64 tokens) as the bf16 A operand of MMA2
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
                 float x[32];
-                tmem_ld32(tmem + lane_off + kRU + 32 * half, x);
+                tmem_ld32(tmem + lane_off + kRU + 64 * s + 32 * hf, x);
                 tmem_wait_ld();
-                store_half_row(sUT, row, half, x, 1.f);
+                store_half_row(sUT, j, hf, x, 1.f);
             }
             fence_proxy_async();
             tc_fence_before();
-            __syncthreads();
-
-            // ---- MMA2: O^T += U^T P^T (R_O) ; S^T += U^T K~ (R_S)
-            if (tid == 0) {
+            group_sync(kBarState, kStateThreads);
+            // ---- MMA2: S^T += U^T K~ (R_S) ; O^T += U^T P^T (R_O[s])
+            if (stid == 0) {
                 tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + kRO, sw128_desc(smem_u32(sUT + 32 * k), 16, 1024),
-                             sw128_desc(smem_u32(sP + 32 * k), 16, 1024), kIdescSQ, 1);
+                uint8_t* sP = sm + kOffP + s * 8192;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(tmem + kRS, sw128_desc(smem_u32(sUT + 32 * k), 16, 1024),
                              sw128_desc(smem_u32(st + kKb0 + 2048 * k), kKb1 - kKb0, 1024), kIdescUK, 1);
-                mma_commit(mbar);
-            }
-            if (!wait_all(mbar, mma_phase)) { aborted = true; break; }
-            mma_phase ^= 1;
-            tc_fence_after();
-
-            // ---- epilogue S and O
-            {
-                const int j = row;
-                float v[64];
-                tmem_ld64(tmem + lane_off + kRS + 64 * half, v);
-                tmem_wait_ld();
-                store_row64(sSA + half * 16384, j, v);
-                if (last && a.hT) {
+                mma_commit(s_bar);
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) a.hT[sbase + (int64_t)(64 * half + e) * kD + j] = v[e];
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem + kRO + 64 * s, sw128_desc(smem_u32(sUT + 32 * k), 16, 1024),
+                             sw128_desc(smem_u32(sP + 32 * k), 16, 1024), kIdescSQ, 1);
+                mma_commit(o_bar);
+            }
+            {
+                const bool ok = mbar_wait_or_abort(s_bar, ph, abort_flag);
+                if (group_any(kBarState, kStateThreads, !ok)) {
+                    if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                    break;
                 }
-                // O^T column j, tokens [32*half, 32*half+32) -> O tile [64 tokens][128]
-                // bf16 staged in this stage's V region (V is dead after MMA_b), then
-                // written out as coalesced 16-byte rows, only the L valid tokens.
-                float x[32];
-                tmem_ld32(tmem + lane_off + kRO + 32 * half, x);
-                tmem_wait_ld();
-                uint16_t* ostage = reinterpret_cast<uint16_t*>(st + kVb0);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ostage[(32 * half + e) * kD + j] = f32_to_bf16(x[e]);
             }
-            __syncthreads();
-            {
-                const uint4* src = reinterpret_cast<const uint4*>(st + kVb0);
-                uint16_t* o = static_cast<uint16_t*>(a.o);
+            tc_fence_after();
+            // ---- new state: bf16 S^T for the next chunk's MMA1; final state at the end
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int vid = tid + kThreads * i;  // 16-byte vector id
-                    const int r = vid >> 4, c16 = vid & 15;
-                    if (r < L)
-                        *reinterpret_cast<uint4*>(o + ((c0 + r) * H + U.h) * kD + 8 * c16) = src[vid];
+            for (int cc = 0; cc < 4; ++cc) {
+                float v[32];
+                tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
+                tmem_wait_ld();
+                store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
+                if (it.last && a.hT) {
+                    float* hTp = a.hT + sbase + j + 32 * cc * kD;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) hTp[e * kD] = v[e];
                 }
             }
             fence_proxy_async();
+            {
+                const bool ok = mbar_wait_or_abort(o_bar, ph, abort_flag);
+                if (group_any(kBarState, kStateThreads, !ok)) {
+                    if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                    break;
+                }
+            }
+            tc_fence_after();
+            ph ^= 1;
+            // ---- O: column j of O^T -> O tile [64 tokens][128] bf16 staged in this
+            // stage's V region (V is dead after the prep's MMA), then written out as
+            // coalesced 16-byte rows, only the chunk's L valid tokens.
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float x[32];
+                tmem_ld32(tmem + lane_off + kRO + 64 * s + 32 * hf, x);
+                tmem_wait_ld();
+                uint16_t* ostage = reinterpret_cast<uint16_t*>(st + kVb0);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ostage[(32 * hf + e) * kD + j] = f32_to_bf16(x[e]);
+            }
             tc_fence_before();
-            __syncthreads();
-            cur ^= 1;
+            group_sync(kBarState, kStateThreads);
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(st + kVb0);
+                // vector vid = stid + 128 k covers token r = 8 k + stid / 16, 16-byte column stid % 16
+                uint16_t* orow = static_cast<uint16_t*>(a.o) + (c0 * H + it.U.h) * kD + 8 * (stid & 15);
+                const int64_t tok_stride = (int64_t)H * kD;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int r = 8 * k + (stid >> 4);
+                    if (r < L) *reinterpret_cast<uint4*>(orow + r * tok_stride) = src[stid + kStateThreads * k];
+                }
+            }
+            fence_proxy_async();  // the next TMA into this stage overwrites this region
+            group_sync(kBarState, kStateThreads);
+            drained = true;
+            // stage s is free: refill it with the chunk two ahead
+            if (have_ahead) {
+                fill(ahead, s, ns + 1);
+                have_ahead = item_next(a, total, ahead);
+            }
         }
-        u = next_nonempty(a, u + gridDim.x, total);
+        if (stid == 0 && !drained) {
+            mma_commit(drain_s);
+            mbar_wait(drain_s, 0, kWaitNs / 4);
+        }
+        // TMA loads the prep group never consumed (only after an abort)
+        if (stid == 0 && *abort_flag)
+            for (int x = 0; x < 2; ++x)
+                if ((issued >> x) & 1u) mbar_wait(&full[x], (issued_par >> x) & 1u, kWaitNs / 4);
     }
 
-    // ---- drain TMA copies still in flight (bounded), free TMEM
-    if (tid == 0) {
-        for (int s = 0; s < 2; ++s)
-            if ((inflight >> s) & 1u) mbar_wait(&full[s], (full_phase >> s) & 1u, kWaitNs);
-    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
