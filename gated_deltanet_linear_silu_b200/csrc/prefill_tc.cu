@@ -87,9 +87,11 @@ static_assert(kOffA % 1024 == 0 && kOffSA % 1024 == 0 && kOffP % 1024 == 0, "swi
 
 // TMEM columns (fp32, 128 lanes).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kRS = 0, kRO = 128, kRU = 256, kRA = 384, kRW = 448;  // R_O, R_U: 2 x 64
+// R_O, R_U: 2 x 64 columns each. R_A holds the 128 x 128 Gram matrix [Q;K][Q;K]^T and is
+// reused for W^T once the P/A epilogue has read it.
+constexpr uint32_t kRS = 0, kRO = 128, kRU = 256, kRA = 384, kRW = 384;
 
-constexpr uint32_t kIdescA = idesc_bf16(128, 64, 0, 0);    // [Q;K] K^T
+constexpr uint32_t kIdescA = idesc_bf16(128, 128, 0, 0);   // [Q;K] [Q;K]^T (Gram)
 constexpr uint32_t kIdescMN = idesc_bf16(128, 64, 1, 1);   // K^T T1^T, V^T T2^T
 constexpr uint32_t kIdescSW = idesc_bf16(128, 64, 0, 1);   // S^T (-W^T)
 constexpr uint32_t kIdescSQ = idesc_bf16(128, 64, 0, 0);   // S^T Q~^T, U^T P^T
@@ -136,21 +138,6 @@ __device__ __forceinline__ void scale_row(uint8_t* tile, int row, float f) {
         unpack_bf16(u.w, a, b); u.w = pack_bf16(a * f, b * f);
         *p = u;
     }
-}
-
-// Sum of squares of a 128-byte bf16 row (order of chunks irrelevant).
-__device__ __forceinline__ float row_sumsq(const uint8_t* tile, int row) {
-    float s = 0.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint4 u = *reinterpret_cast<const uint4*>(tile + sw128_off(row, c));
-        float a, b;
-        unpack_bf16(u.x, a, b); s = fmaf(a, a, s); s = fmaf(b, b, s);
-        unpack_bf16(u.y, a, b); s = fmaf(a, a, s); s = fmaf(b, b, s);
-        unpack_bf16(u.z, a, b); s = fmaf(a, a, s); s = fmaf(b, b, s);
-        unpack_bf16(u.w, a, b); s = fmaf(a, a, s); s = fmaf(b, b, s);
-    }
-    return s;
 }
 
 struct Unit {
@@ -259,8 +246,8 @@ struct Smem {
     uint8_t* base;
     __device__ uint8_t* stage(int s) const { return base + s * kStageBytes; }
     __device__ float* vec(int s) const { return reinterpret_cast<float*>(base + kOffVec + s * kVecBytes); }
-    // vec layout: [0,64) g raw, [64,128) beta raw, [128,192) gamma, [192,256) beta,
-    // [256,320) rq, [320,384) rk
+    // vec layout: [128,192) gamma, [192,256) beta (written by the refill),
+    // [256,320) rq, [320,384) rk (written by the prep group)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -349,47 +336,16 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
             }
 
-            // ---- per-row scalars: cumulative decay, L2 norms (q: tid < 64, k: 64..127)
-            if (ptid < 64) {
-                const int r = ptid;
-                float fq = 0.f;
-                if (r < L) {
-                    const float ss = row_sumsq(st + kQb0, r) + row_sumsq(st + kQb1, r);
-                    fq = (a.qk_l2norm ? 1.f / sqrtf(ss + a.eps) : 1.f) * a.scale;
-                }
-                float x = vec[r];  // g (0 past L); inclusive scan over 64 rows (two warps)
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, o);
-                    if (lane >= o) x += y;
-                }
-                if (ptid == 31) *carry = x;
-                bet[r] = vec[64 + r];
-                rq[r] = fq;
-                gam[r] = x;
-            } else if (ptid < 128) {
-                const int r = ptid - 64;
-                float fk = 0.f;
-                if (r < L) {
-                    const float ss = row_sumsq(st + kKb0, r) + row_sumsq(st + kKb1, r);
-                    fk = a.qk_l2norm ? 1.f / sqrtf(ss + a.eps) : 1.f;
-                }
-                rk[r] = fk;
-            }
-            group_sync(kBarPrep, kPrepThreads);
-            if (ptid >= 32 && ptid < 64) gam[ptid] += *carry;
-            group_sync(kBarPrep, kPrepThreads);
-            const float gL = gam[63];
-
-            // ---- [Q;K] K^T -> R_A
+            // ---- Gram matrix G = [Q;K][Q;K]^T -> R_A (128 x 128). Its diagonal gives
+            // the squared norms of the q and k rows; its lower-right 64 x 64 block is
+            // K K^T and its upper-right block Q K^T.
             if (ptid == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t qo = (k < 4 ? kQb0 : kQb1) + 32 * (k & 3);
-                    const uint32_t ko = (k < 4 ? kKb0 : kKb1) + 32 * (k & 3);
-                    mma_bf16(tmem + kRA, sw128_desc(smem_u32(st + qo), 16, 1024),
-                             sw128_desc(smem_u32(st + ko), 16, 1024), kIdescA, k > 0);
+                    const uint64_t d = sw128_desc(smem_u32(st + qo), 16, 1024);  // 128 rows: Q then K
+                    mma_bf16(tmem + kRA, d, d, kIdescA, k > 0);
                 }
                 mma_commit(pa_bar);
             }
@@ -402,13 +358,31 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 pa_phase ^= 1;
             }
             tc_fence_after();
+            // L2-norm factors of row `row` from G[row][row] (half-0 threads), beta copied
+            {
+                float dg[32];
+                tmem_ld32(tmem + lane_off + kRA + 32 * (warp & 3), dg);
+                tmem_wait_ld();
+                if (half == 0) {
+                    float d2 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) d2 = (e == lane) ? dg[e] : d2;
+                    const int r = row & 63;
+                    float f = 0.f;
+                    if (r < L) f = a.qk_l2norm ? 1.f / sqrtf(d2 + a.eps) : 1.f;
+                    if (row < 64) rq[r] = f * a.scale;
+                    else rk[r] = f;
+                }
+            }
+            group_sync(kBarPrep, kPrepThreads);
+            const float gL = gam[63];
 
             // ---- P rows (lanes < 64) and A rows (lanes >= 64), 32 columns per
             // thread. Branch-free: every element is computed (exponent clamped
             // at 0 so the masked-out upper triangle cannot overflow), then selected.
             {
                 float x[32];
-                tmem_ld32(tmem + lane_off + kRA + 32 * half, x);
+                tmem_ld32(tmem + lane_off + kRA + 64 + 32 * half, x);  // columns = k rows
                 tmem_wait_ld();
                 const int j0 = 32 * half;
                 if (row < 64) {
@@ -609,20 +583,35 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             const int64_t base = ((int64_t)U.n * H + U.h) * kD * kD;
             for (int x = stid; x < kD * kD; x += kStateThreads) a.hT[base + x] = a.h0 ? a.h0[base + x] : 0.f;
         }
-        // Fill stage s with item `f`: gates by threads 0..63, then the leader
-        // arms the stage barrier and issues the six TMA tile loads.
+        // Refill of stage s with item `f`: the gates (loaded earlier into registers
+        // by threads 0..63, row = stid) become beta and the cumulative decay gamma
+        // in the stage's vector block; then the leader arms the stage barrier and
+        // issues the six TMA tile loads.
         uint32_t issued = 0, issued_par = 0;  // for the bounded drain at exit
-        auto fill = [&](const Item& f, int s, int use) {
+        auto load_gates = [&](const Item& f, float& g, float& b) {
+            g = 0.f;
+            b = 0.f;
+            if (stid < 64 && stid < f.L) {
+                g = a.g[(f.c0 + stid) * H + f.U.h];
+                b = a.beta[(f.c0 + stid) * H + f.U.h];
+            }
+        };
+        auto fill = [&](const Item& f, int s, int use, float g, float b) {
             float* v = S.vec(s);
+            float x = g;  // inclusive scan over the 64 rows (warps 8 and 9)
             if (stid < 64) {
-                const int r = stid;
-                float g = 0.f, b = 0.f;
-                if (r < f.L) {
-                    g = a.g[(f.c0 + r) * H + f.U.h];
-                    b = a.beta[(f.c0 + r) * H + f.U.h];
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
                 }
-                v[r] = g;
-                v[64 + r] = b;
+                if (stid == 31) *carry = x;
+            }
+            group_sync(kBarState, kStateThreads);
+            if (stid < 64) {
+                if (stid >= 32) x += *carry;
+                v[128 + stid] = x;  // gamma
+                v[192 + stid] = b;  // beta
             }
             group_sync(kBarState, kStateThreads);
             if (stid == 0) {
@@ -639,12 +628,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         Item it, ahead;
         bool have = item_first(a, total, it);
         bool have_ahead = have;
+        float g_ahead = 0.f, b_ahead = 0.f;  // gates of item `ahead`, prefetched
         if (have) {
             ahead = it;
-            fill(ahead, 0, 0);
+            load_gates(ahead, g_ahead, b_ahead);
+            fill(ahead, 0, 0, g_ahead, b_ahead);
             have_ahead = item_next(a, total, ahead);
             if (have_ahead) {
-                fill(ahead, 1, 0);
+                load_gates(ahead, g_ahead, b_ahead);
+                fill(ahead, 1, 0, g_ahead, b_ahead);
                 have_ahead = item_next(a, total, ahead);  // ahead = item 2
             }
         }
@@ -656,6 +648,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             uint8_t* st = S.stage(s);
             const float* vec = S.vec(s);
             const int64_t sbase = ((int64_t)it.U.n * H + it.U.h) * kD * kD;
+            if (have_ahead) load_gates(ahead, g_ahead, b_ahead);  // used by the refill at the end
             if (it.first) {
                 // initial state: R_S (fp32) and S^T (bf16 A operand); thread = dv lane j
                 const float* h0p = a.h0 ? a.h0 + sbase + j : nullptr;  // column j of S
@@ -819,7 +812,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             drained = true;
             // stage s is free: refill it with the chunk two ahead
             if (have_ahead) {
-                fill(ahead, s, ns + 1);
+                fill(ahead, s, ns + 1, g_ahead, b_ahead);
                 have_ahead = item_next(a, total, ahead);
             }
         }
