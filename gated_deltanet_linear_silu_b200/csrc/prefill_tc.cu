@@ -140,6 +140,34 @@ __device__ __forceinline__ void scale_row(uint8_t* tile, int row, float f) {
     }
 }
 
+// Warp-level m16n8k8 TF32 tensor-core product (fp32 accumulate) used by the
+// merges of the triangular solve: d(16x8) += A(16x8) * B(8x8), both read from
+// fp32 shared memory (A row-major with stride lda, B row-major k x n with
+// stride ldb) and rounded to tf32.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const float* A, int lda, const float* B,
+                                                int ldb) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t a0 = to_tf32(A[g * lda + t]), a1 = to_tf32(A[(g + 8) * lda + t]);
+    const uint32_t a2 = to_tf32(A[g * lda + t + 4]), a3 = to_tf32(A[(g + 8) * lda + t + 4]);
+    const uint32_t b0 = to_tf32(B[t * ldb + g]), b1 = to_tf32(B[(t + 4) * ldb + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Store the 16x8 accumulator tile (times f) row-major with stride ld.
+__device__ __forceinline__ void store_acc_16x8(float* D, int ld, const float (&d)[4], float f) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2*>(D + g * ld + 2 * t) = make_float2(f * d[0], f * d[1]);
+    *reinterpret_cast<float2*>(D + (g + 8) * ld + 2 * t) = make_float2(f * d[2], f * d[3]);
+}
+
 struct Unit {
     int n, h;
     int64_t start, end;
@@ -252,7 +280,8 @@ struct Smem {
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap map_q,
-                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
+                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                  const __grid_constant__ CUtensorMap map_o) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the shared-window address (swizzle atoms, TMA).
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -281,7 +310,6 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     uint64_t* drain_s = bars + 12;  // exit: all state MMAs done
     uint32_t* tmem_base_p = reinterpret_cast<uint32_t*>(sm + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
-    float* carry = reinterpret_cast<float*>(sm + kOffMisc + 8);
 
     if (tid == 0) {
         mbar_init(&full[0], 1);
@@ -452,57 +480,40 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 for (int e = ptid - 192; e < 32 * 32; e += 64) sT[(e >> 5) * kLdA + 32 + (e & 31)] = 0.f;
             }
             group_sync(kBarPrep, kPrepThreads);
-            {
-                // 16 -> 32 for the block pairs at o = 0 and 32: thread -> 1 row x 2 columns
-                const int o = 32 * (ptid >> 7), idx = ptid & 127;
-                const int r = idx >> 3, cc = 2 * (idx & 7);
-                float y0 = 0.f, y1 = 0.f;
+            // 16 -> 32 for the block pairs at o = 0 and 32 (warps 0-3: pair, 8-column tile):
+            // Y = A_10 T_00 into the unused upper-right block of A, then T_10 = -T_11 Y.
+            if (warp < 4) {
+                const int o = 32 * (warp >> 1), nt = 8 * (warp & 1);
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float2 t2 = *reinterpret_cast<const float2*>(sT + (o + m) * kLdA + o + cc);
-                    const float av = sA[(o + 16 + r) * kLdA + o + m];
-                    y0 = fmaf(av, t2.x, y0);
-                    y1 = fmaf(av, t2.y, y1);
-                }
-                group_sync(kBarPrep, kPrepThreads);  // A_10 blocks fully read
-                *reinterpret_cast<float2*>(sA + (o + 16 + r) * kLdA + o + cc) = make_float2(y0, y1);
-                group_sync(kBarPrep, kPrepThreads);
-                float z0 = 0.f, z1 = 0.f;
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_tf32_16x8x8(d, sA + (o + 16) * kLdA + o + 8 * ks, kLdA, sT + (o + 8 * ks) * kLdA + o + nt, kLdA);
+                float* Y = sA + o * kLdA + o + 16;  // 16 x 16 scratch, row-major
+                store_acc_16x8(Y + nt, kLdA, d, 1.f);
+                __syncwarp();
+                float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float2 y2 = *reinterpret_cast<const float2*>(sA + (o + 16 + m) * kLdA + o + cc);
-                    const float tv = sT[(o + 16 + r) * kLdA + o + 16 + m];
-                    z0 = fmaf(tv, y2.x, z0);
-                    z1 = fmaf(tv, y2.y, z1);
-                }
-                *reinterpret_cast<float2*>(sT + (o + 16 + r) * kLdA + o + cc) = make_float2(-z0, -z1);
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_tf32_16x8x8(z, sT + (o + 16) * kLdA + o + 16 + 8 * ks, kLdA, Y + 8 * ks * kLdA + nt, kLdA);
+                store_acc_16x8(sT + (o + 16) * kLdA + o + nt, kLdA, z, -1.f);
             }
             group_sync(kBarPrep, kPrepThreads);
             {
-                // 32 -> 64: Y = A_10 T_00 then T_10 = -T_11 Y; thread -> 2 rows x 2 columns
-                const int r0 = 2 * (ptid >> 4), c0b = 2 * (ptid & 15);
-                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 8
-                for (int m = 0; m < 32; ++m) {
-                    const float2 t2 = *reinterpret_cast<const float2*>(sT + m * kLdA + c0b);
-                    const float a0 = sA[(32 + r0) * kLdA + m], a1 = sA[(33 + r0) * kLdA + m];
-                    y00 = fmaf(a0, t2.x, y00); y01 = fmaf(a0, t2.y, y01);
-                    y10 = fmaf(a1, t2.x, y10); y11 = fmaf(a1, t2.y, y11);
-                }
-                group_sync(kBarPrep, kPrepThreads);  // A_10 fully read
-                *reinterpret_cast<float2*>(sA + (32 + r0) * kLdA + c0b) = make_float2(y00, y01);
-                *reinterpret_cast<float2*>(sA + (33 + r0) * kLdA + c0b) = make_float2(y10, y11);
+                // 32 -> 64 (all 8 warps: 16-row x 8-column tile each): Y = A_10 T_00 into the
+                // unused upper-right 32 x 32 block of A, then T_10 = -T_11 Y.
+                const int mt = 16 * (warp & 1), nt = 8 * (warp >> 1);
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_tf32_16x8x8(d, sA + (32 + mt) * kLdA + 8 * ks, kLdA, sT + 8 * ks * kLdA + nt, kLdA);
+                float* Y = sA + 32;  // rows 0..31, columns 32..63 of A
+                store_acc_16x8(Y + mt * kLdA + nt, kLdA, d, 1.f);
                 group_sync(kBarPrep, kPrepThreads);
-                float z00 = 0.f, z01 = 0.f, z10 = 0.f, z11 = 0.f;
-#pragma unroll 8
-                for (int m = 0; m < 32; ++m) {
-                    const float2 y2 = *reinterpret_cast<const float2*>(sA + (32 + m) * kLdA + c0b);
-                    const float t0 = sT[(32 + r0) * kLdA + 32 + m], t1 = sT[(33 + r0) * kLdA + 32 + m];
-                    z00 = fmaf(t0, y2.x, z00); z01 = fmaf(t0, y2.y, z01);
-                    z10 = fmaf(t1, y2.x, z10); z11 = fmaf(t1, y2.y, z11);
-                }
-                *reinterpret_cast<float2*>(sT + (32 + r0) * kLdA + c0b) = make_float2(-z00, -z01);
-                *reinterpret_cast<float2*>(sT + (33 + r0) * kLdA + c0b) = make_float2(-z10, -z11);
+                float z[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_tf32_16x8x8(z, sT + (32 + mt) * kLdA + 32 + 8 * ks, kLdA, Y + 8 * ks * kLdA + nt, kLdA);
+                store_acc_16x8(sT + (32 + mt) * kLdA + nt, kLdA, z, -1.f);
             }
             group_sync(kBarPrep, kPrepThreads);
             // T1^T, T2^T rows (row m = column m of T) as bf16 MN-major B operands,
@@ -583,38 +594,38 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             const int64_t base = ((int64_t)U.n * H + U.h) * kD * kD;
             for (int x = stid; x < kD * kD; x += kStateThreads) a.hT[base + x] = a.h0 ? a.h0[base + x] : 0.f;
         }
-        // Refill of stage s with item `f`: the gates (loaded earlier into registers
-        // by threads 0..63, row = stid) become beta and the cumulative decay gamma
-        // in the stage's vector block; then the leader arms the stage barrier and
-        // issues the six TMA tile loads.
+        // Refill of stage s with item `f`, by the state group's first warp: the gates
+        // (prefetched into registers, rows 2*lane and 2*lane+1) become beta and the
+        // cumulative decay gamma in the stage's vector block; then lane 0 arms the
+        // stage barrier and issues the six TMA tile loads (after any TMA store of O
+        // out of this stage has finished reading it).
         uint32_t issued = 0, issued_par = 0;  // for the bounded drain at exit
-        auto load_gates = [&](const Item& f, float& g, float& b) {
-            g = 0.f;
-            b = 0.f;
-            if (stid < 64 && stid < f.L) {
-                g = a.g[(f.c0 + stid) * H + f.U.h];
-                b = a.beta[(f.c0 + stid) * H + f.U.h];
+        auto load_gates = [&](const Item& f, float4& gb) {
+            gb = make_float4(0.f, 0.f, 0.f, 0.f);  // g(2l), g(2l+1), beta(2l), beta(2l+1)
+            if (stid < 32) {
+                const int r = 2 * stid;
+                if (r < f.L) { gb.x = a.g[(f.c0 + r) * H + f.U.h]; gb.z = a.beta[(f.c0 + r) * H + f.U.h]; }
+                if (r + 1 < f.L) { gb.y = a.g[(f.c0 + r + 1) * H + f.U.h]; gb.w = a.beta[(f.c0 + r + 1) * H + f.U.h]; }
             }
         };
-        auto fill = [&](const Item& f, int s, int use, float g, float b) {
+        auto fill = [&](const Item& f, int s, int use, const float4& gb) {
+            if (stid >= 32) return;
             float* v = S.vec(s);
-            float x = g;  // inclusive scan over the 64 rows (warps 8 and 9)
-            if (stid < 64) {
+            const float pair = gb.x + gb.y;
+            float x = pair;  // inclusive scan of the row-pair sums over the warp
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, o);
-                    if (lane >= o) x += y;
-                }
-                if (stid == 31) *carry = x;
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
             }
-            group_sync(kBarState, kStateThreads);
-            if (stid < 64) {
-                if (stid >= 32) x += *carry;
-                v[128 + stid] = x;  // gamma
-                v[192 + stid] = b;  // beta
-            }
-            group_sync(kBarState, kStateThreads);
+            const int r = 2 * stid;
+            v[128 + r] = x - pair + gb.x;  // gamma
+            v[128 + r + 1] = x;
+            v[192 + r] = gb.z;             // beta
+            v[192 + r + 1] = gb.w;
+            __syncwarp();
             if (stid == 0) {
+                bulk_wait_group_read0();
                 issue_tiles(S.stage(s), &full[s], &map_q, &map_k, &map_v, f.U.h, f.c0);
                 issued |= 1u << s;
                 issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(use & 1) << s);
@@ -624,22 +635,24 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             prefetch_tmap(&map_q);
             prefetch_tmap(&map_k);
             prefetch_tmap(&map_v);
+            prefetch_tmap(&map_o);
         }
         Item it, ahead;
         bool have = item_first(a, total, it);
         bool have_ahead = have;
-        float g_ahead = 0.f, b_ahead = 0.f;  // gates of item `ahead`, prefetched
+        float4 gb_ahead;  // gates of item `ahead`, prefetched
         if (have) {
             ahead = it;
-            load_gates(ahead, g_ahead, b_ahead);
-            fill(ahead, 0, 0, g_ahead, b_ahead);
+            load_gates(ahead, gb_ahead);
+            fill(ahead, 0, 0, gb_ahead);
             have_ahead = item_next(a, total, ahead);
             if (have_ahead) {
-                load_gates(ahead, g_ahead, b_ahead);
-                fill(ahead, 1, 0, g_ahead, b_ahead);
+                load_gates(ahead, gb_ahead);
+                fill(ahead, 1, 0, gb_ahead);
                 have_ahead = item_next(a, total, ahead);  // ahead = item 2
             }
         }
+        group_sync(kBarState, kStateThreads);  // the refills' gamma/beta are read by all state warps
         bool drained = true;
         for (int i = 0; have; ++i, have = item_next(a, total, it)) {
             const int s = i & 1, ns = i >> 1;
@@ -648,10 +661,13 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             uint8_t* st = S.stage(s);
             const float* vec = S.vec(s);
             const int64_t sbase = ((int64_t)it.U.n * H + it.U.h) * kD * kD;
-            if (have_ahead) load_gates(ahead, g_ahead, b_ahead);  // used by the refill at the end
+            if (have_ahead) load_gates(ahead, gb_ahead);  // used by the refill at the end
             if (it.first) {
-                // initial state: R_S (fp32) and S^T (bf16 A operand); thread = dv lane j
+                // initial state: S^T as the bf16 A operand (thread = dv lane j) and, in
+                // TMEM, e^{gamma_L} S^T -- R_S always holds the state pre-decayed by the
+                // coming chunk, ready for the accumulation of K~^T U.
                 const float* h0p = a.h0 ? a.h0 + sbase + j : nullptr;  // column j of S
+                const float eL = expf(vec[128 + 63]);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     float v[32];
@@ -662,16 +678,12 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = 0.f;
                     }
+                    store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] *= eL;
                     tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
                 }
                 tmem_wait_st();
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
-                    tmem_wait_ld();
-                    store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
-                }
                 fence_proxy_async();
                 tc_fence_before();
                 group_sync(kBarState, kStateThreads);
@@ -702,20 +714,6 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     mma_bf16(tmem + kRO + 64 * s, sa, sw128_desc(smem_u32(st + qo), 16, 1024), kIdescSQ,
                              k > 0);
                 }
-            }
-            // R_S <- e^{gamma_L} R_S while MMA1 runs (MMA1 does not touch R_S)
-            {
-                const float eL = expf(vec[128 + 63]);
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= eL;
-                    tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
-                }
-                tmem_wait_st();
             }
             {
                 const bool ok = mbar_wait_or_abort(u_bar, ph, abort_flag);
@@ -759,18 +757,30 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
             }
             tc_fence_after();
-            // ---- new state: bf16 S^T for the next chunk's MMA1; final state at the end
+            // ---- new state: bf16 S^T for the next chunk's MMA1, and R_S pre-decayed
+            // by the next chunk's e^{gamma_L} (its gates are already in the other
+            // stage's vector block); the final state at the end of a sequence.
+            {
+                const float eL = it.last ? 1.f : expf(S.vec(s ^ 1)[128 + 63]);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                float v[32];
-                tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
-                tmem_wait_ld();
-                store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
-                if (it.last && a.hT) {
-                    float* hTp = a.hT + sbase + j + 32 * cc * kD;
+                for (int cc = 0; cc < 4; ++cc) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
+                    tmem_wait_ld();
+                    store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
+                    if (it.last) {
+                        if (a.hT) {
+                            float* hTp = a.hT + sbase + j + 32 * cc * kD;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) hTp[e * kD] = v[e];
+                            for (int e = 0; e < 32; ++e) hTp[e * kD] = v[e];
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] *= eL;
+                        tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
+                    }
                 }
+                tmem_wait_st();
             }
             fence_proxy_async();
             {
@@ -782,40 +792,53 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             }
             tc_fence_after();
             ph ^= 1;
-            // ---- O: column j of O^T -> O tile [64 tokens][128] bf16 staged in this
-            // stage's V region (V is dead after the prep's MMA), then written out as
-            // coalesced 16-byte rows, only the chunk's L valid tokens.
+            // ---- O: column j of O^T -> O tile staged in this stage's V region (V is
+            // dead after the prep's MMA) as two [64 tokens][64 d_v] row-major boxes;
+            // a full chunk leaves by one TMA store, a partial one as 16-byte rows of
+            // its L valid tokens.
+            {
+                uint16_t* ostage = reinterpret_cast<uint16_t*>(st + kVb0) + (j >> 6) * 4096 + (j & 63);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float x[32];
-                tmem_ld32(tmem + lane_off + kRO + 64 * s + 32 * hf, x);
-                tmem_wait_ld();
-                uint16_t* ostage = reinterpret_cast<uint16_t*>(st + kVb0);
+                for (int hf = 0; hf < 2; ++hf) {
+                    float x[32];
+                    tmem_ld32(tmem + lane_off + kRO + 64 * s + 32 * hf, x);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) ostage[(32 * hf + e) * kD + j] = f32_to_bf16(x[e]);
+                    for (int e = 0; e < 32; ++e) ostage[(32 * hf + e) * 64] = f32_to_bf16(x[e]);
+                }
             }
+            fence_proxy_async();
             tc_fence_before();
             group_sync(kBarState, kStateThreads);
-            {
-                const uint4* src = reinterpret_cast<const uint4*>(st + kVb0);
-                // vector vid = stid + 128 k covers token r = 8 k + stid / 16, 16-byte column stid % 16
-                uint16_t* orow = static_cast<uint16_t*>(a.o) + (c0 * H + it.U.h) * kD + 8 * (stid & 15);
+            if (L == kC) {
+                if (stid == 0) {
+                    tma_store_3d(&map_o, st + kVb0, 0, it.U.h, (int)c0);
+                    tma_store_3d(&map_o, st + kVb1, 64, it.U.h, (int)c0);
+                    bulk_commit_group();
+                }
+            } else {
+                uint16_t* obase = static_cast<uint16_t*>(a.o) + (c0 * H + it.U.h) * kD;
                 const int64_t tok_stride = (int64_t)H * kD;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const int r = 8 * k + (stid >> 4);
-                    if (r < L) *reinterpret_cast<uint4*>(orow + r * tok_stride) = src[stid + kStateThreads * k];
+                    const int vid = stid + kStateThreads * k;  // token r, 16-byte column c16
+                    const int r = vid >> 4, c16 = vid & 15;
+                    if (r < L) {
+                        const uint8_t* src = st + kVb0 + (c16 >> 3) * 8192 + r * 128 + (c16 & 7) * 16;
+                        *reinterpret_cast<uint4*>(obase + r * tok_stride + 8 * c16) =
+                            *reinterpret_cast<const uint4*>(src);
+                    }
                 }
+                group_sync(kBarState, kStateThreads);  // staging read before the refill
             }
-            fence_proxy_async();  // the next TMA into this stage overwrites this region
-            group_sync(kBarState, kStateThreads);
             drained = true;
             // stage s is free: refill it with the chunk two ahead
             if (have_ahead) {
-                fill(ahead, s, ns + 1, g_ahead, b_ahead);
+                fill(ahead, s, ns + 1, gb_ahead);
                 have_ahead = item_next(a, total, ahead);
             }
         }
+        if (stid == 0) bulk_wait_group0();  // O stores issued by this thread
         if (stid == 0 && !drained) {
             mma_commit(drain_s);
             mbar_wait(drain_s, 0, kWaitNs / 4);
@@ -848,8 +871,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [T_tot, H, 128] bf16 viewed as a 3-D tensor (feature, head, token); boxes of
-// 64 features x 1 head x 64 tokens, 128-byte swizzle, zero fill past T_tot.
-bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t T) {
+// 64 features x 1 head x 64 tokens, zero fill past T_tot on loads, clipped on
+// stores. Loads use the 128-byte swizzle the MMA descriptors expect; the O
+// store reads a plain row-major staging tile.
+bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t T, bool swizzle) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T};
@@ -857,7 +882,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t T) {
     cuuint32_t box[3] = {64, 1, 64};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -869,9 +895,9 @@ bool prefill_tc_supported(const PrefillArgs& a) {
 }
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, a.H, a.T_tot) || !make_map(&mk, a.k, a.H, a.T_tot) ||
-        !make_map(&mv, a.v, a.H, a.T_tot))
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, a.q, a.H, a.T_tot, true) || !make_map(&mk, a.k, a.H, a.T_tot, true) ||
+        !make_map(&mv, a.v, a.H, a.T_tot, true) || !make_map(&mo, a.o, a.H, a.T_tot, false))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemAlloc);
@@ -882,7 +908,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sms ? units : sms);
     TcParams p{a};
-    prefill_tc_kernel<<<grid, kThreads, kSmemAlloc, s>>>(p, mq, mk, mv);
+    prefill_tc_kernel<<<grid, kThreads, kSmemAlloc, s>>>(p, mq, mk, mv, mo);
     return cudaGetLastError();
 }
 
