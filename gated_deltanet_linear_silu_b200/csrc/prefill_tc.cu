@@ -597,8 +597,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         // Refill of stage s with item `f`, by the state group's first warp: the gates
         // (prefetched into registers, rows 2*lane and 2*lane+1) become beta and the
         // cumulative decay gamma in the stage's vector block; then lane 0 arms the
-        // stage barrier and issues the six TMA tile loads (after any TMA store of O
-        // out of this stage has finished reading it).
+        // stage barrier and issues the six TMA tile loads.
         uint32_t issued = 0, issued_par = 0;  // for the bounded drain at exit
         auto load_gates = [&](const Item& f, float4& gb) {
             gb = make_float4(0.f, 0.f, 0.f, 0.f);  // g(2l), g(2l+1), beta(2l), beta(2l+1)
@@ -625,7 +624,6 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             v[192 + r + 1] = gb.w;
             __syncwarp();
             if (stid == 0) {
-                bulk_wait_group_read0();
                 issue_tiles(S.stage(s), &full[s], &map_q, &map_k, &map_v, f.U.h, f.c0);
                 issued |= 1u << s;
                 issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(use & 1) << s);
@@ -715,6 +713,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                              k > 0);
                 }
             }
+            if (stid == 0) bulk_wait_group_read0();  // previous O store has read U^T
             {
                 const bool ok = mbar_wait_or_abort(u_bar, ph, abort_flag);
                 if (group_any(kBarState, kStateThreads, !ok)) {
@@ -792,12 +791,12 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             }
             tc_fence_after();
             ph ^= 1;
-            // ---- O: column j of O^T -> O tile staged in this stage's V region (V is
-            // dead after the prep's MMA) as two [64 tokens][64 d_v] row-major boxes;
-            // a full chunk leaves by one TMA store, a partial one as 16-byte rows of
-            // its L valid tokens.
+            // ---- O: column j of O^T -> O tile staged in the U^T tile (dead until the
+            // next chunk's U epilogue) as two [64 tokens][64 d_v] row-major boxes; a
+            // full chunk leaves by one TMA store, a partial one as 16-byte rows of its
+            // L valid tokens.
             {
-                uint16_t* ostage = reinterpret_cast<uint16_t*>(st + kVb0) + (j >> 6) * 4096 + (j & 63);
+                uint16_t* ostage = reinterpret_cast<uint16_t*>(sUT) + (j >> 6) * 4096 + (j & 63);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float x[32];
@@ -812,8 +811,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             group_sync(kBarState, kStateThreads);
             if (L == kC) {
                 if (stid == 0) {
-                    tma_store_3d(&map_o, st + kVb0, 0, it.U.h, (int)c0);
-                    tma_store_3d(&map_o, st + kVb1, 64, it.U.h, (int)c0);
+                    tma_store_3d(&map_o, sUT, 0, it.U.h, (int)c0);
+                    tma_store_3d(&map_o, sUT + 8192, 64, it.U.h, (int)c0);
                     bulk_commit_group();
                 }
             } else {
@@ -824,12 +823,12 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     const int vid = stid + kStateThreads * k;  // token r, 16-byte column c16
                     const int r = vid >> 4, c16 = vid & 15;
                     if (r < L) {
-                        const uint8_t* src = st + kVb0 + (c16 >> 3) * 8192 + r * 128 + (c16 & 7) * 16;
+                        const uint8_t* src = sUT + (c16 >> 3) * 8192 + r * 128 + (c16 & 7) * 16;
                         *reinterpret_cast<uint4*>(obase + r * tok_stride + 8 * c16) =
                             *reinterpret_cast<const uint4*>(src);
                     }
                 }
-                group_sync(kBarState, kStateThreads);  // staging read before the refill
+                group_sync(kBarState, kStateThreads);  // staging read before U^T is rewritten
             }
             drained = true;
             // stage s is free: refill it with the chunk two ahead
