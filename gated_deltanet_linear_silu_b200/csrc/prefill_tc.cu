@@ -32,9 +32,11 @@
 //               Q~ and K~ -- for chunk c+1 ...
 //   warps 8-11  state group: ... while these run the state chain of chunk c
 //               (U, the state update, O) with the state resident in TMEM. When
-//               the state group is done with a stage of the two-stage ring it
-//               refills it (TMA for the q/k/v tiles, plain loads for the gates)
-//               with the chunk two ahead.
+//               the state group is done with a stage of the two-stage ring one
+//               of its lanes refills it by TMA with the chunk two ahead.
+// The prep group's first warp turns a chunk's gates into beta and the cumulative
+// decay gamma while the Gram MMA runs and signals the state group, which needs
+// only gamma_L (to pre-decay its state for the coming chunk).
 // The groups hand off through mbarriers; TMEM holds double-buffered U~/U
 // and O regions so the prep of c+1 never waits for the epilogues of c.
 // Every wait is bounded: on timeout the kernel records the timeout status,
@@ -274,7 +276,7 @@ struct Smem {
     uint8_t* base;
     __device__ uint8_t* stage(int s) const { return base + s * kStageBytes; }
     __device__ float* vec(int s) const { return reinterpret_cast<float*>(base + kOffVec + s * kVecBytes); }
-    // vec layout: [128,192) gamma, [192,256) beta (written by the refill),
+    // vec layout: [128,192) gamma, [192,256) beta (written by the prep group's first warp),
     // [256,320) rq, [320,384) rk (written by the prep group)
 };
 
@@ -299,7 +301,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     float* sA = reinterpret_cast<float*>(sm + kOffA);
     float* sT = reinterpret_cast<float*>(sm + kOffTf);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
-    uint64_t* full = bars + 0;      // [2] tiles + gates of a stage landed (state -> prep)
+    uint64_t* full = bars + 0;      // [2] q/k/v tiles of a stage landed (TMA -> prep)
+    uint64_t* gready = bars + 2;    // [2] gamma/beta of a stage written (prep -> state)
     uint64_t* pdone = bars + 4;     // [2] prep -> state        (count 1)
     uint64_t* pa_bar = bars + 6;    // prep MMA completions
     uint64_t* u_bar = bars + 7;     // state MMA1 (U) completion
@@ -314,6 +317,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
+        mbar_init(&gready[0], 1);
+        mbar_init(&gready[1], 1);
         mbar_init(&pdone[0], 1);
         mbar_init(&pdone[1], 1);
         mbar_init(pa_bar, 1);
@@ -356,6 +361,16 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             float* rq = vec + 256;
             float* rk = vec + 320;
             uint8_t* sP = sm + kOffP + s * 8192;
+            // gates g, beta of rows 2*lane and 2*lane+1 (first warp), in flight
+            // across the tile wait and the Gram MMA
+            float4 gb = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (warp == 0) {
+                const int r = 2 * lane;
+                const float* gp = a.g + (it.c0 + r) * H + it.U.h;
+                const float* bp = a.beta + (it.c0 + r) * H + it.U.h;
+                if (r < L) { gb.x = gp[0]; gb.z = bp[0]; }
+                if (r + 1 < L) { gb.y = gp[H]; gb.w = bp[H]; }
+            }
             {
                 const bool ok = mbar_wait_or_abort(&full[s], ns & 1, abort_flag);
                 if (group_any(kBarPrep, kPrepThreads, !ok)) {
@@ -376,6 +391,23 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     mma_bf16(tmem + kRA, d, d, kIdescA, k > 0);
                 }
                 mma_commit(pa_bar);
+            }
+            // gamma = inclusive prefix sum of g (scan of the row-pair sums over the
+            // warp) and beta into the stage's vector block; the state group waits
+            // for them on gready[s].
+            if (warp == 0) {
+                const float pair = gb.x + gb.y;
+                float x = pair;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x += y;
+                }
+                const int r = 2 * lane;
+                *reinterpret_cast<float2*>(gam + r) = make_float2(x - pair + gb.x, x);
+                *reinterpret_cast<float2*>(bet + r) = make_float2(gb.z, gb.w);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&gready[s]);
             }
             {
                 const bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag);
@@ -594,40 +626,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             const int64_t base = ((int64_t)U.n * H + U.h) * kD * kD;
             for (int x = stid; x < kD * kD; x += kStateThreads) a.hT[base + x] = a.h0 ? a.h0[base + x] : 0.f;
         }
-        // Refill of stage s with item `f`, by the state group's first warp: the gates
-        // (prefetched into registers, rows 2*lane and 2*lane+1) become beta and the
-        // cumulative decay gamma in the stage's vector block; then lane 0 arms the
-        // stage barrier and issues the six TMA tile loads.
+        // Refill of stage s with item `f`: one lane outside the MMA-issuing warp arms
+        // the stage barrier and issues the six TMA tile loads.
+        constexpr int kRefill = 32;
         uint32_t issued = 0, issued_par = 0;  // for the bounded drain at exit
-        auto load_gates = [&](const Item& f, float4& gb) {
-            gb = make_float4(0.f, 0.f, 0.f, 0.f);  // g(2l), g(2l+1), beta(2l), beta(2l+1)
-            if (stid < 32) {
-                const int r = 2 * stid;
-                if (r < f.L) { gb.x = a.g[(f.c0 + r) * H + f.U.h]; gb.z = a.beta[(f.c0 + r) * H + f.U.h]; }
-                if (r + 1 < f.L) { gb.y = a.g[(f.c0 + r + 1) * H + f.U.h]; gb.w = a.beta[(f.c0 + r + 1) * H + f.U.h]; }
-            }
-        };
-        auto fill = [&](const Item& f, int s, int use, const float4& gb) {
-            if (stid >= 32) return;
-            float* v = S.vec(s);
-            const float pair = gb.x + gb.y;
-            float x = pair;  // inclusive scan of the row-pair sums over the warp
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            const int r = 2 * stid;
-            v[128 + r] = x - pair + gb.x;  // gamma
-            v[128 + r + 1] = x;
-            v[192 + r] = gb.z;             // beta
-            v[192 + r + 1] = gb.w;
-            __syncwarp();
-            if (stid == 0) {
-                issue_tiles(S.stage(s), &full[s], &map_q, &map_k, &map_v, f.U.h, f.c0);
-                issued |= 1u << s;
-                issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(use & 1) << s);
-            }
+        auto fill = [&](const Item& f, int s, int use) {
+            if (stid != kRefill) return;
+            issue_tiles(S.stage(s), &full[s], &map_q, &map_k, &map_v, f.U.h, f.c0);
+            issued |= 1u << s;
+            issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(use & 1) << s);
         };
         if (stid == 0) {
             prefetch_tmap(&map_q);
@@ -638,19 +645,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         Item it, ahead;
         bool have = item_first(a, total, it);
         bool have_ahead = have;
-        float4 gb_ahead;  // gates of item `ahead`, prefetched
         if (have) {
             ahead = it;
-            load_gates(ahead, gb_ahead);
-            fill(ahead, 0, 0, gb_ahead);
+            fill(ahead, 0, 0);
             have_ahead = item_next(a, total, ahead);
             if (have_ahead) {
-                load_gates(ahead, gb_ahead);
-                fill(ahead, 1, 0, gb_ahead);
+                fill(ahead, 1, 0);
                 have_ahead = item_next(a, total, ahead);  // ahead = item 2
             }
         }
-        group_sync(kBarState, kStateThreads);  // the refills' gamma/beta are read by all state warps
         bool drained = true;
         for (int i = 0; have; ++i, have = item_next(a, total, it)) {
             const int s = i & 1, ns = i >> 1;
@@ -659,11 +662,17 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             uint8_t* st = S.stage(s);
             const float* vec = S.vec(s);
             const int64_t sbase = ((int64_t)it.U.n * H + it.U.h) * kD * kD;
-            if (have_ahead) load_gates(ahead, gb_ahead);  // used by the refill at the end
             if (it.first) {
                 // initial state: S^T as the bf16 A operand (thread = dv lane j) and, in
                 // TMEM, e^{gamma_L} S^T -- R_S always holds the state pre-decayed by the
                 // coming chunk, ready for the accumulation of K~^T U.
+                {
+                    const bool ok = mbar_wait_or_abort(&gready[s], ns & 1, abort_flag);
+                    if (group_any(kBarState, kStateThreads, !ok)) {
+                        if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
+                        break;
+                    }
+                }
                 const float* h0p = a.h0 ? a.h0 + sbase + j : nullptr;  // column j of S
                 const float eL = expf(vec[128 + 63]);
 #pragma unroll
@@ -749,7 +758,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 mma_commit(o_bar);
             }
             {
-                const bool ok = mbar_wait_or_abort(s_bar, ph, abort_flag);
+                bool ok = mbar_wait_or_abort(s_bar, ph, abort_flag);
+                // gamma of the next chunk (other stage), for the pre-decay below
+                if (ok && !it.last) ok = mbar_wait_or_abort(&gready[s ^ 1], ((i + 1) >> 1) & 1, abort_flag);
                 if (group_any(kBarState, kStateThreads, !ok)) {
                     if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;
@@ -833,7 +844,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             drained = true;
             // stage s is free: refill it with the chunk two ahead
             if (have_ahead) {
-                fill(ahead, s, ns + 1, gb_ahead);
+                fill(ahead, s, ns + 1);
                 have_ahead = item_next(a, total, ahead);
             }
         }
@@ -843,7 +854,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             mbar_wait(drain_s, 0, kWaitNs / 4);
         }
         // TMA loads the prep group never consumed (only after an abort)
-        if (stid == 0 && *abort_flag)
+        if (stid == kRefill && *abort_flag)
             for (int x = 0; x < 2; ++x)
                 if ((issued >> x) & 1u) mbar_wait(&full[x], (issued_par >> x) & 1u, kWaitNs / 4);
     }
