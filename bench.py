@@ -6,7 +6,7 @@
 Headline workload (one step): chunked gated-delta-rule prefill of 8 sequences x
 16384 tokens, 16 heads, d_k = d_v = 128, bf16 q/k/v, fp32 gates and fp32 final
 state, chunk 64 -- one gdn_prefill call over the packed batch. Inputs stay
-resident in HBM (about 1.1 GB, larger than the 126 MB L2). The same JSON line
+resident in HBM (q, k, v, gates and o: about 2.2 GB, far larger than the 126 MB L2). The same JSON line
 carries two more measured workloads of the same hot path: batched decode
 (256 sequences, 100 in-place steps) and one 0.8B-shaped layer prefill
 (conv + SiLU + L2 norm, then the chunked prefill, T = 4096).
@@ -239,7 +239,12 @@ def config_block(n):
     return {"workload": f"long_prefill_{SEQS}x{SEQ_LEN}_h16_d128_bf16", "global_batch": SEQS * n,
             "seq_len": SEQ_LEN, "heads": H, "head_dim": D, "chunk": CHUNK,
             "parallelism": f"replicas{n}" if n > 1 else "single",
-            "l2": "inputs larger than L2 (1.1 GB resident per step)"}
+            "l2": f"inputs larger than L2 ({resident_bytes() / 1e9:.2f} GB resident per step, L2 126 MB)"}
+
+
+def resident_bytes():
+    """q/k/v/o bf16 and g/beta fp32 of the timed prefill: what one step touches."""
+    return SEQS * SEQ_LEN * H * (4 * D * 2 + 2 * 4)
 
 
 # ----------------------------------------------------------------------------
@@ -383,9 +388,9 @@ def bench_layer(args, dist, pk):
     cu = torch.from_numpy(Lw.cu_seqlens).to(dev)
     y = torch.empty_like(x)
     st = torch.empty((1, Lw.C, 3), dtype=torch.bfloat16, device=dev)
-    q = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
-    k, v = torch.empty_like(q), torch.empty_like(q)
-    o = torch.empty_like(q)
+    qkv = y.view(T, 3, H, D)
+    q, k, v = qkv[:, 0], qkv[:, 1], qkv[:, 2]  # token-strided views: no copies
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
     hT = torch.empty((1, H, D, D), dtype=torch.float32, device=dev)
     ws = torch.empty(gdn.prefill_workspace_size(1, T, H, D, D, CHUNK), dtype=torch.uint8, device=dev)
     flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
@@ -396,8 +401,6 @@ def bench_layer(args, dist, pk):
 
     def layer():
         conv()
-        qkv = y.view(T, 3, H, D)
-        q.copy_(qkv[:, 0]); k.copy_(qkv[:, 1]); v.copy_(qkv[:, 2])
         gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, qk_l2norm=False)
 
     conv_ms, layer_ms = [], []
@@ -415,7 +418,7 @@ def bench_layer(args, dist, pk):
     conv_bytes = 2 * T * Lw.C * 2 + Lw.C * 4 * 2
     return {"value": T / (lms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": lms,
             "workload": "layer_0p8b_T4096_conv_then_prefill",
-            "note": "layer time includes three torch copies splitting [q|k|v] for the prefill",
+            "note": "two launches (conv, prefill); the prefill reads q, k, v as strided views of the conv output",
             "conv": {"ms": cms, "roofline": {
                 "bound": "hbm", "achieved": conv_bytes / (cms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": conv_bytes / (cms * 1e-3) / 1e9 / pk["hbm_gbs"],
@@ -468,7 +471,7 @@ def run_ours(args, dist: Dist):
         "config": config_block(dist.world),
         "roofline": {"bound": "hbm", "achieved": hbm_ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": hbm_ach / pk["hbm_gbs"],
-                     "traffic": profiled_traffic("prefill", ["prefill_simt.cu", "prefill_tc.cu"],
+                     "traffic": profiled_traffic("prefill", ["prefill_simt.cu", "prefill_tc.cu", "tc_ptx.cuh"],
                                                  th),
                      "kernel": "gdn_prefill (schedule + chunk kernel), CUDA events per call",
                      "algorithmic_bytes": bytes_alg, "peak_source": pk["source"]},

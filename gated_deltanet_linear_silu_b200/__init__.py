@@ -53,8 +53,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_conv_silu.restype = i32
         L.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
         L.gdn_prefill_workspace_size.restype = sz
-        L.gdn_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32, f32, i32,
-                                  f32, i32, vp, vp, vp, vp, sz, i32, vp]
+        L.gdn_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                  i64, i64, i64, f32, i32, f32, i32, vp, vp, vp, vp, sz, i32, vp]
         L.gdn_prefill.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, i32, f32,
                                       vp, vp]
@@ -64,7 +64,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_check_device_status.argtypes = [vp]
         L.gdn_check_device_status.restype = i32
         L.gdn_prefill_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32,
-                                          f32, i32, f32, i32, vp, vp, vp, i32, vp]
+                                          i64, i64, i64, f32, i32, f32, i32, vp, vp, vp, i32, vp]
         L.gdn_prefill_noalloc.restype = i32
         L.gdn_prefill_noalloc_max_scratch.argtypes = []
         L.gdn_prefill_noalloc_max_scratch.restype = sz
@@ -103,6 +103,17 @@ def _cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _token_stride(t: torch.Tensor) -> int:
+    """Elements between consecutive tokens of a [T, H, d] tensor whose rows
+    may be views into a wider fused buffer (each row itself dense)."""
+    if not t.is_cuda:
+        raise ValueError("tensors must be CUDA tensors")
+    T, H, d = t.shape
+    if t.stride(2) != 1 or (H > 1 and t.stride(1) != d) or t.stride(0) < H * d:
+        raise ValueError("q, k, v must have dense [H, d] rows (token stride may be larger)")
+    return int(t.stride(0))
+
+
 def conv_silu(x: torch.Tensor, w: torch.Tensor, cu_seqlens: torch.Tensor, *,
               conv_state: Optional[torch.Tensor] = None, conv_state_out: Optional[torch.Tensor] = None,
               return_state: bool = True, qk_l2norm: bool = True, n_qk_channels: Optional[int] = None,
@@ -139,7 +150,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
             cu_seqlens_host: Optional[torch.Tensor] = None, algo: str = "auto",
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None
             ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Chunked gated delta rule. q,k [T,H,dk], v [T,H,dv] (bf16 or fp32),
+    """Chunked gated delta rule. q,k [T,H,dk], v [T,H,dv] (bf16 or fp32; each
+    may be a token-strided view, e.g. a slice of the fused conv output),
     g,beta [T,H] fp32, cu_seqlens int32 [N+1] (device). Returns (o, hT);
     final_state may be initial_state itself for an in-place update."""
     T, H, dk = q.shape
@@ -152,14 +164,15 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     ws_bytes = prefill_workspace_size(N, T, H, dk, dv, chunk)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    _cuda(q, k, v, g, beta, cu_seqlens, initial_state, hT, o, workspace)
+    ld = [_token_stride(t) for t in (q, k, v)]
+    _cuda(g, beta, cu_seqlens, initial_state, hT, o, workspace)
     host_cu = None
     if cu_seqlens_host is not None:
         host_cu = cu_seqlens_host.to(torch.int32).contiguous()
     st = lib().gdn_prefill(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
         None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, dk, dv,
-        float(scale), int(qk_l2norm), float(eps), int(chunk), _ptr(initial_state), _ptr(hT),
+        ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(chunk), _ptr(initial_state), _ptr(hT),
         _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill")
     return o, hT
@@ -176,10 +189,11 @@ def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
     T, H, dk = q.shape
     dv = v.shape[2]
     N = cu_seqlens.shape[0] - 1
-    _cuda(q, k, v, g, beta, cu_seqlens, initial_state, final_state, out)
+    ld = [_token_stride(t) for t in (q, k, v)]
+    _cuda(g, beta, cu_seqlens, initial_state, final_state, out)
     st = lib().gdn_prefill_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens), None,
-        N, T, H, dk, dv, float(scale), int(qk_l2norm), float(eps), int(chunk),
+        N, T, H, dk, dv, ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(chunk),
         _ptr(initial_state), _ptr(final_state), _ptr(out), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill_noalloc")
 

@@ -116,7 +116,7 @@ size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, i
 gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                          const float* g, const float* beta, const int32_t* cu_seqlens,
                          const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int dk,
-                         int dv, float scale, int qk_l2norm, float eps, int chunk, const float* h0,
+                         int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale, int qk_l2norm, float eps, int chunk, const float* h0,
                          float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
                          void* stream) {
     if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
@@ -131,6 +131,13 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
         !aligned16(hT))
         return GDN_ERR_INVALID_ARG;
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    const int64_t esz = dtype == GDN_BF16 ? 2 : 4;
+    if (ld_q == 0) ld_q = (int64_t)H * dk;
+    if (ld_k == 0) ld_k = (int64_t)H * dk;
+    if (ld_v == 0) ld_v = (int64_t)H * dv;
+    if (ld_q < (int64_t)H * dk || ld_k < (int64_t)H * dk || ld_v < (int64_t)H * dv ||
+        (ld_q * esz) % 16 != 0 || (ld_k * esz) % 16 != 0 || (ld_v * esz) % 16 != 0)
+        return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H * 2 >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
     if (T_tot >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;  // cu_seqlens is int32
     if (gdn_status_t st = check_host_seqlens(cu_seqlens_host, N, T_tot)) return st;
@@ -140,7 +147,7 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
         return GDN_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     gdn::PrefillArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, dk, dv,
-                       scale, qk_l2norm, eps, chunk, h0, hT, o,
+                       ld_q, ld_k, ld_v, scale, qk_l2norm, eps, chunk, h0, hT, o,
                        reinterpret_cast<int32_t*>(ws + wl.order_off),
                        reinterpret_cast<int32_t*>(ws + wl.counter_off), status_ptr()};
     if (!a.status) return GDN_ERR_CUDA;

@@ -7,19 +7,23 @@
 // that owns it (plus a 3-row halo that hits L2), every output row written once.
 //
 // Thread layout: a thread owns 8 consecutive channels (one 16-byte bf16
-// vector) and walks TT consecutive tokens, keeping the previous K-1 inputs in
-// registers. A warp covers 256 channels; the L2 norm of a head (head_dim
-// channels = head_dim/8 lanes) is a shuffle reduction inside the warp.
+// vector) of TT consecutive tokens. A warp covers 256 channels; the L2 norm of
+// a head (head_dim channels = head_dim/8 lanes) is a shuffle reduction inside
+// the warp. When the CTA's tokens and their 3-token halo lie inside one
+// sequence (the common case) every thread issues all TT + 3 row loads before
+// the first use, so a CTA keeps (TT + 3) x 16 bytes per thread in flight; tiles
+// that touch a sequence start take a token-by-token path that reads the conv
+// state (or zeros) for positions before the start.
 #include "common.cuh"
 #include "launch.h"
 
 namespace gdn {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;
 constexpr int kVec = 8;                       // channels per thread
-constexpr int kChanPerCta = kThreads * kVec;  // 2048
-constexpr int kTT = 32;                       // tokens per CTA
+constexpr int kChanPerCta = kThreads * kVec;  // 1024
+constexpr int kTT = 8;                        // tokens per CTA
 
 template <typename T> struct Vec8;
 template <> struct Vec8<uint16_t> {
@@ -53,6 +57,56 @@ template <> struct Vec8<float> {
         *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
     }
 };
+
+// One token's 8 channels as loaded (converted to fp32 at first use).
+template <typename T> struct Raw8;
+template <> struct Raw8<uint16_t> {
+    uint4 u;
+    __device__ __forceinline__ void load(const uint16_t* p) { u = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void get(float (&x)[8]) const {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = *reinterpret_cast<const float4*>(p);
+        b = *reinterpret_cast<const float4*>(p + 4);
+    }
+    __device__ __forceinline__ void get(float (&x)[8]) const {
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+};
+
+// SiLU(x) = x * sigmoid(x) = x / (1 + e^-x), with the fast exponential and
+// divide (both within a few ulp of fp32; the result is 0 when e^-x overflows).
+__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// conv (4-wide window, taps right-aligned) + SiLU for one token; returns the
+// squared norm of the 8 outputs.
+template <typename T>
+__device__ __forceinline__ float conv_token(const float (&wp)[4][8], const float (&xm3)[8],
+                                            const float (&xm2)[8], const float (&xm1)[8],
+                                            const float (&xt)[8], float (&y)[8]) {
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float acc = wp[0][i] * xm3[i];
+        acc = fmaf(wp[1][i], xm2[i], acc);
+        acc = fmaf(wp[2][i], xm1[i], acc);
+        acc = fmaf(wp[3][i], xt[i], acc);
+        acc = silu(acc);
+        y[i] = acc;
+        ss = fmaf(acc, acc, ss);
+    }
+    return ss;
+}
 
 // Input of sequence n at absolute token p for the thread's 8 channels; p may
 // precede the sequence start, in which case the conv state (or 0) supplies it.
@@ -88,15 +142,29 @@ __global__ void __launch_bounds__(kThreads) conv_silu_kernel(ConvArgs a) {
 
     // Taps, right-aligned into a 4-wide window: y = sum_j wp[j] * x[t-3+j].
     float wp[4][8];
+    if (a.K == 4 && active && (reinterpret_cast<uintptr_t>(a.w) & 15u) == 0) {
+        // the thread's 8 x 4 taps are 32 contiguous values
+        const T* wr = static_cast<const T*>(a.w) + (int64_t)c0 * 4;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+        for (int q = 0; q < 4; ++q) {
+            Raw8<T> r;
+            r.load(wr + 8 * q);
+            float f[8];
+            r.get(f);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int jj = j - (4 - a.K);
-            wp[j][i] = (active && jj >= 0)
-                           ? Elem<T>::load(static_cast<const T*>(a.w), (int64_t)(c0 + i) * a.K + jj)
-                           : 0.f;
+            for (int e = 0; e < 8; ++e) wp[e & 3][2 * q + (e >> 2)] = f[e];  // channel 2q + e/4, tap e%4
         }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int jj = j - (4 - a.K);
+                wp[j][i] = (active && jj >= 0)
+                               ? Elem<T>::load(static_cast<const T*>(a.w), (int64_t)(c0 + i) * a.K + jj)
+                               : 0.f;
+            }
+    }
 
     int n = find_sequence(a.cu, a.N, t0);
     int64_t seq_start = a.cu[n], seq_end = a.cu[n + 1];
@@ -104,12 +172,48 @@ __global__ void __launch_bounds__(kThreads) conv_silu_kernel(ConvArgs a) {
         if (threadIdx.x == 0) set_status(a.status, kStatusBadSeqlens);
         return;
     }
+    const int lanes_per_head = a.head_dim / kVec;
+    const bool norm_me = a.qk_l2norm && c0 < a.n_qk;
+    if (t0 - 3 >= seq_start && t1 <= seq_end) {
+        // All rows of the window in one sequence: issue every load first.
+        Raw8<T> r[kTT + 3];
+        const T* xp = static_cast<const T*>(a.x) + (t0 - 3) * a.C + c0;
+#pragma unroll
+        for (int u = 0; u < kTT + 3; ++u)
+            if (active && t0 - 3 + u < t1) r[u].load(xp + (int64_t)u * a.C);
+        float xm3[8], xm2[8], xm1[8];
+        r[0].get(xm3);
+        r[1].get(xm2);
+        r[2].get(xm1);
+#pragma unroll
+        for (int u = 0; u < kTT; ++u) {
+            const int64_t t = t0 + u;
+            if (t >= t1) break;  // uniform over the CTA
+            float xt[8], y[8];
+            r[u + 3].get(xt);
+            float ss = conv_token<T>(wp, xm3, xm2, xm1, xt, y);
+            if (a.qk_l2norm) {
+                ss = group_sum(ss, lanes_per_head);
+                if (norm_me) {
+                    const float inv = 1.f / sqrtf(ss + a.eps);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) y[i] *= inv;
+                }
+            }
+            if (active) Vec8<T>::store(static_cast<T*>(a.y) + t * a.C + c0, y);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                xm3[i] = xm2[i];
+                xm2[i] = xm1[i];
+                xm1[i] = xt[i];
+            }
+        }
+        return;
+    }
     float xm3[8], xm2[8], xm1[8], xt[8];
     fetch<T>(a, n, seq_start, t0 - 3, c0, active, xm3);
     fetch<T>(a, n, seq_start, t0 - 2, c0, active, xm2);
     fetch<T>(a, n, seq_start, t0 - 1, c0, active, xm1);
-    const int lanes_per_head = a.head_dim / kVec;
-    const bool norm_me = a.qk_l2norm && c0 < a.n_qk;
 
     for (int64_t t = t0; t < t1; ++t) {
         if (t == seq_end) {  // next non-empty sequence: window restarts from its state
@@ -126,17 +230,7 @@ __global__ void __launch_bounds__(kThreads) conv_silu_kernel(ConvArgs a) {
         }
         fetch<T>(a, n, seq_start, t, c0, active, xt);
         float y[8];
-        float ss = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float acc = wp[0][i] * xm3[i];
-            acc = fmaf(wp[1][i], xm2[i], acc);
-            acc = fmaf(wp[2][i], xm1[i], acc);
-            acc = fmaf(wp[3][i], xt[i], acc);
-            acc = acc / (1.f + expf(-acc));  // SiLU
-            y[i] = acc;
-            ss = fmaf(acc, acc, ss);
-        }
+        float ss = conv_token<T>(wp, xm3, xm2, xm1, xt, y);
         if (a.qk_l2norm) {  // every lane joins the shuffle; only q/k lanes use it
             ss = group_sum(ss, lanes_per_head);
             if (norm_me) {

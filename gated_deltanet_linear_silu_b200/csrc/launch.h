@@ -52,6 +52,7 @@ struct PrefillArgs {
     int N;
     int64_t T_tot;
     int H, dk, dv;
+    int64_t ld_q, ld_k, ld_v;  // elements between consecutive tokens of q, k, v
     float scale;
     int qk_l2norm;
     float eps;

@@ -146,16 +146,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
                 const int r = e / dk, i = e % dk;
                 float qv = 0.f, kv = 0.f;
                 if (r < L) {
-                    const int64_t off = ((c0 + r) * H + h) * dk + i;
-                    qv = Elem<T>::load(q, off);
-                    kv = Elem<T>::load(k, off);
+                    qv = Elem<T>::load(q, (c0 + r) * a.ld_q + h * dk + i);
+                    kv = Elem<T>::load(k, (c0 + r) * a.ld_k + h * dk + i);
                 }
                 Qs[r * ldk + i] = qv;
                 Ks[r * ldk + i] = kv;
             }
             for (int e = tid; e < C * DVT; e += kThreads) {
                 const int r = e / DVT, j = e % DVT;
-                Vs[r * ldv + j] = r < L ? Elem<T>::load(v, ((c0 + r) * H + h) * dv + j0 + j) : 0.f;
+                Vs[r * ldv + j] = r < L ? Elem<T>::load(v, (c0 + r) * a.ld_v + h * dv + j0 + j) : 0.f;
             }
             if (tid < C) {
                 gam[tid] = tid < L ? a.g[(c0 + tid) * H + h] : 0.f;

@@ -880,15 +880,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [T_tot, H, 128] bf16 viewed as a 3-D tensor (feature, head, token); boxes of
+// [T_tot, H, 128] bf16 (tokens `ld` elements apart) viewed as a 3-D tensor
+// (feature, head, token); boxes of
 // 64 features x 1 head x 64 tokens, zero fill past T_tot on loads, clipped on
 // stores. Loads use the 128-byte swizzle the MMA descriptors expect; the O
 // store reads a plain row-major staging tile.
-bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t T, bool swizzle) {
+bool make_map(CUtensorMap* m, const void* ptr, int H, int64_t T, int64_t ld, bool swizzle) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T};
-    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)ld * 2};
     cuuint32_t box[3] = {64, 1, 64};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -906,8 +907,9 @@ bool prefill_tc_supported(const PrefillArgs& a) {
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, a.q, a.H, a.T_tot, true) || !make_map(&mk, a.k, a.H, a.T_tot, true) ||
-        !make_map(&mv, a.v, a.H, a.T_tot, true) || !make_map(&mo, a.o, a.H, a.T_tot, false))
+    if (!make_map(&mq, a.q, a.H, a.T_tot, a.ld_q, true) || !make_map(&mk, a.k, a.H, a.T_tot, a.ld_k, true) ||
+        !make_map(&mv, a.v, a.H, a.T_tot, a.ld_v, true) ||
+        !make_map(&mo, a.o, a.H, a.T_tot, (int64_t)a.H * kD, false))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemAlloc);

@@ -134,7 +134,14 @@ GDN_API size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, i
  *                                           is validated on the host
  *   h0              [N, H, dk, dv]  fp32    nullable initial state
  *   hT              [N, H, dk, dv]  fp32    nullable final state; may alias h0
- *   o               [T_tot, H, dv]  dtype   output
+ *   o               [T_tot, H, dv]  dtype   output (dense)
+ *   ld_q, ld_k, ld_v                        elements from one token of q, k, v
+ *                                           to the next; 0 = dense (H*dk, H*dk,
+ *                                           H*dv). Larger strides let q, k and v
+ *                                           be views into one fused [T_tot, C]
+ *                                           buffer, e.g. the conv output. Each
+ *                                           stride must be at least the dense
+ *                                           one and a multiple of 16 bytes.
  *   workspace       ws_bytes >= gdn_prefill_workspace_size(...)
  * A sequence of length 0 writes hT = h0 (or zeros) and no output.
  * Supported: dk, dv in {16, 32, ..., 128}; chunk in {16, 32, 64}.
@@ -144,6 +151,7 @@ GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gd
                          const float* g, const float* beta,
                          const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
                          int N, int64_t T_tot, int H, int dk, int dv,
+                         int64_t ld_q, int64_t ld_k, int64_t ld_v,
                          float scale, int qk_l2norm, float eps, int chunk,
                          const float* h0, float* hT, void* o,
                          void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream);
@@ -173,6 +181,7 @@ GDN_API gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const voi
                                          gdn_dtype_t dtype, const float* g, const float* beta,
                                          const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
                                          int N, int64_t T_tot, int H, int dk, int dv,
+                                         int64_t ld_q, int64_t ld_k, int64_t ld_v,
                                          float scale, int qk_l2norm, float eps, int chunk,
                                          const float* h0, float* hT, void* o, gdn_algo_t algo,
                                          void* stream);

@@ -64,7 +64,7 @@ FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails
 
 def _prefill(L, **kw):
     args = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, g=FAKE, beta=FAKE, cu=FAKE, cu_host=None, N=1,
-                T=64, H=2, dk=128, dv=128, scale=1.0, l2=1, eps=1e-6, chunk=64, h0=None, hT=None,
+                T=64, H=2, dk=128, dv=128, ldq=0, ldk=0, ldv=0, scale=1.0, l2=1, eps=1e-6, chunk=64, h0=None, hT=None,
                 o=FAKE, ws=FAKE, ws_bytes=1 << 20, algo=0, stream=None)
     args.update(kw)
     return L.gdn_prefill(*args.values())
@@ -76,6 +76,7 @@ def _prefill(L, **kw):
     (dict(q=None), 1), (dict(o=ctypes.c_void_p((1 << 20) + 4)), 1), (dict(cu=None), 1),
     (dict(ws=None), 3), (dict(ws_bytes=16), 3), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), 3),
     (dict(eps=float("nan")), 1),
+    (dict(ldq=255), 1), (dict(ldk=257), 1), (dict(ldv=8), 1), (dict(dt=0, ldq=258), 1),
 ])
 def test_prefill_rejects_bad_arguments(L, kw, expect):
     assert _prefill(L, **kw) == expect

@@ -69,6 +69,26 @@ def test_prefill_without_l2norm_and_strong_decay():
     assert err(o, o_ref) <= TOL_F32 and err(hT, h_ref) <= TOL_F32
 
 
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_token_strided_views_equal_dense(algo):
+    """q, k, v as views into one padded fused buffer give the dense result bit for bit."""
+    P = gi.random_prefill(12, [70, 129, 0, 64], H=2, dk=128, dv=128, with_h0=True)
+    o_d, h_d = prefill_gpu(P, algo=algo)
+    T, H, d = P.q.shape
+    ld = 3 * H * d + 64
+    fused = torch.zeros((T, ld), dtype=torch.bfloat16, device=DEV)
+    views = []
+    for i, a in enumerate((P.q, P.k, P.v)):
+        fused[:, i * H * d:(i + 1) * H * d] = dev_tensor(a, "bf16").view(T, H * d)
+        views.append(fused[:, i * H * d:(i + 1) * H * d].view(T, H, d))
+    assert views[0].stride(0) == ld and not views[0].is_contiguous()
+    o, hT = gdn.prefill(*views, dev_tensor(P.g, "f32"), dev_tensor(P.beta, "f32"),
+                        torch.from_numpy(P.cu_seqlens).to(DEV),
+                        initial_state=dev_tensor(P.h0, "f32"), algo=algo)
+    gdn.check_device_status(DEV)
+    assert np.array_equal(host(o), o_d) and np.array_equal(host(hT), h_d)
+
+
 def test_chunk_sizes_agree():
     P = gi.random_prefill(4, [100, 37], H=2, dk=32, dv=32, dtype="f32", with_h0=True)
     outs = [prefill_gpu(P, chunk=c) for c in (16, 32, 64)]
@@ -225,7 +245,7 @@ def test_layer_0p8b_conv_then_prefill():
     y, _ = gdn.conv_silu(dev_tensor(Lw.mixed_qkv, "bf16"), dev_tensor(Lw.conv_w, "bf16"), cu,
                          n_qk_channels=2 * H * d, head_dim=d)
     qkv = y.view(T, 3, H, d)
-    q, k, v = (qkv[:, i].contiguous() for i in range(3))
+    q, k, v = (qkv[:, i] for i in range(3))  # token-strided views of the conv output
     o, hT = gdn.prefill(q, k, v, dev_tensor(Lw.g, "f32"), dev_tensor(Lw.beta, "f32"), cu,
                         qk_l2norm=False)
     gdn.check_device_status(DEV)
