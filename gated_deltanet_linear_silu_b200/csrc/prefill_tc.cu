@@ -15,16 +15,20 @@
 // B200 mapping. Every contraction is issued as an M = 128 tcgen05.mma by
 // computing the transposed products, so the 128-wide head dimension is the
 // MMA's M and no tile is padded:
-//   [Q;K] K^T          -> TMEM  R_A   (128 lanes = 64 q rows + 64 k rows, 64 cols)
+//   [Q;K][Q;K]^T       -> TMEM  R_A   (128 lanes = 64 q rows + 64 k rows)
 //   W^T  = K^T T1^T    -> TMEM  R_W   (lanes = dk, cols = tokens)
 //   U~^T = V^T T2^T    -> TMEM  R_U   (lanes = dv, cols = tokens)
 //   U^T  = U~^T + S^T (-W^T)         (accumulated in R_U)
 //   O^T  = S^T Q~^T + U^T P^T        (R_O, lanes = dv, cols = tokens)
 //   S^T <- e^{gamma_L} S^T + U^T K~  (R_S, fp32 master state, lanes = dv, cols = dk)
-// The algorithmic 11.5 MFLOP per (chunk, head) are exactly the MMAs issued.
+// The algorithmic 11.5 MFLOP per (chunk, head) are the MMAs issued, plus the
+// q-by-q block of the Gram matrix, whose diagonal gives the q norms.
 // The L2 norms, scale and decays are applied as per-row factors in the
 // epilogues, so the MMAs read the raw bf16 input tiles that TMA brings in
-// (128-byte swizzle). The solve for T runs on CUDA cores in fp32.
+// (128-byte swizzle). The state chain's A operands, S^T and U^T, never touch
+// shared memory: the epilogues write them back to TMEM as packed bf16 and the
+// MMAs read A from there, so those MMAs stream only B from shared memory. The
+// solve for T runs on CUDA cores in fp32 (with tf32 tensor-core merges).
 //
 // Warp specialisation (one CTA of 12 warps per SM, persistent over units):
 //   warps 0-7   prep group: everything that does not depend on the state --
@@ -72,10 +76,9 @@ constexpr uint32_t kVb0 = 4 * kBox, kVb1 = 5 * kBox;
 constexpr uint32_t kStageBytes = 6 * kBox;        // 48 KB: Q, K, V tiles (V later holds O)
 constexpr uint32_t kOffVec = 2 * kStageBytes;     // per stage: g, beta, gamma, bet, rq, rk (6 x 64 fp32)
 constexpr uint32_t kVecBytes = 2048;
-constexpr uint32_t kOffSA = kOffVec + 2 * kVecBytes;  // S^T bf16, 2 x [128 dv][64 dk] K-major
-constexpr uint32_t kOffWT = kOffSA + 32768;       // -W^T bf16 [128 dk][64 tok] MN-major
-constexpr uint32_t kOffUT = kOffWT + 16384;       // U^T bf16 [128 dv][64 tok] K-major
-constexpr uint32_t kOffP = kOffUT + 16384;        // P bf16 [64 r][64 j] K-major, per stage
+constexpr uint32_t kOffWT = kOffVec + 2 * kVecBytes;  // -W^T bf16 [128 dk][64 tok] MN-major
+constexpr uint32_t kOffO = kOffWT + 16384;        // O staging bf16, 2 x [64 tok][64 dv] row-major
+constexpr uint32_t kOffP = kOffO + 16384;         // P bf16 [64 r][64 j] K-major, per stage
 constexpr int kLdA = 68;                          // padded fp32 row stride (272 B)
 constexpr uint32_t kOffA = kOffP + 2 * 8192;      // A fp32 [64][kLdA]; after the solve T1^T, T2^T
 constexpr uint32_t kOffT1 = kOffA, kOffT2 = kOffA + 8192;
@@ -85,13 +88,16 @@ constexpr uint32_t kOffMisc = kOffBar + 128;      // tmem base, abort flag, scan
 constexpr uint32_t kSmemBytes = kOffMisc + 64;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(kOffA % 1024 == 0 && kOffSA % 1024 == 0 && kOffP % 1024 == 0, "swizzle alignment");
+static_assert(kOffA % 1024 == 0 && kOffWT % 1024 == 0 && kOffP % 1024 == 0, "swizzle alignment");
 
 // TMEM columns (fp32, 128 lanes).
 constexpr uint32_t kTmemCols = 512;
-// R_O, R_U: 2 x 64 columns each. R_A holds the 128 x 128 Gram matrix [Q;K][Q;K]^T and is
-// reused for W^T once the P/A epilogue has read it.
-constexpr uint32_t kRS = 0, kRO = 128, kRU = 256, kRA = 384, kRW = 384;
+// R_S: fp32 state S^T (128 columns). R_SB: S^T as packed bf16 (64 columns), the
+// TMEM-resident A operand of MMA1. R_O: O^T of the chunk in flight (64).
+// R_U: U~^T / U^T per stage (2 x 64); after the U epilogue its first 32 columns
+// hold U^T as packed bf16, the A operand of MMA2. R_A holds the 128 x 128 Gram
+// matrix [Q;K][Q;K]^T and is reused for W^T once the P/A epilogue has read it.
+constexpr uint32_t kRS = 0, kRSB = 128, kRO = 192, kRU = 256, kRA = 384, kRW = 384;
 
 constexpr uint32_t kIdescA = idesc_bf16(128, 128, 0, 0);   // [Q;K] [Q;K]^T (Gram)
 constexpr uint32_t kIdescMN = idesc_bf16(128, 64, 1, 1);   // K^T T1^T, V^T T2^T
@@ -106,6 +112,11 @@ struct TcParams {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+// 32 fp32 values (times f) as 16 packed bf16 pairs, even index in the low half.
+__device__ __forceinline__ void pack_row32(const float (&v)[32], float f, uint32_t (&w)[16]) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) w[c] = pack_bf16(v[2 * c] * f, v[2 * c + 1] * f);
 }
 __device__ __forceinline__ void unpack_bf16(uint32_t w, float& lo, float& hi) {
     lo = __uint_as_float(w << 16);
@@ -293,9 +304,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     const int H = a.H;
     const int64_t total = (int64_t)a.N * H;
 
-    uint8_t* sSA = sm + kOffSA;
     uint8_t* sWT = sm + kOffWT;
-    uint8_t* sUT = sm + kOffUT;
+    uint8_t* sO = sm + kOffO;
     uint8_t* sT1 = sm + kOffT1;
     uint8_t* sT2 = sm + kOffT2;
     float* sA = reinterpret_cast<float*>(sm + kOffA);
@@ -663,9 +673,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             const float* vec = S.vec(s);
             const int64_t sbase = ((int64_t)it.U.n * H + it.U.h) * kD * kD;
             if (it.first) {
-                // initial state: S^T as the bf16 A operand (thread = dv lane j) and, in
-                // TMEM, e^{gamma_L} S^T -- R_S always holds the state pre-decayed by the
-                // coming chunk, ready for the accumulation of K~^T U.
+                // initial state: S^T as the bf16 A operand in R_SB (thread = dv lane j)
+                // and e^{gamma_L} S^T in R_S -- R_S always holds the state pre-decayed
+                // by the coming chunk, ready for the accumulation of K~^T U.
                 {
                     const bool ok = mbar_wait_or_abort(&gready[s], ns & 1, abort_flag);
                     if (group_any(kBarState, kStateThreads, !ok)) {
@@ -685,13 +695,14 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
 #pragma unroll
                         for (int e = 0; e < 32; ++e) v[e] = 0.f;
                     }
-                    store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
+                    uint32_t w[16];
+                    pack_row32(v, 1.f, w);
+                    tmem_st16(tmem + lane_off + kRSB + 16 * cc, w);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] *= eL;
                     tmem_st32(tmem + lane_off + kRS + 32 * cc, v);
                 }
                 tmem_wait_st();
-                fence_proxy_async();
                 tc_fence_before();
                 group_sync(kBarState, kStateThreads);
             }
@@ -704,25 +715,21 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             }
             tc_fence_after();
             drained = false;
-            // ---- MMA1: U^T += S^T (-W^T) (R_U[s]) ; O^T = S^T Q~^T (R_O[s])
+            // ---- MMA1: U^T += S^T (-W^T) (R_U[s]) ; O^T = S^T Q~^T (R_O), A = S^T from R_SB
             if (stid == 0) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint64_t sa = sw128_desc(smem_u32(sSA + (k >> 2) * 16384 + 32 * (k & 3)), 16, 1024);
-                    mma_bf16(tmem + kRU + 64 * s, sa, sw128_desc(smem_u32(sWT + 2048 * k), 8192, 1024),
-                             kIdescSW, 1);
-                }
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ta(tmem + kRU + 64 * s, tmem + kRSB + 8 * k,
+                                sw128_desc(smem_u32(sWT + 2048 * k), 8192, 1024), kIdescSW, 1);
                 mma_commit(u_bar);
                 mma_commit(wt_free);
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint64_t sa = sw128_desc(smem_u32(sSA + (k >> 2) * 16384 + 32 * (k & 3)), 16, 1024);
                     const uint32_t qo = (k < 4 ? kQb0 : kQb1) + 32 * (k & 3);
-                    mma_bf16(tmem + kRO + 64 * s, sa, sw128_desc(smem_u32(st + qo), 16, 1024), kIdescSQ,
-                             k > 0);
+                    mma_bf16_ta(tmem + kRO, tmem + kRSB + 8 * k, sw128_desc(smem_u32(st + qo), 16, 1024),
+                                kIdescSQ, k > 0);
                 }
             }
-            if (stid == 0) bulk_wait_group_read0();  // previous O store has read U^T
             {
                 const bool ok = mbar_wait_or_abort(u_bar, ph, abort_flag);
                 if (group_any(kBarState, kStateThreads, !ok)) {
@@ -731,15 +738,21 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
             }
             tc_fence_after();
-            // ---- U^T row j (64 tokens) as the bf16 A operand of MMA2
+            // ---- U^T row j (64 tokens) as packed bf16 in the first 32 columns of
+            // R_U[s]: the TMEM-resident A operand of MMA2
+            {
+                uint32_t w[32];
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                float x[32];
-                tmem_ld32(tmem + lane_off + kRU + 64 * s + 32 * hf, x);
-                tmem_wait_ld();
-                store_half_row(sUT, j, hf, x, 1.f);
+                for (int hf = 0; hf < 2; ++hf) {
+                    float x[32];
+                    tmem_ld32(tmem + lane_off + kRU + 64 * s + 32 * hf, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) w[16 * hf + c] = pack_bf16(x[2 * c], x[2 * c + 1]);
+                }
+                tmem_st32(tmem + lane_off + kRU + 64 * s, w);
+                tmem_wait_st();
             }
-            fence_proxy_async();
             tc_fence_before();
             group_sync(kBarState, kStateThreads);
             // ---- MMA2: S^T += U^T K~ (R_S) ; O^T += U^T P^T (R_O[s])
@@ -748,14 +761,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 uint8_t* sP = sm + kOffP + s * 8192;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + kRS, sw128_desc(smem_u32(sUT + 32 * k), 16, 1024),
-                             sw128_desc(smem_u32(st + kKb0 + 2048 * k), kKb1 - kKb0, 1024), kIdescUK, 1);
+                    mma_bf16_ta(tmem + kRS, tmem + kRU + 64 * s + 8 * k,
+                                sw128_desc(smem_u32(st + kKb0 + 2048 * k), kKb1 - kKb0, 1024), kIdescUK, 1);
                 mma_commit(s_bar);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + kRO + 64 * s, sw128_desc(smem_u32(sUT + 32 * k), 16, 1024),
-                             sw128_desc(smem_u32(sP + 32 * k), 16, 1024), kIdescSQ, 1);
+                    mma_bf16_ta(tmem + kRO, tmem + kRU + 64 * s + 8 * k,
+                                sw128_desc(smem_u32(sP + 32 * k), 16, 1024), kIdescSQ, 1);
                 mma_commit(o_bar);
+                bulk_wait_group_read0();  // the previous O store has read the staging tile
             }
             {
                 bool ok = mbar_wait_or_abort(s_bar, ph, abort_flag);
@@ -766,18 +780,28 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     break;
                 }
             }
+            // MMA1 and MMA2's state half, the last readers of stage s, are done:
+            // refill it with the chunk two ahead
+            if (have_ahead) {
+                fill(ahead, s, ns + 1);
+                have_ahead = item_next(a, total, ahead);
+            }
             tc_fence_after();
             // ---- new state: bf16 S^T for the next chunk's MMA1, and R_S pre-decayed
             // by the next chunk's e^{gamma_L} (its gates are already in the other
             // stage's vector block); the final state at the end of a sequence.
             {
                 const float eL = it.last ? 1.f : expf(S.vec(s ^ 1)[128 + 63]);
-#pragma unroll
+#pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     float v[32];
                     tmem_ld32(tmem + lane_off + kRS + 32 * cc, v);
                     tmem_wait_ld();
-                    store_half_row(sSA + (cc >> 1) * 16384, j, cc & 1, v, 1.f);
+                    {
+                        uint32_t w[16];
+                        pack_row32(v, 1.f, w);
+                        tmem_st16(tmem + lane_off + kRSB + 16 * cc, w);
+                    }
                     if (it.last) {
                         if (a.hT) {
                             float* hTp = a.hT + sbase + j + 32 * cc * kD;
@@ -792,7 +816,6 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
                 tmem_wait_st();
             }
-            fence_proxy_async();
             {
                 const bool ok = mbar_wait_or_abort(o_bar, ph, abort_flag);
                 if (group_any(kBarState, kStateThreads, !ok)) {
@@ -802,16 +825,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             }
             tc_fence_after();
             ph ^= 1;
-            // ---- O: column j of O^T -> O tile staged in the U^T tile (dead until the
-            // next chunk's U epilogue) as two [64 tokens][64 d_v] row-major boxes; a
-            // full chunk leaves by one TMA store, a partial one as 16-byte rows of its
-            // L valid tokens.
+            // ---- O: column j of O^T -> O staging tile as two [64 tokens][64 d_v]
+            // row-major boxes; a full chunk leaves by one TMA store, a partial one as
+            // 16-byte rows of its L valid tokens.
             {
-                uint16_t* ostage = reinterpret_cast<uint16_t*>(sUT) + (j >> 6) * 4096 + (j & 63);
+                uint16_t* ostage = reinterpret_cast<uint16_t*>(sO) + (j >> 6) * 4096 + (j & 63);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     float x[32];
-                    tmem_ld32(tmem + lane_off + kRO + 64 * s + 32 * hf, x);
+                    tmem_ld32(tmem + lane_off + kRO + 32 * hf, x);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) ostage[(32 * hf + e) * 64] = f32_to_bf16(x[e]);
@@ -822,8 +844,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             group_sync(kBarState, kStateThreads);
             if (L == kC) {
                 if (stid == 0) {
-                    tma_store_3d(&map_o, sUT, 0, it.U.h, (int)c0);
-                    tma_store_3d(&map_o, sUT + 8192, 64, it.U.h, (int)c0);
+                    tma_store_3d(&map_o, sO, 0, it.U.h, (int)c0);
+                    tma_store_3d(&map_o, sO + 8192, 64, it.U.h, (int)c0);
                     bulk_commit_group();
                 }
             } else {
@@ -834,19 +856,14 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     const int vid = stid + kStateThreads * k;  // token r, 16-byte column c16
                     const int r = vid >> 4, c16 = vid & 15;
                     if (r < L) {
-                        const uint8_t* src = sUT + (c16 >> 3) * 8192 + r * 128 + (c16 & 7) * 16;
+                        const uint8_t* src = sO + (c16 >> 3) * 8192 + r * 128 + (c16 & 7) * 16;
                         *reinterpret_cast<uint4*>(obase + r * tok_stride + 8 * c16) =
                             *reinterpret_cast<const uint4*>(src);
                     }
                 }
-                group_sync(kBarState, kStateThreads);  // staging read before U^T is rewritten
+                group_sync(kBarState, kStateThreads);  // staging read before it is rewritten
             }
             drained = true;
-            // stage s is free: refill it with the chunk two ahead
-            if (have_ahead) {
-                fill(ahead, s, ns + 1);
-                have_ahead = item_next(a, total, ahead);
-            }
         }
         if (stid == 0) bulk_wait_group0();  // O stores issued by this thread
         if (stid == 0 && !drained) {
