@@ -445,37 +445,40 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
             }
             group_sync(kBarPrep, kPrepThreads);
-            const float gL = gam[63];
 
             // ---- P rows (lanes < 64) and A rows (lanes >= 64), 32 columns per
-            // thread. Branch-free: every element is computed (exponent clamped
-            // at 0 so the masked-out upper triangle cannot overflow), then selected.
+            // thread; a warp covers one 32 x 32 block. Blocks above the diagonal are
+            // zero: P's is stored as zeros, A's is never read (the solve uses it as
+            // scratch). Inside the diagonal blocks P keeps j <= r; A needs no mask
+            // (the solve reads only its strictly lower part). Every element is
+            // computed branch-free (exponent clamped at 0 so masked or unread
+            // entries stay finite), then selected.
             {
-                float x[32];
-                tmem_ld32(tmem + lane_off + kRA + 64 + 32 * half, x);  // columns = k rows
-                tmem_wait_ld();
+                const int rb = warp & 1, cb = half;  // row and column block of this warp
+                const bool is_p = row < 64;
+                const int r = row & 63;
                 const int j0 = 32 * half;
-                if (row < 64) {
-                    const int r = row;
-                    const float gr = gam[r], fr = rq[r];
+                float x[32];
+                if (rb >= cb) {
+                    tmem_ld32(tmem + lane_off + kRA + 64 + 32 * half, x);  // columns = k rows
+                    tmem_wait_ld();
+                    const float gr = gam[r];
+                    const float fr = is_p ? rq[r] : bet[r] * rk[r];
+                    const int lim = (is_p && rb == cb) ? r : 64;  // keep j <= lim
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int j = j0 + e;
                         const float ex = __expf(fminf(gr - gam[j], 0.f));
                         const float val = ex * (fr * rk[j]) * x[e];
-                        x[e] = (j <= r) ? val : 0.f;
+                        x[e] = (j <= lim) ? val : 0.f;
                     }
-                    store_half_row(sP, r, half, x, 1.f);
                 } else {
-                    const int r = row - 64;
-                    const float gr = gam[r], fr = bet[r] * rk[r];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = j0 + e;
-                        const float ex = __expf(fminf(gr - gam[j], 0.f));
-                        const float val = ex * (fr * rk[j]) * x[e];
-                        x[e] = (j < r) ? val : 0.f;
-                    }
+                    for (int e = 0; e < 32; ++e) x[e] = 0.f;
+                }
+                if (is_p) {
+                    store_half_row(sP, r, half, x, 1.f);
+                } else if (rb >= cb) {
                     float4* Ar = reinterpret_cast<float4*>(sA + r * kLdA + j0);
 #pragma unroll
                     for (int q4 = 0; q4 < 8; ++q4)
@@ -599,16 +602,12 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             }
             tc_fence_after();
 
-            // ---- -W^T rows (lane = dk i, 32 columns each); K -> K~ in place
+            // ---- -W^T rows (lane = dk i, 32 columns each)
             {
                 float x[32];
                 tmem_ld32(tmem + lane_off + kRW + 32 * half, x);
                 tmem_wait_ld();
                 store_half_row(sWT, row, half, x, -1.f);
-                if (ptid < 128) {
-                    const int r = ptid & 63;
-                    scale_row(st + (ptid < 64 ? kKb0 : kKb1), r, expf(gL - gam[r]) * rk[r]);
-                }
             }
             fence_proxy_async();
             tc_fence_before();
@@ -729,6 +728,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     mma_bf16_ta(tmem + kRO, tmem + kRSB + 8 * k, sw128_desc(smem_u32(st + qo), 16, 1024),
                                 kIdescSQ, k > 0);
                 }
+            } else if (stid >= 32) {
+                // while MMA1 runs: K -> K~ = diag(e^{gamma_L - gamma} / |k|) K in place
+                // for MMA2 (the prep group's W^T MMA has read the raw K), 128 rows
+                // over the state group's other three warps
+                const float gL = vec[128 + 63];
+                for (int x = stid - 32; x < 128; x += kStateThreads - 32) {
+                    const int r = x & 63;
+                    scale_row(st + (x < 64 ? kKb0 : kKb1), r, expf(gL - vec[128 + r]) * vec[320 + r]);
+                }
             }
             {
                 const bool ok = mbar_wait_or_abort(u_bar, ph, abort_flag);
@@ -753,6 +761,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 tmem_st32(tmem + lane_off + kRU + 64 * s, w);
                 tmem_wait_st();
             }
+            fence_proxy_async();  // K~ (generic writes) is read by MMA2
             tc_fence_before();
             group_sync(kBarState, kStateThreads);
             // ---- MMA2: S^T += U^T K~ (R_S) ; O^T += U^T P^T (R_O[s])
