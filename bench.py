@@ -25,6 +25,7 @@ import ctypes
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -198,13 +199,16 @@ def oracle_sample(P, tokens: int, n_seq: int):
 
 
 def calibrated_sample(P, target_s: float):
-    """Pick (tokens, n_seq) so one oracle pass takes about target_s seconds."""
+    """Pick (tokens, n_seq) so one oracle pass takes about target_s seconds
+    (at most the whole workload): a prefix of every sampled sequence while
+    that fits, whole sequences beyond it."""
     import oracle
-    n_seq = max(1, min(P.N, oracle.default_threads() // P.H or 1))
-    tok, dt, _ = oracle_sample(P, 512, n_seq)
-    rate = tok / max(dt, 1e-6)  # tokens/s with n_seq sequences in parallel
-    tokens = int(max(256, min(SEQ_LEN, rate * target_s / n_seq)))
-    return tokens, n_seq
+    n0 = max(1, min(P.N, oracle.default_threads() // P.H or 1))  # sequences filling the cores
+    tok, dt, _ = oracle_sample(P, 512, n0)
+    budget = tok / max(dt, 1e-6) * target_s  # tokens the cores get through in target_s
+    if budget <= n0 * SEQ_LEN:
+        return int(max(256, budget / n0)), n0
+    return SEQ_LEN, int(min(P.N, math.ceil(budget / SEQ_LEN)))
 
 
 def run_reference(args, dist: Dist):
@@ -212,7 +216,7 @@ def run_reference(args, dist: Dist):
     if dist.rank != 0:
         return
     P = gi.long_prefill(SEQS, SEQ_LEN, H, D)
-    tokens, n_seq = calibrated_sample(P, 5.0)
+    tokens, n_seq = calibrated_sample(P, 3.0)
     for _ in range(args.warmup):
         oracle_sample(P, min(tokens, 1024), n_seq)
     times, toks, threads = [], 0, 1
