@@ -38,7 +38,7 @@
 //               (U, the state update, O) with the state resident in TMEM. When
 //               the state group is done with a stage of the two-stage ring one
 //               of its lanes refills it by TMA with the chunk two ahead.
-// The prep group's first warp turns a chunk's gates into beta and the cumulative
+// The prep group's second warp turns a chunk's gates into beta and the cumulative
 // decay gamma while the Gram MMA runs and signals the state group, which needs
 // only gamma_L (to pre-decay its state for the coming chunk).
 // The groups hand off through mbarriers; TMEM holds double-buffered U~/U
@@ -113,6 +113,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
+// 2^x on the XU unit (PTX ex2.approx: relative error about 2^-22; 0 for very
+// negative x).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // 32 fp32 values (times f) as 16 packed bf16 pairs, even index in the low half.
 __device__ __forceinline__ void pack_row32(const float (&v)[32], float f, uint32_t (&w)[16]) {
 #pragma unroll
@@ -287,7 +295,8 @@ struct Smem {
     uint8_t* base;
     __device__ uint8_t* stage(int s) const { return base + s * kStageBytes; }
     __device__ float* vec(int s) const { return reinterpret_cast<float*>(base + kOffVec + s * kVecBytes); }
-    // vec layout: [128,192) gamma, [192,256) beta (written by the prep group's first warp),
+    // vec layout: [0,64) e^{gmax - gamma}, [64] gmax, [65] factored-decay flag,
+    // [128,192) gamma, [192,256) beta (written by the prep group's second warp),
     // [256,320) rq, [320,384) rk (written by the prep group)
 };
 
@@ -371,10 +380,10 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             float* rq = vec + 256;
             float* rk = vec + 320;
             uint8_t* sP = sm + kOffP + s * 8192;
-            // gates g, beta of rows 2*lane and 2*lane+1 (first warp), in flight
-            // across the tile wait and the Gram MMA
+            // gates g, beta of rows 2*lane and 2*lane+1 (second warp: the first one
+            // issues the Gram MMA), in flight across the tile wait
             float4 gb = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (warp == 0) {
+            if (warp == 1) {
                 const int r = 2 * lane;
                 const float* gp = a.g + (it.c0 + r) * H + it.U.h;
                 const float* bp = a.beta + (it.c0 + r) * H + it.U.h;
@@ -405,7 +414,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             // gamma = inclusive prefix sum of g (scan of the row-pair sums over the
             // warp) and beta into the stage's vector block; the state group waits
             // for them on gready[s].
-            if (warp == 0) {
+            if (warp == 1) {
                 const float pair = gb.x + gb.y;
                 float x = pair;
 #pragma unroll
@@ -414,10 +423,27 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     if (lane >= o) x += y;
                 }
                 const int r = 2 * lane;
-                *reinterpret_cast<float2*>(gam + r) = make_float2(x - pair + gb.x, x);
+                const float g0 = x - pair + gb.x, g1 = x;
+                *reinterpret_cast<float2*>(gam + r) = make_float2(g0, g1);
                 *reinterpret_cast<float2*>(bet + r) = make_float2(gb.z, gb.w);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gready[s]);
+                // range of gamma over the chunk: when it is below 80, e^{gamma_r - gamma_j}
+                // factors as e^{gamma_r - gmax} e^{gmax - gamma_j} within fp32, and the
+                // P/A epilogue needs no exponential per element
+                float mx = fmaxf(g0, g1), mn = fminf(g0, g1);
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                }
+                constexpr float kLog2e = 1.4426950408889634f;
+                *reinterpret_cast<float2*>(vec + r) =
+                    make_float2(ex2((mx - g0) * kLog2e), ex2((mx - g1) * kLog2e));
+                if (lane == 0) {
+                    vec[64] = mx;
+                    vec[65] = (mx - mn < 80.f) ? 1.f : 0.f;
+                }
             }
             {
                 const bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag);
@@ -452,7 +478,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             // scratch). Inside the diagonal blocks P keeps j <= r; A needs no mask
             // (the solve reads only its strictly lower part). Every element is
             // computed branch-free (exponent clamped at 0 so masked or unread
-            // entries stay finite), then selected.
+            // entries stay finite), then selected. When the chunk's decay range is
+            // below 80 the decay factors split into a row and a column factor.
             {
                 const int rb = warp & 1, cb = half;  // row and column block of this warp
                 const bool is_p = row < 64;
@@ -465,12 +492,24 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     const float gr = gam[r];
                     const float fr = is_p ? rq[r] : bet[r] * rk[r];
                     const int lim = (is_p && rb == cb) ? r : 64;  // keep j <= lim
+                    if (vec[65] != 0.f) {
+                        // factored decay: row factor e^{gamma_r - gmax} <= 1, column
+                        // factors e^{gmax - gamma_j} < e^80 from the scan
+                        const float frr = fr * ex2((gr - vec[64]) * 1.4426950408889634f);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = j0 + e;
-                        const float ex = __expf(fminf(gr - gam[j], 0.f));
-                        const float val = ex * (fr * rk[j]) * x[e];
-                        x[e] = (j <= lim) ? val : 0.f;
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = j0 + e;
+                            const float val = (frr * (vec[j] * rk[j])) * x[e];
+                            x[e] = (j <= lim) ? val : 0.f;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = j0 + e;
+                            const float ex = __expf(fminf(gr - gam[j], 0.f));
+                            const float val = ex * (fr * rk[j]) * x[e];
+                            x[e] = (j <= lim) ? val : 0.f;
+                        }
                     }
                 } else {
 #pragma unroll
@@ -490,9 +529,10 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             group_sync(kBarPrep, kPrepThreads);
 
             // ---- solve T = (I + A)^-1 by blocks: 16x16 diagonal inverses by forward
-            // substitution (one column per thread, ptid < 64), merged to 32x32
-            // (T_10 = -T_11 A_10 T_00), then to 64x64. Meanwhile ptid 64..191
-            // turn Q into Q~ and ptid 192..255 clear the upper-right 32x32 block.
+            // substitution (one column per thread, ptid < 64), each warp then merging
+            // its pair to 32x32 (T_10 = -T_11 A_10 T_00), then all warps to 64x64.
+            // Meanwhile ptid 64..191 turn Q into Q~ and ptid 192..255 clear the
+            // upper-right 32x32 block.
             if (ptid < 64) {
                 const int o = 16 * (ptid >> 4), c = ptid & 15;
                 float x[16];
@@ -518,29 +558,41 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     sT[(o + r) * kLdA + o + c] = x[r];
                     if (left) sT[(o + r) * kLdA + o + 16 + c] = 0.f;
                 }
+                __syncwarp();
+                // 16 -> 32 for this warp's block pair at op (its T_00 and T_11 were just
+                // written by the warp): Y = A_10 T_00 into the unused upper-right block
+                // of A, then T_10 = -T_11 Y.
+                const int op = 32 * warp;
+                float* Y = sA + op * kLdA + op + 16;  // 16 x 16 scratch, row-major
+                {
+                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const float* a10 = sA + (op + 16) * kLdA + op + 8 * ks;
+                        const float* t00 = sT + (op + 8 * ks) * kLdA + op;
+                        mma_tf32_16x8x8(d0, a10, kLdA, t00, kLdA);
+                        mma_tf32_16x8x8(d1, a10, kLdA, t00 + 8, kLdA);
+                    }
+                    store_acc_16x8(Y, kLdA, d0, 1.f);
+                    store_acc_16x8(Y + 8, kLdA, d1, 1.f);
+                }
+                __syncwarp();
+                {
+                    float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const float* t11 = sT + (op + 16) * kLdA + op + 16 + 8 * ks;
+                        mma_tf32_16x8x8(z0, t11, kLdA, Y + 8 * ks * kLdA, kLdA);
+                        mma_tf32_16x8x8(z1, t11, kLdA, Y + 8 * ks * kLdA + 8, kLdA);
+                    }
+                    store_acc_16x8(sT + (op + 16) * kLdA + op, kLdA, z0, -1.f);
+                    store_acc_16x8(sT + (op + 16) * kLdA + op + 8, kLdA, z1, -1.f);
+                }
             } else if (ptid < 192) {
                 const int rr = ptid - 64, r = rr & 63;
                 scale_row(st + ((rr >> 6) ? kQb1 : kQb0), r, expf(gam[r]) * rq[r]);
             } else {
                 for (int e = ptid - 192; e < 32 * 32; e += 64) sT[(e >> 5) * kLdA + 32 + (e & 31)] = 0.f;
-            }
-            group_sync(kBarPrep, kPrepThreads);
-            // 16 -> 32 for the block pairs at o = 0 and 32 (warps 0-3: pair, 8-column tile):
-            // Y = A_10 T_00 into the unused upper-right block of A, then T_10 = -T_11 Y.
-            if (warp < 4) {
-                const int o = 32 * (warp >> 1), nt = 8 * (warp & 1);
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    mma_tf32_16x8x8(d, sA + (o + 16) * kLdA + o + 8 * ks, kLdA, sT + (o + 8 * ks) * kLdA + o + nt, kLdA);
-                float* Y = sA + o * kLdA + o + 16;  // 16 x 16 scratch, row-major
-                store_acc_16x8(Y + nt, kLdA, d, 1.f);
-                __syncwarp();
-                float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)
-                    mma_tf32_16x8x8(z, sT + (o + 16) * kLdA + o + 16 + 8 * ks, kLdA, Y + 8 * ks * kLdA + nt, kLdA);
-                store_acc_16x8(sT + (o + 16) * kLdA + o + nt, kLdA, z, -1.f);
             }
             group_sync(kBarPrep, kPrepThreads);
             {

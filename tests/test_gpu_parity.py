@@ -49,6 +49,18 @@ def test_prefill_bf16_ragged_with_state(algo):
     assert np.array_equal(hT[n_empty], P.h0[n_empty])  # empty sequence passes its state through
 
 
+@pytest.mark.parametrize("g_scale", [1.6, 4.0])
+def test_prefill_bf16_decay_ranges(g_scale):
+    """Chunks whose decay range (gamma_0 - gamma_63, about 51 * g_scale here) stays
+    below or exceeds the range the tensor-core path factors into row and column
+    terms (80): both ways of forming e^{gamma_r - gamma_j} against the oracle."""
+    P = gi.random_prefill(13, [130, 64, 200], H=2, dk=128, dv=128, g_scale=g_scale, with_h0=True)
+    o, hT = prefill_gpu(P, algo="tensor")
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_BF16
+    assert err(hT, h_ref) <= TOL_BF16
+
+
 @pytest.mark.parametrize("dk,dv", [(16, 16), (64, 128), (128, 64), (32, 96), (48, 80), (128, 128)])
 def test_prefill_fp32_shapes(dk, dv):
     P = gi.random_prefill(2, [70, 5, 129], H=2, dk=dk, dv=dv, dtype="f32", with_h0=True, chunk=32,
