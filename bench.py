@@ -367,8 +367,33 @@ def bench_decode(args, dist, pk):
     total_ms, per = timed(step, steps, stream)
     total_ms = dist.max(total_ms)
     step_ms = total_ms / steps
+    # the same 100 steps captured once in a CUDA graph and replayed (launch cost
+    # of the library call and ctypes marshalling out of the loop)
+    graph_ms = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap):
+                for i in range(steps):
+                    gdn.decode_step(*ins[i], state, out=o)
+        stream.wait_stream(cap)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = dist.max(e0.elapsed_time(e1)) / steps
+        del g
+    except Exception as exc:  # reported, not fatal: the eager number stands
+        graph_ms = f"unavailable: {type(exc).__name__}: {exc}"[:200]
     bytes_step = 2 * N * H * STATE_BYTES + N * H * (4 * D * 2 + 8)
     return {"value": N / (step_ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": step_ms,
+            "ms_per_step_graph": graph_ms,
             "workload": "decode_256x16_d128_100steps",
             "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -376,6 +401,60 @@ def bench_decode(args, dist, pk):
                          "traffic": profiled_traffic("decode_step_kernel", ["decode.cu"], N * H),
                          "algorithmic_bytes": bytes_step},
             "gpu_launches": steps}
+
+
+def bench_varlen(args, dist, pk):
+    """64 packed sequences of 256..32768 tokens (about 1.06 M), 16 heads, h0 and hT."""
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    P = gi.varlen()
+    T = int(P.cu_seqlens[-1])
+    bf = lambda a: torch.from_numpy(a.view("int16")).to(dev).view(torch.bfloat16)
+    q, k, v = bf(P.q), bf(P.k), bf(P.v)
+    g, beta = torch.from_numpy(P.g).to(dev), torch.from_numpy(P.beta).to(dev)
+    cu = torch.from_numpy(P.cu_seqlens).to(dev)
+    h0 = torch.from_numpy(P.h0).to(dev)
+    N = P.N
+    o = torch.empty_like(q)
+    hT = torch.empty_like(h0)
+    ws = torch.empty(gdn.prefill_workspace_size(N, T, H, D, D, CHUNK), dtype=torch.uint8, device=dev)
+    host_cu = torch.from_numpy(P.cu_seqlens)
+    del P
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.prefill(q, k, v, g, beta, cu, initial_state=h0, final_state=hT, out=o, workspace=ws,
+                    cu_seqlens_host=host_cu)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    reps = 5
+    total_ms, _ = timed(step, reps, stream)
+    ms = dist.max(total_ms) / reps
+    flops = T * H * FLOP_PER_TOKEN_HEAD
+    byts = T * H * BYTES_PER_TOKEN_HEAD + 2 * N * H * STATE_BYTES
+    # per-CTA work of the tensor-core kernel: (sequence, head) units in longest-first
+    # order, unit u on CTA u mod grid
+    lens = np.diff(host_cu.numpy().astype(np.int64))
+    order = sorted(range(N), key=lambda n: (-int(lens[n]), n))
+    grid = min(torch.cuda.get_device_properties(dev).multi_processor_count, N * H)
+    work = np.zeros(grid)
+    for u in range(N * H):
+        work[u % grid] += lens[order[u // H]]
+    return {"value": T / (ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": ms,
+            "workload": f"varlen_64seqs_{T}tok_h16_d128_bf16_h0",
+            "tc_roofline": {"achieved": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                            "peak": pk["bf16_tflops"],
+                            "frac": flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops"]},
+            "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "algorithmic_bytes": byts},
+            "tail_imbalance": {"max_over_mean_cta_tokens": float(work.max() / work.mean()),
+                               "ctas": grid}}
 
 
 def bench_layer(args, dist, pk):
@@ -454,6 +533,7 @@ def run_ours(args, dist: Dist):
     if not args.no_extras:
         extras["decode"] = bench_decode(args, dist, pk)
         extras["layer"] = bench_layer(args, dist, pk)
+        extras["varlen"] = bench_varlen(args, dist, pk)
     clocks.active = False
     clk = clocks.stop()
 
