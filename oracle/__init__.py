@@ -4,8 +4,10 @@ A plain fp64 restatement (C, threads over (sequence, head)) of what the mixer
 computes, used by the tests, the smoke check and the benchmark's CPU baseline.
 The CUDA library never imports or links it, and it shares no code with it.
 
-Functions here only marshal numpy arrays into the C library built from
-``gdn_oracle.c``; see that file's header for the sources each step follows.
+The recurrence, chunked evaluator and conv marshal numpy arrays into the C
+library built from ``gdn_oracle.c`` (see that file's header for the sources
+each step follows). The gated RMSNorm output is plain numpy in fp64, and the
+decode layer step is the composition of the conv, the recurrence and that norm.
 """
 from __future__ import annotations
 
@@ -139,3 +141,53 @@ def conv_silu(x, w, cu_seqlens, *, dtype: str, state_in=None, apply_silu: bool =
     if rc != 0:
         raise ValueError("oracle conv: bad arguments")
     return y, st_out
+
+
+def _to_f64(a: np.ndarray, kind: str) -> np.ndarray:
+    """Inputs as float64; kind 'bf16' decodes uint16 bit patterns exactly."""
+    if kind == "bf16":
+        b = np.ascontiguousarray(a, dtype=np.uint16).astype(np.uint32) << 16
+        return b.view(np.float32).astype(np.float64)
+    return np.asarray(a, dtype=np.float64)
+
+
+def gated_rmsnorm(y, z, w, *, dtype: str, eps: float = 1e-6):
+    """Output gate of the linear-attention layer ("Qwen3.5 ... linear-attention
+    hybrid", 7.6.2, gated RMSNorm output; RMSNorm as in 7.6.3):
+        out = y / sqrt(mean(y^2) + eps) * w * SiLU(z),   SiLU(z) = z / (1 + e^-z)
+    over the last axis (one head's d_v values), in fp64. The scale vector w is
+    applied as given (a caller with zero-centred parameters passes 1 + w).
+    y, z [..., dv] in `dtype` encoding, w [dv] float. Returns float64."""
+    y = _to_f64(y, dtype)
+    z = _to_f64(z, dtype)
+    w = np.asarray(w, dtype=np.float64)
+    ms = np.mean(y * y, axis=-1, keepdims=True)
+    return y / np.sqrt(ms + eps) * w * (z / (1.0 + np.exp(-z)))
+
+
+def decode_layer_step(x, conv_w, conv_state, g, beta, state, *, dtype: str, H: int, dk: int,
+                      dv: int, z=None, norm_w=None, norm_eps: float = 1e-6, scale: float = 1.0,
+                      qk_l2norm: bool = True, eps: float = 1e-6):
+    """One decode token of the whole mixer per sequence: the conv update over the
+    fused [q | k | v] channels from the conv state (then SiLU and the per-head L2
+    norm of q and k), one step of the gated delta rule from `state`, and, when z
+    is given, the gated RMSNorm output. Composed from `conv_silu`, `recurrence`
+    and `gated_rmsnorm`, each run as documented there.
+
+    x [N, C] (C = 2 H dk + H dv), conv_w [C, K], conv_state [N, C, K-1] in `dtype`
+    encoding; g, beta [N, H]; state [N, H, dk, dv] float.
+    Returns (o [N, H, dv], new conv state [N, C, K-1], new state [N, H, dk, dv]),
+    all float64."""
+    N, C = x.shape
+    cu = np.arange(N + 1, dtype=np.int64)
+    y, cs = conv_silu(x, conv_w, cu, dtype=dtype, state_in=conv_state, qk_l2norm=qk_l2norm,
+                      n_qk=2 * H * dk, head_dim=dk, eps=eps, threads=1)
+    q = y[:, :H * dk].reshape(N, H, dk)
+    k = y[:, H * dk:2 * H * dk].reshape(N, H, dk)
+    v = y[:, 2 * H * dk:].reshape(N, H, dv)
+    o, hT = recurrence(q, k, v, np.asarray(g, np.float64), np.asarray(beta, np.float64), cu,
+                       dtype="f64", h0=np.asarray(state, np.float64), scale=scale,
+                       qk_l2norm=False, threads=1)
+    if z is not None:
+        o = gated_rmsnorm(o, z, norm_w, dtype=dtype, eps=norm_eps)
+    return o, cs, hT

@@ -6,8 +6,8 @@ bound and the independent fp64 chunkwise evaluator.
 The recurrence pinned here is the decay-first gated delta rule of the
 Qwen3.5-MoE source walkthrough, section 4.3; in matrix form (state [d_k, d_v])
 S_t = a_t (I - b_t k_t k_t^T) S_{t-1} + b_t k_t v_t^T and o_t = S_t^T q_t,
-the transpose of the spec form S_t = a_t S_{t-1}(I - b_t k k^T) + b_t v k^T,
-o_t = S_t q_t written with the state as [d_v, d_k].
+the transpose of the form S_t = a_t S_{t-1}(I - b_t k k^T) + b_t v k^T,
+o_t = S_t q_t, in which the state is [d_v, d_k].
 
 The last test plants each plausible mistake in the oracle (on the CPU) and
 checks that at least one pin catches it.
@@ -116,7 +116,7 @@ def pin_decay_first(rec):
 
 
 def _unrolled(q, k, v, alpha, beta, S0):
-    """North-star orientation P = S^T ([d_v, d_k]); P_t = P_0 prod B_j +
+    """Transposed orientation P = S^T ([d_v, d_k]); P_t = P_0 prod B_j +
     sum_i b_i v_i k_i^T prod_{j>i} B_j with B_j = a_j (I - b_j k_j k_j^T),
     every product formed explicitly left to right. Returns (o [T,dv], P_T)."""
     T, dk = k.shape
@@ -367,6 +367,76 @@ def test_bf16_decode_is_exact():
     y, _ = oracle.conv_silu(bits[:, None], gdn_inputs.to_bf16_bits(np.array([[0, 0, 0, 1.0]], np.float32)),
                             [0, len(vals)], dtype="bf16", apply_silu=False)
     assert np.array_equal(y[:, 0], widened)
+
+
+# --------------------------------------------------------------------------
+# Gated RMSNorm output ("Qwen3.5 ... linear-attention hybrid", 7.6.2 and 7.6.3)
+# --------------------------------------------------------------------------
+
+def test_gated_rmsnorm_hand_example():
+    # one head, d_v = 2: y = (3, 4), mean(y^2) = 12.5, eps = 0.5 -> rms = sqrt(13)
+    # z = (0, ln 3): SiLU(0) = 0, SiLU(ln 3) = ln 3 * 3/4; w = (2, 5)
+    y = np.array([[3.0, 4.0]])
+    z = np.array([[0.0, math.log(3.0)]])
+    out = oracle.gated_rmsnorm(y, z, np.array([2.0, 5.0]), dtype="f64", eps=0.5)
+    want = np.array([[0.0, 4.0 / math.sqrt(13.0) * 5.0 * math.log(3.0) * 0.75]])
+    assert np.abs(out - want).max() < 1e-15
+
+
+def test_gated_rmsnorm_per_head_scale_invariance():
+    # eps = 0: scaling one head's y by any c > 0 leaves every output unchanged, so
+    # the norm runs over that head's d_v values only (not over tokens or heads)
+    r = _rng(21)
+    y, z, w = r.normal(size=(5, 3, 8)), r.normal(size=(5, 3, 8)), r.normal(size=8)
+    base = oracle.gated_rmsnorm(y, z, w, dtype="f64", eps=0.0)
+    y2 = y.copy()
+    y2[2, 1] *= 37.0
+    assert np.abs(oracle.gated_rmsnorm(y2, z, w, dtype="f64", eps=0.0) - base).max() < 1e-13
+    y3 = y.copy()
+    y3[:, 1] *= 0.01
+    assert np.abs(oracle.gated_rmsnorm(y3, z, w, dtype="f64", eps=0.0) - base).max() < 1e-13
+
+
+def test_gated_rmsnorm_gate_is_silu():
+    # SiLU(z) - SiLU(-z) = z: the difference of the two gated outputs is the plain
+    # normalised, scaled y times z; w = 1 and eps = 0 make it unit-RMS per head
+    r = _rng(22)
+    y, z = r.normal(size=(4, 2, 16)), r.normal(size=(4, 2, 16))
+    w = np.ones(16)
+    d = oracle.gated_rmsnorm(y, z, w, dtype="f64", eps=0.0) - \
+        oracle.gated_rmsnorm(y, -z, w, dtype="f64", eps=0.0)
+    ratio = d / z
+    assert np.abs(np.sqrt(np.mean(ratio ** 2, axis=-1)) - 1.0).max() < 1e-12
+    assert np.abs(ratio * np.sqrt(np.mean(y ** 2, axis=-1, keepdims=True)) - y).max() < 1e-12
+
+
+def test_decode_layer_steps_equal_packed_layer():
+    # Token-by-token decode of the whole mixer (conv state and recurrent state
+    # carried across calls) equals the packed path: conv over the sequence, then
+    # the recurrence over it -- so the conv-state shift and hand-off are right.
+    r = _rng(23)
+    H, dk, dv, K, T = 2, 4, 3, 4, 7
+    C = 2 * H * dk + H * dv
+    x = r.normal(size=(T, C))
+    cw = r.normal(size=(C, K))
+    cs0 = r.normal(size=(1, C, K - 1))
+    h0 = r.normal(size=(1, H, dk, dv)) * 0.3
+    g = -np.abs(r.normal(size=(T, H))) * 0.3
+    b = 1.0 / (1.0 + np.exp(-r.normal(size=(T, H))))
+    y, cs_ref = oracle.conv_silu(x, cw, [0, T], dtype="f64", state_in=cs0, qk_l2norm=True,
+                                 n_qk=2 * H * dk, head_dim=dk, eps=1e-6)
+    o_ref, h_ref = oracle.recurrence(y[:, :H * dk].reshape(T, H, dk),
+                                     y[:, H * dk:2 * H * dk].reshape(T, H, dk),
+                                     y[:, 2 * H * dk:].reshape(T, H, dv), g, b, [0, T],
+                                     dtype="f64", h0=h0, qk_l2norm=False)
+    cs, st = cs0, h0
+    for t in range(T):
+        o, cs, st = oracle.decode_layer_step(x[t:t + 1], cw, cs, g[t:t + 1], b[t:t + 1], st,
+                                             dtype="f64", H=H, dk=dk, dv=dv)
+        assert np.abs(o[0] - o_ref[t]).max() < 1e-12
+    assert np.abs(cs - cs_ref).max() < 1e-15 and np.abs(st - h_ref).max() < 1e-12
+    # the final conv state is the last K-1 inputs, oldest first
+    assert np.array_equal(cs[0], x[T - (K - 1):].T)
 
 
 # --------------------------------------------------------------------------
