@@ -457,6 +457,86 @@ def bench_varlen(args, dist, pk):
                                "ctas": grid}}
 
 
+def bench_decode_layer(args, dist, pk):
+    """The whole mixer for one decode token (conv update + SiLU + L2 norm +
+    recurrent step + gated RMSNorm output) in one kernel: 256 sequences x 16
+    heads, d=128, conv k=4, 100 in-place steps."""
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    N, steps, K = 256, 100, 4
+    C = 3 * H * D
+    r = np.random.default_rng(7)
+    bf = lambda a: torch.from_numpy(gi.to_bf16_bits(a.astype(np.float32)).view("int16")).to(dev) \
+        .view(torch.bfloat16)
+    state = torch.from_numpy(gi.decode_state(N, H, D)).to(dev)
+    conv_state = bf(r.normal(size=(N, C, K - 1)))
+    conv_w = bf(r.normal(size=(C, K)) * 0.5)
+    norm_w = torch.ones(D, dtype=torch.float32, device=dev)
+    ins = []
+    for s_ in range(8):  # a few distinct inputs, cycled
+        ins.append((bf(r.normal(size=(N, C))), torch.from_numpy(
+            (-np.log1p(np.exp(r.normal(size=(N, H))))).astype(np.float32)).to(dev),
+            torch.from_numpy((1 / (1 + np.exp(-r.normal(size=(N, H))))).astype(np.float32)).to(dev),
+            bf(r.normal(size=(N, H, D)))))
+    o = torch.empty((N, H, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    it = iter(range(10 ** 9))
+
+    def step():
+        x, g, b, z = ins[next(it) % len(ins)]
+        gdn.decode_layer_step(x, conv_w, conv_state, g, b, state, H=H, dk=D, dv=D, z=z,
+                              norm_w=norm_w, out=o)
+
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    total_ms, _ = timed(step, steps, stream)
+    step_ms = dist.max(total_ms) / steps
+    # state in and out, x, conv state in and out, z, o, gates; taps once
+    bytes_step = (2 * N * H * STATE_BYTES + N * C * 2 + 2 * N * C * (K - 1) * 2
+                  + 2 * N * H * D * 2 + N * H * 8 + C * K * 2)
+    return {"value": N / (step_ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": step_ms,
+            "workload": "decode_layer_256x16_d128_conv4_gated_100steps",
+            "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "algorithmic_bytes": bytes_step},
+            "gpu_launches": steps}
+
+
+def bench_gated_norm(args, dist, pk):
+    """Gated RMSNorm output over the long-prefill output: 8 x 16384 tokens x 16
+    heads, d_v = 128, bf16 (read o and z, write the gated output)."""
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    dev = torch.device("cuda", dist.local)
+    rows = SEQS * SEQ_LEN * H
+    gen = torch.Generator(device=dev).manual_seed(11)
+    y = torch.randn((rows, D), generator=gen, device=dev).to(torch.bfloat16)
+    z = torch.randn((rows, D), generator=gen, device=dev).to(torch.bfloat16)
+    w = torch.ones(D, dtype=torch.float32, device=dev)
+    out = torch.empty_like(y)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.gated_rmsnorm(y, z, w, out=out)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    reps = 10
+    total_ms, _ = timed(step, reps, stream)
+    ms = dist.max(total_ms) / reps
+    byts = 3 * rows * D * 2
+    return {"ms": ms, "workload": f"gated_rmsnorm_{rows}x{D}_bf16",
+            "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "algorithmic_bytes": byts}}
+
+
 def bench_layer(args, dist, pk):
     """0.8B-shaped layer prefill: conv + SiLU + L2 norm, then chunked prefill."""
     import torch
@@ -534,6 +614,8 @@ def run_ours(args, dist: Dist):
         extras["decode"] = bench_decode(args, dist, pk)
         extras["layer"] = bench_layer(args, dist, pk)
         extras["varlen"] = bench_varlen(args, dist, pk)
+        extras["decode_layer"] = bench_decode_layer(args, dist, pk)
+        extras["gated_rmsnorm"] = bench_gated_norm(args, dist, pk)
     clocks.active = False
     clk = clocks.stop()
 

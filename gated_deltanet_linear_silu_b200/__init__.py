@@ -12,6 +12,9 @@ Operations (the Qwen3.5 linear-attention layer's token mixer):
   prefill       chunked gated delta rule over packed sequences (cu_seqlens),
                 optional initial state, fp32 final state.
   decode_step   one token per sequence, fp32 state updated in place.
+  decode_layer_step  the whole mixer for one decode token (conv update, SiLU,
+                L2 norm, recurrent step, optional gated RMSNorm) in one kernel.
+  gated_rmsnorm the gated RMSNorm output for prefill outputs.
 """
 from __future__ import annotations
 
@@ -58,6 +61,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, i32, f32,
                                       vp, vp]
+        L.gdn_decode_layer_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, f32, i32, i32,
+                                            i32, i32, f32, i32, f32, vp, vp]
+        L.gdn_decode_layer_step.restype = i32
+        L.gdn_gated_rmsnorm.argtypes = [vp, vp, vp, i32, i64, i32, f32, vp, vp]
+        L.gdn_gated_rmsnorm.restype = i32
         L.gdn_decode_step.restype = i32
         L.gdn_status_string.argtypes = [i32]
         L.gdn_status_string.restype = ctypes.c_char_p
@@ -222,6 +230,41 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
                                _ptr(state), N, H, dk, dv, float(scale), int(qk_l2norm), float(eps),
                                _ptr(o), _stream(q.device))
     _check(st, "gdn_decode_step")
+    return o
+
+
+def decode_layer_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: Optional[torch.Tensor],
+                      g: torch.Tensor, beta: torch.Tensor, state: torch.Tensor, *, H: int, dk: int,
+                      dv: int, z: Optional[torch.Tensor] = None,
+                      norm_w: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
+                      scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One decode token of the whole mixer per sequence. x [N, C] fused
+    [q | k | v] projections (C = 2 H dk + H dv), conv_w [C, K], conv_state
+    [N, C, K-1] and state [N, H, dk, dv] fp32 updated in place, g/beta [N, H]
+    fp32, optional gate z [N, H, dv] with norm_w [dv] fp32. Returns o [N, H, dv]."""
+    N, C = x.shape
+    K = conv_w.shape[1]
+    o = torch.empty((N, H, dv), dtype=x.dtype, device=x.device) if out is None else out
+    _cuda(x, conv_w, conv_state, g, beta, state, z, norm_w, o)
+    st = lib().gdn_decode_layer_step(_ptr(x), _ptr(conv_w), _ptr(conv_state), K, _dtype_code(x),
+                                     _ptr(g), _ptr(beta), _ptr(state), _ptr(z), _ptr(norm_w),
+                                     float(norm_eps), N, H, dk, dv, float(scale), int(qk_l2norm),
+                                     float(eps), _ptr(o), _stream(x.device))
+    _check(st, "gdn_decode_layer_step")
+    return o
+
+
+def gated_rmsnorm(y: torch.Tensor, z: torch.Tensor, w: torch.Tensor, *, eps: float = 1e-6,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out = y / sqrt(mean(y^2) + eps) * w * SiLU(z) over the last axis (d_v).
+    y, z [..., dv] bf16 or fp32, w [dv] fp32 (applied as given)."""
+    dv = y.shape[-1]
+    o = torch.empty_like(y) if out is None else out
+    _cuda(y, z, w, o)
+    st = lib().gdn_gated_rmsnorm(_ptr(y), _ptr(z), _ptr(w), _dtype_code(y), y.numel() // dv, dv,
+                                 float(eps), _ptr(o), _stream(y.device))
+    _check(st, "gdn_gated_rmsnorm")
     return o
 
 

@@ -189,8 +189,44 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dt
         return GDN_ERR_INVALID_ARG;
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
-    gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, dk, dv, scale, qk_l2norm, eps, o};
+    gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, dk, dv, scale, qk_l2norm, eps, o,
+                      nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0.f};
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv_state, int K,
+                                   gdn_dtype_t dtype, const float* g, const float* beta, float* state,
+                                   const void* z, const float* norm_w, float norm_eps, int N, int H,
+                                   int dk, int dv, float scale, int qk_l2norm, float eps, void* o,
+                                   void* stream) {
+    if (!dtype_ok(dtype) || N < 0 || H <= 0 || K < 1) return GDN_ERR_INVALID_ARG;
+    if (K > 4) return GDN_ERR_UNSUPPORTED;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (N == 0) return GDN_OK;
+    if (!x || !conv_w || !g || !beta || !state || !o || (K > 1 && !conv_state))
+        return GDN_ERR_INVALID_ARG;
+    if (z && !norm_w) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(o) || !aligned16(state) || !aligned16(z) || !aligned16(norm_w) ||
+        !aligned16(conv_w) || !aligned16(conv_state))
+        return GDN_ERR_INVALID_ARG;
+    if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if (z && !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
+    gdn::DecodeArgs a{nullptr, nullptr, nullptr, dtype == GDN_BF16, g, beta, state, N, H, dk, dv,
+                      scale, qk_l2norm, eps, o, x, conv_w, conv_state, K, z, norm_w, norm_eps};
+    return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
+}
+
+gdn_status_t gdn_gated_rmsnorm(const void* y, const void* z, const float* w, gdn_dtype_t dtype,
+                               int64_t rows, int dv, float eps, void* out, void* stream) {
+    if (!dtype_ok(dtype) || rows < 0) return GDN_ERR_INVALID_ARG;
+    if (dv < 4 || dv > 256 || dv % 4 != 0) return GDN_ERR_UNSUPPORTED;
+    if (rows == 0) return GDN_OK;
+    if (!y || !z || !w || !out) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(z) || !aligned16(w) || !aligned16(out)) return GDN_ERR_INVALID_ARG;
+    if (!(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    gdn::GatedNormArgs a{y, z, w, dtype == GDN_BF16, rows, dv, eps, out};
+    return from_cuda(gdn::launch_gated_rmsnorm(a, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -61,6 +61,15 @@ __device__ __forceinline__ float group_sum(float x, int width) {
     return x;
 }
 
+// 16-byte asynchronous global -> shared copy (both addresses 16-byte aligned),
+// its commit and the wait for every committed group of this thread.
+__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all_groups() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Index of the sequence that contains token t: largest n with cu[n] <= t.
 __device__ __forceinline__ int find_sequence(const int32_t* cu, int N, int64_t t) {
     int lo = 0, hi = N - 1;

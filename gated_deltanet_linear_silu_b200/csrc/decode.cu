@@ -8,13 +8,23 @@
 //   delta = beta (v - m),  o = alpha b + (k^ . q^) delta,  S' = alpha S + k^ delta^T.
 // Layout: thread (rg, cg) owns columns [4cg, 4cg+4) of rows [rg*RPT, rg*RPT+RPT);
 // a warp reads whole 512-byte state rows (float4 per lane), fully coalesced.
+//
+// The same kernel runs the whole mixer for the decode token when CONV is set
+// ("7.6 Qwen3.5: linear-attention hybrid", 7.6.2): the CTA of (n, h) owns the
+// conv channels of its head's q, k and v, so it applies the causal conv to the
+// token's fused projections against the conv state, shifts that state, and
+// applies SiLU before the recurrent step -- q, k, v never leave the SM. With a
+// gate z the output goes through the gated RMSNorm of 7.6.2 (RMSNorm as in
+// 7.6.3, scale vector as given) on the way out.
 #include "common.cuh"
 #include "launch.h"
 
 namespace gdn {
 namespace {
 
-template <typename T, int RPT>
+__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
+
+template <typename T, int RPT, bool CONV>
 __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
     extern __shared__ float sm[];
     const int dk = a.dk, dv = a.dv;
@@ -29,21 +39,84 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
     float* ks = qs + dk;         // [dk]
     float* red = ks + dk;        // [2][RG][dv]
     float* scal = red + 2 * RG * dv;  // [4]: inv_k, q_scale, kq
+    float* vs = scal + 4;        // [dv] (CONV only)
 
-    // 1. Issue the state loads first: they are the bulk of the traffic.
+    // 0. (whole-mixer step) the conv inputs of this head's q, k, v channels -- x,
+    // the taps and the conv state, a few KB -- are copied to shared memory
+    // asynchronously ahead of the state's 64 KB, so they are in when needed and
+    // hold no registers meanwhile. Three contiguous channel blocks: q (dk channels
+    // from h*dk), k (dk from H*dk + h*dk), v (dv from 2*H*dk + h*dv).
+    const int nconv = 2 * dk + dv;
+    T* cx_s = reinterpret_cast<T*>(vs + dv);          // [nconv]
+    T* cw_s = cx_s + nconv;                           // [nconv][K]
+    T* cs_s = cw_s + nconv * a.K;                     // [nconv][K-1]
+    if constexpr (CONV) {
+        const int H = a.H, K = a.K;
+        const int n = (int)(nh / H), h = (int)(nh % H);
+        const int64_t C = 2 * H * dk + H * dv;
+        const T* x = static_cast<const T*>(a.x) + n * C;
+        const T* w = static_cast<const T*>(a.conv_w);
+        const T* cs = static_cast<const T*>(a.conv_state) + n * C * (K - 1);
+        constexpr int E = 16 / (int)sizeof(T);  // elements per 16-byte piece
+#pragma unroll
+        for (int b = 0; b < 3; ++b) {
+            const int nb = b < 2 ? dk : dv;                       // channels in the block
+            const int64_t ch0 = b == 0 ? h * dk : (b == 1 ? H * dk + h * dk : 2 * H * dk + h * dv);
+            const int c0 = b == 0 ? 0 : (b == 1 ? dk : 2 * dk);  // first local channel
+            for (int p = tid; p < nb / E; p += blockDim.x) cp_async_16(cx_s + c0 + p * E, x + ch0 + p * E);
+            for (int p = tid; p < nb * K / E; p += blockDim.x)
+                cp_async_16(cw_s + c0 * K + p * E, w + ch0 * K + p * E);
+            for (int p = tid; p < nb * (K - 1) / E; p += blockDim.x)
+                cp_async_16(cs_s + c0 * (K - 1) + p * E, cs + ch0 * (K - 1) + p * E);
+        }
+        cp_async_commit_group();
+    }
+
+    // 1. Issue the state loads: they are the bulk of the traffic.
     float* Sg = a.state + nh * dk * dv;
     float4 s[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r)
         s[r] = __ldcs(reinterpret_cast<const float4*>(Sg + (int64_t)(rg * RPT + r) * dv + 4 * cg));
 
-    const T* qg = static_cast<const T*>(a.q) + nh * dk;
-    const T* kg = static_cast<const T*>(a.k) + nh * dk;
-    for (int i = tid; i < dk; i += blockDim.x) {
-        qs[i] = Elem<T>::load(qg, i);
-        ks[i] = Elem<T>::load(kg, i);
+    float4 v4;
+    if constexpr (CONV) {
+        // causal conv of this head's q, k, v channels against the conv state
+        // (window: the K-1 stored inputs, oldest first, then x); the state shifts
+        // by one and takes x as its newest entry
+        const int H = a.H, K = a.K;
+        const int n = (int)(nh / H), h = (int)(nh % H);
+        const int64_t C = 2 * H * dk + H * dv;
+        T* cs = static_cast<T*>(a.conv_state) + n * C * (K - 1);
+        cp_async_wait_all_groups();
+        __syncthreads();
+        for (int c = tid; c < nconv; c += blockDim.x) {
+            const int64_t ch = c < dk ? h * dk + c : (c < 2 * dk ? H * dk + h * dk + (c - dk)
+                                                                 : 2 * H * dk + h * dv + (c - 2 * dk));
+            const float xt = Elem<T>::load(cx_s, c);
+            float acc = Elem<T>::load(cw_s, c * K + K - 1) * xt;
+            for (int j = 0; j < K - 1; ++j) {
+                const float pj = Elem<T>::load(cs_s, c * (K - 1) + j);
+                acc = fmaf(Elem<T>::load(cw_s, c * K + j), pj, acc);
+                if (j > 0) Elem<T>::store(cs, ch * (K - 1) + j - 1, pj);
+            }
+            if (K > 1) Elem<T>::store(cs, ch * (K - 1) + K - 2, xt);
+            const float y = silu_f(acc);
+            if (c < dk) qs[c] = y;
+            else if (c < 2 * dk) ks[c - dk] = y;
+            else vs[c - 2 * dk] = y;
+        }
+        __syncthreads();
+        v4 = *reinterpret_cast<const float4*>(vs + 4 * cg);
+    } else {
+        const T* qg = static_cast<const T*>(a.q) + nh * dk;
+        const T* kg = static_cast<const T*>(a.k) + nh * dk;
+        for (int i = tid; i < dk; i += blockDim.x) {
+            qs[i] = Elem<T>::load(qg, i);
+            ks[i] = Elem<T>::load(kg, i);
+        }
+        v4 = load4(static_cast<const T*>(a.v) + nh * dv + 4 * cg);
     }
-    const float4 v4 = load4(static_cast<const T*>(a.v) + nh * dv + 4 * cg);
     const float alpha = expf(a.g[nh]);
     const float beta = a.beta[nh];
     __syncthreads();
@@ -100,13 +173,29 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
     d.y = beta * (v4.y - alpha * inv_k * A.y);
     d.z = beta * (v4.z - alpha * inv_k * A.z);
     d.w = beta * (v4.w - alpha * inv_k * A.w);
-    if (rg == 0) {
-        float4 o;
-        o.x = alpha * qsc * B.x + kq * d.x;
-        o.y = alpha * qsc * B.y + kq * d.y;
-        o.z = alpha * qsc * B.z + kq * d.z;
-        o.w = alpha * qsc * B.w + kq * d.w;
-        store4(static_cast<T*>(a.o) + nh * dv + 4 * cg, o);
+    // output: the rg == 0 threads, all in warp 0 (dv / 4 <= 32 columns groups)
+    if (tid < 32) {
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (rg == 0) {
+            o.x = alpha * qsc * B.x + kq * d.x;
+            o.y = alpha * qsc * B.y + kq * d.y;
+            o.z = alpha * qsc * B.z + kq * d.z;
+            o.w = alpha * qsc * B.w + kq * d.w;
+        }
+        if (a.z) {  // gated RMSNorm over this head's dv outputs
+            float ss = o.x * o.x + o.y * o.y + o.z * o.z + o.w * o.w;
+            ss = warp_sum(ss);
+            const float inv = 1.f / sqrtf(ss / (float)dv + a.norm_eps);
+            if (rg == 0) {
+                const float4 z4 = load4(static_cast<const T*>(a.z) + nh * dv + 4 * cg);
+                const float4 w4 = *reinterpret_cast<const float4*>(a.norm_w + 4 * cg);
+                o.x = o.x * inv * w4.x * silu_f(z4.x);
+                o.y = o.y * inv * w4.y * silu_f(z4.y);
+                o.z = o.z * inv * w4.z * silu_f(z4.z);
+                o.w = o.w * inv * w4.w * silu_f(z4.w);
+            }
+        }
+        if (rg == 0) store4(static_cast<T*>(a.o) + nh * dv + 4 * cg, o);
     }
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
@@ -125,9 +214,14 @@ cudaError_t launch_rpt(const DecodeArgs& a, cudaStream_t s) {
     const int cols4 = a.dv / 4;
     const int RG = a.dk / RPT;
     const int threads = cols4 * RG;
-    const size_t smem = sizeof(float) * (2 * a.dk + 2 * RG * a.dv + 4);
+    size_t smem = sizeof(float) * (2 * a.dk + 2 * RG * a.dv + 4 + a.dv);
+    if (a.x)  // conv inputs: x, taps, conv state of the head's channels
+        smem += (size_t)(2 * a.dk + a.dv) * (2 * a.K) * (a.is_bf16 ? 2 : 4);
     const int64_t blocks = (int64_t)a.N * a.H;
-    decode_step_kernel<T, RPT><<<(unsigned)blocks, threads, smem, s>>>(a);
+    if (a.x)
+        decode_step_kernel<T, RPT, true><<<(unsigned)blocks, threads, smem, s>>>(a);
+    else
+        decode_step_kernel<T, RPT, false><<<(unsigned)blocks, threads, smem, s>>>(a);
     return cudaGetLastError();
 }
 

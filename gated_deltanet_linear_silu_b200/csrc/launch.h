@@ -38,8 +38,29 @@ struct DecodeArgs {
     int qk_l2norm;
     float eps;
     void* o;
+    // whole-mixer step (x != nullptr): q, k, v come from the conv update of x
+    const void* x;        // [N, C] fused projections, C = 2*H*dk + H*dv
+    const void* conv_w;   // [C, K]
+    void* conv_state;     // [N, C, K-1], updated in place
+    int K;
+    // gated RMSNorm output (z != nullptr)
+    const void* z;        // [N, H, dv]
+    const float* norm_w;  // [dv]
+    float norm_eps;
 };
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
+
+struct GatedNormArgs {
+    const void* y;
+    const void* z;
+    const float* w;
+    int is_bf16;
+    int64_t rows;
+    int dv;
+    float eps;
+    void* out;
+};
+cudaError_t launch_gated_rmsnorm(const GatedNormArgs& a, cudaStream_t s);
 
 struct PrefillArgs {
     const void* q;

@@ -9,6 +9,10 @@
  *   gdn_prefill      chunked gated delta rule over packed variable-length
  *                    sequences, optional initial state, fp32 final state.
  *   gdn_decode_step  one recurrent token per sequence, state updated in place.
+ *   gdn_decode_layer_step  the whole mixer for one decode token: conv update
+ *                    from the conv state, SiLU, L2 norm, the recurrent step
+ *                    and (optionally) the gated RMSNorm output, in one kernel.
+ *   gdn_gated_rmsnorm  the gated RMSNorm output for prefill outputs.
  *
  * Sources (page title, section):
  *   [R] "Qwen3.5-MoE source walkthrough", 4.3 Qwen3_5MoeGatedDeltaNet: the
@@ -22,6 +26,10 @@
  *   [C] "7.6 Qwen3.5: linear-attention hybrid", 7.6.2: depthwise causal
  *       Conv1d, kernel 4, padding 3, over conv_dim = 2*key_dim + value_dim
  *       channels; L2 normalisation of q and k before the recurrence.
+ *   [G] same page, 7.6.2 (gated RMSNorm output): o = RMSNorm(y) * SiLU(z), z
+ *       a separate projection of the layer input; 7.6.3: RMSNorm(x) =
+ *       x / sqrt(mean(x^2) + eps) times a per-feature scale (stored there as
+ *       1 + w, zero-centred).
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
@@ -211,6 +219,48 @@ GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v
                              const float* g, const float* beta, float* state,
                              int N, int H, int dk, int dv, float scale, int qk_l2norm,
                              float eps, void* o, void* stream);
+
+/*
+ * The whole mixer for one decode token per sequence, in one kernel. [C] [R] [G] [P]
+ *
+ * For each sequence n the fused channels x[n] = [q | k | v] (C = 2*H*dk + H*dv,
+ * head-major inside each block) go through the causal conv against the
+ * sequence's conv state (the K-1 previous inputs, oldest first):
+ *   y_c = w[c, K-1] * x[n, c] + sum_{j<K-1} w[c, j] * conv_state[n, c, j]
+ * after which conv_state[n, c] shifts by one and takes x[n, c] as its newest
+ * entry; then SiLU, the L2 norm of q and k (when qk_l2norm), and the recurrent
+ * step of gdn_decode_step on state[n]. When z is given the output is gated:
+ *   o = y / sqrt(mean(y^2) + norm_eps) * norm_w * SiLU(z)   per (n, head),
+ * norm_w applied as given (a zero-centred scale w is passed as 1 + w).
+ *
+ *   x           [N, C]            dtype   the token's fused projections (pre-conv)
+ *   conv_w      [C, K]            dtype   depthwise taps, K in 1..4
+ *   conv_state  [N, C, K-1]       dtype   updated in place (ignored when K == 1)
+ *   g, beta     [N, H]            fp32
+ *   state       [N, H, dk, dv]    fp32    updated in place
+ *   z           [N, H, dv]        dtype   nullable: no gate
+ *   norm_w      [dv]              fp32    required when z is given
+ *   o           [N, H, dv]        dtype   output
+ * Supported: dk, dv in {16, 32, ..., 128}. No buffer may overlap another.
+ */
+GDN_API gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv_state, int K,
+                                           gdn_dtype_t dtype, const float* g, const float* beta,
+                                           float* state, const void* z, const float* norm_w,
+                                           float norm_eps, int N, int H, int dk, int dv,
+                                           float scale, int qk_l2norm, float eps, void* o,
+                                           void* stream);
+
+/*
+ * Gated RMSNorm output over rows of dv features (a row = one (token, head)). [G]
+ *   out[r] = y[r] / sqrt(mean(y[r]^2) + eps) * w * SiLU(z[r]),  SiLU(z) = z / (1 + e^-z)
+ * w is applied as given (a zero-centred scale is passed as 1 + w).
+ *
+ *   y, z, out   [rows, dv]   dtype   (out may alias y)
+ *   w           [dv]         fp32
+ * Supported: dv a multiple of 4, 4 <= dv <= 256.
+ */
+GDN_API gdn_status_t gdn_gated_rmsnorm(const void* y, const void* z, const float* w, gdn_dtype_t dtype,
+                                       int64_t rows, int dv, float eps, void* out, void* stream);
 
 /* Static, human-readable name of a status code. */
 GDN_API const char* gdn_status_string(gdn_status_t status);

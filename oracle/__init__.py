@@ -188,6 +188,6 @@ def decode_layer_step(x, conv_w, conv_state, g, beta, state, *, dtype: str, H: i
     o, hT = recurrence(q, k, v, np.asarray(g, np.float64), np.asarray(beta, np.float64), cu,
                        dtype="f64", h0=np.asarray(state, np.float64), scale=scale,
                        qk_l2norm=False, threads=1)
-    if z is not None:
-        o = gated_rmsnorm(o, z, norm_w, dtype=dtype, eps=norm_eps)
+    if z is not None:  # o is already fp64; z arrives in the inputs' encoding
+        o = gated_rmsnorm(o, _to_f64(z, dtype), norm_w, dtype="f64", eps=norm_eps)
     return o, cs, hT

@@ -245,6 +245,95 @@ def test_conv_state_in_place_and_continuation():
 
 
 # ----------------------------------------------------------------------------
+# gated RMSNorm output, whole-mixer decode step
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+@pytest.mark.parametrize("dv", [128, 64, 256, 20])
+def test_gated_rmsnorm_matches_oracle(kind, dv):
+    r = np.random.default_rng(31)
+    rows = 1000 + 7
+    y = (r.normal(size=(rows, dv)) * 3).astype(np.float32)
+    z = (r.normal(size=(rows, dv)) * 2).astype(np.float32)
+    w = (1.0 + 0.1 * r.normal(size=dv)).astype(np.float32)
+    yb, zb = (gi.to_bf16_bits(y), gi.to_bf16_bits(z)) if kind == "bf16" else (y, z)
+    out = gdn.gated_rmsnorm(dev_tensor(yb, kind), dev_tensor(zb, kind),
+                            torch.from_numpy(w).to(DEV), eps=1e-6)
+    ref = oracle.gated_rmsnorm(yb, zb, w, dtype=kind, eps=1e-6)
+    assert err(host(out), ref) <= (TOL_BF16 if kind == "bf16" else 1e-5)
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+@pytest.mark.parametrize("gate", [False, True])
+@pytest.mark.parametrize("K", [4, 2])
+def test_decode_layer_step_matches_oracle(kind, gate, K):
+    """Five decode tokens through the fused kernel (conv state and recurrent state
+    carried in place) against the oracle's conv + recurrence + gate."""
+    r = np.random.default_rng(32)
+    N, H, dk, dv = 5, 3, 64, 128
+    C = 2 * H * dk + H * dv
+    to = (lambda a: gi.to_bf16_bits(a.astype(np.float32))) if kind == "bf16" else (
+        lambda a: a.astype(np.float32))
+    cw = to(r.normal(size=(C, K)) * 0.5)
+    cs = to(r.normal(size=(N, C, K - 1)))
+    st = (r.normal(size=(N, H, dk, dv)) * 0.1).astype(np.float32)
+    nw = (1.0 + 0.1 * r.normal(size=dv)).astype(np.float32)
+    cs_d, st_d = dev_tensor(cs, kind), torch.from_numpy(st).to(DEV)
+    cs_o, st_o = cs, st.astype(np.float64)
+    worst = 0.0
+    for t in range(5):
+        x = to(r.normal(size=(N, C)))
+        z = to(r.normal(size=(N, H, dv))) if gate else None
+        g = (-np.log1p(np.exp(r.normal(size=(N, H))))).astype(np.float32)
+        b = (1.0 / (1.0 + np.exp(-r.normal(size=(N, H))))).astype(np.float32)
+        o = gdn.decode_layer_step(dev_tensor(x, kind), dev_tensor(cw, kind), cs_d,
+                                  torch.from_numpy(g).to(DEV), torch.from_numpy(b).to(DEV), st_d,
+                                  H=H, dk=dk, dv=dv,
+                                  z=None if z is None else dev_tensor(z, kind),
+                                  norm_w=torch.from_numpy(nw).to(DEV) if gate else None)
+        o_ref, cs_n, st_o = oracle.decode_layer_step(x, cw, cs_o, g, b, st_o, dtype=kind, H=H,
+                                                     dk=dk, dv=dv, z=z, norm_w=nw if gate else None)
+        cs_o = to(cs_n) if kind == "bf16" else cs_n  # the conv state is stored in dtype
+        worst = max(worst, err(host(o), o_ref))
+    gdn.check_device_status(DEV)
+    tol = TOL_BF16 if kind == "bf16" else TOL_F32
+    assert worst <= tol
+    assert err(host(st_d), st_o) <= tol
+    assert np.array_equal(host(cs_d), (gi.bf16_bits_to_f32(cs_o) if kind == "bf16" else cs_o)
+                          .astype(np.float32))  # a pure shift: bit exact
+
+
+def test_decode_layer_step_equals_separate_kernels():
+    """The fused step equals conv_silu, then decode_step, then gated_rmsnorm run as
+    three library calls (fp32, same arithmetic order up to rounding)."""
+    r = np.random.default_rng(33)
+    N, H, dk, dv, K = 4, 2, 32, 64, 4
+    C = 2 * H * dk + H * dv
+    x = torch.from_numpy(r.normal(size=(N, C)).astype(np.float32)).to(DEV)
+    cw = torch.from_numpy((r.normal(size=(C, K)) * 0.5).astype(np.float32)).to(DEV)
+    cs = torch.from_numpy(r.normal(size=(N, C, K - 1)).astype(np.float32)).to(DEV)
+    st = torch.from_numpy((r.normal(size=(N, H, dk, dv)) * 0.1).astype(np.float32)).to(DEV)
+    z = torch.from_numpy(r.normal(size=(N, H, dv)).astype(np.float32)).to(DEV)
+    nw = torch.from_numpy((1.0 + 0.1 * r.normal(size=dv)).astype(np.float32)).to(DEV)
+    g = torch.from_numpy((-np.abs(r.normal(size=(N, H)))).astype(np.float32)).to(DEV)
+    b = torch.from_numpy((1.0 / (1.0 + np.exp(-r.normal(size=(N, H))))).astype(np.float32)).to(DEV)
+    cs2, st2 = cs.clone(), st.clone()
+    o = gdn.decode_layer_step(x, cw, cs, g, b, st, H=H, dk=dk, dv=dv, z=z, norm_w=nw)
+    cu = torch.arange(N + 1, dtype=torch.int32, device=DEV)
+    y, _ = gdn.conv_silu(x, cw, cu, conv_state=cs2, conv_state_out=cs2, n_qk_channels=2 * H * dk,
+                         head_dim=dk)
+    q = y[:, :H * dk].reshape(N, H, dk).contiguous()
+    k = y[:, H * dk:2 * H * dk].reshape(N, H, dk).contiguous()
+    v = y[:, 2 * H * dk:].reshape(N, H, dv).contiguous()
+    o2 = gdn.decode_step(q, k, v, g, b, st2, qk_l2norm=False)
+    o2 = gdn.gated_rmsnorm(o2, z, nw)
+    gdn.check_device_status(DEV)
+    assert err(host(o), host(o2)) <= 1e-5
+    assert err(host(st), host(st2)) <= 1e-5
+    assert torch.equal(cs, cs2)
+
+
+# ----------------------------------------------------------------------------
 # full-size workloads
 # ----------------------------------------------------------------------------
 

@@ -439,6 +439,30 @@ def test_decode_layer_steps_equal_packed_layer():
     assert np.array_equal(cs[0], x[T - (K - 1):].T)
 
 
+def test_decode_layer_step_gate_and_input_encoding():
+    # With a gate the step's output is the gated RMSNorm of the ungated output;
+    # bf16-encoded inputs give exactly the result of their decoded fp64 values.
+    import gdn_inputs
+    r = _rng(24)
+    N, H, dk, dv, K = 2, 2, 4, 4, 4
+    C = 2 * H * dk + H * dv
+    bits = lambda a: gdn_inputs.to_bf16_bits(a.astype(np.float32))
+    dec = lambda b: gdn_inputs.bf16_bits_to_f32(b).astype(np.float64)
+    x, cw, cs0 = bits(r.normal(size=(N, C))), bits(r.normal(size=(C, K))), bits(r.normal(size=(N, C, K - 1)))
+    z = bits(r.normal(size=(N, H, dv)))
+    st = r.normal(size=(N, H, dk, dv)) * 0.2
+    g, b = -np.abs(r.normal(size=(N, H))), np.full((N, H), 0.5)
+    nw = 1.0 + 0.1 * r.normal(size=dv)
+    o_b, cs_b, st_b = oracle.decode_layer_step(x, cw, cs0, g, b, st, dtype="bf16", H=H, dk=dk, dv=dv,
+                                               z=z, norm_w=nw)
+    o_f, cs_f, st_f = oracle.decode_layer_step(dec(x), dec(cw), dec(cs0), g, b, st, dtype="f64",
+                                               H=H, dk=dk, dv=dv, z=dec(z), norm_w=nw)
+    assert np.array_equal(o_b, o_f) and np.array_equal(cs_b, cs_f) and np.array_equal(st_b, st_f)
+    o_u, _, _ = oracle.decode_layer_step(dec(x), dec(cw), dec(cs0), g, b, st, dtype="f64", H=H,
+                                         dk=dk, dv=dv)
+    assert np.array_equal(o_f, oracle.gated_rmsnorm(o_u, dec(z), nw, dtype="f64"))
+
+
 # --------------------------------------------------------------------------
 # Pin sensitivity: each planted mistake must fail at least one pin.
 # --------------------------------------------------------------------------
