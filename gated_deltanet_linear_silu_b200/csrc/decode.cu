@@ -22,7 +22,7 @@
 namespace gdn {
 namespace {
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
 template <typename T, int RPT, bool CONV>
 __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
@@ -91,20 +91,49 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
         cp_async_wait_all_groups();
         __syncthreads();
         for (int c = tid; c < nconv; c += blockDim.x) {
-            const int64_t ch = c < dk ? h * dk + c : (c < 2 * dk ? H * dk + h * dk + (c - dk)
-                                                                 : 2 * H * dk + h * dv + (c - 2 * dk));
             const float xt = Elem<T>::load(cx_s, c);
-            float acc = Elem<T>::load(cw_s, c * K + K - 1) * xt;
-            for (int j = 0; j < K - 1; ++j) {
-                const float pj = Elem<T>::load(cs_s, c * (K - 1) + j);
-                acc = fmaf(Elem<T>::load(cw_s, c * K + j), pj, acc);
-                if (j > 0) Elem<T>::store(cs, ch * (K - 1) + j - 1, pj);
+            float acc;
+            if (K == 4) {
+                const float4 w4 = load4(cw_s + 4 * c);  // the channel's four taps at once
+                const float p0 = Elem<T>::load(cs_s, 3 * c), p1 = Elem<T>::load(cs_s, 3 * c + 1),
+                            p2 = Elem<T>::load(cs_s, 3 * c + 2);
+                acc = fmaf(w4.x, p0, fmaf(w4.y, p1, fmaf(w4.z, p2, w4.w * xt)));
+                Elem<T>::store(cs_s, 3 * c, p1);  // shifted state, stored below
+                Elem<T>::store(cs_s, 3 * c + 1, p2);
+                Elem<T>::store(cs_s, 3 * c + 2, xt);
+            } else {
+                float pv[3] = {0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    if (j < K - 1) pv[j] = Elem<T>::load(cs_s, c * (K - 1) + j);
+                acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float in = (j == K - 1) ? xt : (j < K - 1 ? pv[j < 3 ? j : 2] : 0.f);
+                    if (j < K) acc = fmaf(Elem<T>::load(cw_s, c * K + j), in, acc);
+                }
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    if (j < K - 1) Elem<T>::store(cs_s, c * (K - 1) + j, j < K - 2 ? pv[j < 2 ? j + 1 : 2] : xt);
             }
-            if (K > 1) Elem<T>::store(cs, ch * (K - 1) + K - 2, xt);
             const float y = silu_f(acc);
             if (c < dk) qs[c] = y;
             else if (c < 2 * dk) ks[c - dk] = y;
             else vs[c - 2 * dk] = y;
+        }
+        __syncthreads();
+        // the shifted conv state back to global memory, 16 bytes per store
+        if (K > 1) {
+            constexpr int E = 16 / (int)sizeof(T);
+#pragma unroll
+            for (int b = 0; b < 3; ++b) {
+                const int nb = b < 2 ? dk : dv;
+                const int64_t ch0 = b == 0 ? h * dk : (b == 1 ? H * dk + h * dk : 2 * H * dk + h * dv);
+                const int c0 = b == 0 ? 0 : (b == 1 ? dk : 2 * dk);
+                for (int p = tid; p < nb * (K - 1) / E; p += blockDim.x)
+                    *reinterpret_cast<uint4*>(cs + ch0 * (K - 1) + p * E) =
+                        *reinterpret_cast<const uint4*>(cs_s + c0 * (K - 1) + p * E);
+            }
         }
         __syncthreads();
         v4 = *reinterpret_cast<const float4*>(vs + 4 * cg);
