@@ -3,8 +3,9 @@
 // as in 7.6.3):
 //   out = y / sqrt(mean(y^2) + eps) * w * SiLU(z),   SiLU(z) = z / (1 + e^-z).
 // HBM-bound (read y and z, write out, once each): one warp per row, four
-// features per lane per pass, each warp keeping eight rows' loads in flight
-// (raw, streaming) before the first reduction; w stays in registers.
+// features per lane per pass; each warp keeps two batches of eight rows' loads
+// in flight (raw, streaming): the next batch is requested before the current one
+// is reduced and written. w stays in registers.
 #include "common.cuh"
 #include "launch.h"
 
@@ -49,8 +50,11 @@ __global__ void __launch_bounds__(kWarps * 32) gated_rmsnorm_kernel(GatedNormArg
     const T* y = static_cast<const T*>(a.y);
     const T* z = static_cast<const T*>(a.z);
     T* out = static_cast<T*>(a.out);
-    for (int64_t r0 = warp_id * ROWS; r0 < a.rows; r0 += nwarps * ROWS) {
-        Raw4<T> yv[ROWS][QUADS], zv[ROWS][QUADS];
+    const int64_t stride = nwarps * ROWS;
+    // two batches of ROWS rows in flight: the next batch's loads are issued before
+    // the current one is reduced and written
+    Raw4<T> ya[ROWS][QUADS], za[ROWS][QUADS], yb[ROWS][QUADS], zb[ROWS][QUADS];
+    auto load = [&](Raw4<T> (&yv)[ROWS][QUADS], Raw4<T> (&zv)[ROWS][QUADS], int64_t r0) {
 #pragma unroll
         for (int i = 0; i < ROWS; ++i)
 #pragma unroll
@@ -62,6 +66,8 @@ __global__ void __launch_bounds__(kWarps * 32) gated_rmsnorm_kernel(GatedNormArg
                     zv[i][p].load(z + off);
                 }
             }
+    };
+    auto finish = [&](const Raw4<T> (&yv)[ROWS][QUADS], const Raw4<T> (&zv)[ROWS][QUADS], int64_t r0) {
 #pragma unroll
         for (int i = 0; i < ROWS; ++i) {
             float4 v[QUADS];
@@ -88,6 +94,18 @@ __global__ void __launch_bounds__(kWarps * 32) gated_rmsnorm_kernel(GatedNormArg
                 store4(out + (r0 + i) * dv + 4 * qd, o);
             }
         }
+    };
+    int64_t r0 = warp_id * ROWS;
+    if (r0 < a.rows) load(ya, za, r0);
+    while (r0 < a.rows) {
+        const int64_t r1 = r0 + stride;
+        if (r1 < a.rows) load(yb, zb, r1);
+        finish(ya, za, r0);
+        if (r1 >= a.rows) break;
+        const int64_t r2 = r1 + stride;
+        if (r2 < a.rows) load(ya, za, r2);
+        finish(yb, zb, r1);
+        r0 = r2;
     }
 }
 
