@@ -503,6 +503,7 @@ def bench_decode_layer(args, dist, pk):
             "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": profiled_traffic("decode_layer_kernel", ["decode.cu"], N * H),
                          "algorithmic_bytes": bytes_step},
             "gpu_launches": steps}
 
@@ -534,6 +535,7 @@ def bench_gated_norm(args, dist, pk):
     return {"ms": ms, "workload": f"gated_rmsnorm_{rows}x{D}_bf16",
             "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                          "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": profiled_traffic("gated_rmsnorm_kernel", ["gated_norm.cu"], rows),
                          "algorithmic_bytes": byts}}
 
 
@@ -671,6 +673,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqs", type=int, default=SEQS, help="sequences (profiling runs only)")
     ap.add_argument("--seq-len", type=int, default=SEQ_LEN, help="tokens per sequence (profiling)")
+    ap.add_argument("--only", choices=sorted(ONLY), default=None,
+                    help="run one secondary workload alone and print its object (profiling runs)")
     args = ap.parse_args()
     SEQS, SEQ_LEN = args.seqs, args.seq_len
     if args.warmup < 3:
@@ -681,10 +685,20 @@ def main():
         return
     dist.init()
     try:
-        run_ours(args, dist)
+        if args.only:
+            import gated_deltanet_linear_silu_b200 as gdn
+            gdn.lib()
+            res = ONLY[args.only](args, dist, peaks())
+            if dist.rank == 0:
+                print(json.dumps({"only": args.only, **res}), flush=True)
+        else:
+            run_ours(args, dist)
     finally:
         dist.close()
 
+
+ONLY = {"decode": bench_decode, "layer": bench_layer, "varlen": bench_varlen,
+        "decode_layer": bench_decode_layer, "gated_rmsnorm": bench_gated_norm}
 
 if __name__ == "__main__":
     main()
