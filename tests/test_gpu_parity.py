@@ -49,6 +49,30 @@ def test_prefill_bf16_ragged_with_state(algo):
     assert np.array_equal(hT[n_empty], P.h0[n_empty])  # empty sequence passes its state through
 
 
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_degenerate_gates(algo):
+    """beta = 0 leaves only the decay: S_T = e^{sum g} S_0 and o_t = e^{gamma_t} S_0^T q^_t
+    (closed form); with g = 0 as well the state passes through unchanged. Zero q rows give
+    zero outputs."""
+    P = gi.random_prefill(14, [200, 64, 1], H=2, dk=128, dv=128, with_h0=True)
+    P.beta = np.zeros_like(P.beta)
+    P.q[5] = 0
+    o, hT = prefill_gpu(P, algo=algo)
+    q = gi.bf16_bits_to_f32(P.q).astype(np.float64)
+    qn = q / np.sqrt((q * q).sum(-1, keepdims=True) + P.eps)
+    for n in range(P.N):
+        a, b = int(P.cu_seqlens[n]), int(P.cu_seqlens[n + 1])
+        gam = np.cumsum(P.g[a:b].astype(np.float64), axis=0)          # [L, H]
+        h_cf = np.exp(gam[-1])[:, None, None] * P.h0[n]
+        o_cf = np.exp(gam)[:, :, None] * np.einsum("lhi,hij->lhj", qn[a:b], P.h0[n])
+        assert err(hT[n], h_cf) <= TOL_BF16
+        assert err(o[a:b], o_cf) <= TOL_BF16
+    assert np.all(o[5] == 0)
+    P.g = np.zeros_like(P.g)
+    o, hT = prefill_gpu(P, algo=algo)
+    assert err(hT, P.h0) <= TOL_BF16
+
+
 @pytest.mark.parametrize("g_scale", [1.6, 4.0])
 def test_prefill_bf16_decay_ranges(g_scale):
     """Chunks whose decay range (gamma_0 - gamma_63, about 51 * g_scale here) stays
