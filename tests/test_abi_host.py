@@ -135,6 +135,50 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
         gdn.lib()
 
 
+def _layer_step(L, **kw):
+    args = dict(x=FAKE, cw=FAKE, cs=FAKE, K=4, dt=1, g=FAKE, beta=FAKE, st=FAKE, z=None, nw=None,
+                neps=1e-6, N=2, H=16, dk=128, dv=128, scale=1.0, l2=1, eps=1e-6, o=FAKE,
+                stream=None)
+    args.update(kw)
+    return L.gdn_decode_layer_step(*args.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=5), 1), (dict(N=-1), 1), (dict(H=0), 1), (dict(K=0), 1), (dict(K=5), 2),
+    (dict(dk=96 + 8), 2), (dict(dv=256), 2), (dict(x=None), 1), (dict(cs=None), 1),
+    (dict(z=FAKE), 1),                       # a gate needs norm_w
+    (dict(z=FAKE, nw=FAKE, neps=-1.0), 1), (dict(o=ctypes.c_void_p((1 << 20) + 8)), 1),
+    (dict(cs=ctypes.c_void_p((1 << 20) + 2)), 1), (dict(eps=float("nan")), 1),
+])
+def test_decode_layer_step_rejects_bad_arguments(L, kw, expect):
+    assert _layer_step(L, **kw) == expect
+
+
+def test_decode_layer_step_k1_needs_no_conv_state_and_empty_is_noop(L):
+    assert _layer_step(L, N=0) == 0
+    # K = 1 has no conv state: only the state pointer check remains (NULL state -> invalid)
+    assert _layer_step(L, K=1, cs=None, st=None) == 1
+
+
+def _gnorm(L, **kw):
+    args = dict(y=FAKE, z=FAKE, w=FAKE, dt=1, rows=10, dv=128, eps=1e-6, out=FAKE, stream=None)
+    args.update(kw)
+    return L.gdn_gated_rmsnorm(*args.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=9), 1), (dict(rows=-1), 1), (dict(dv=130), 2), (dict(dv=2), 2), (dict(dv=260), 2),
+    (dict(y=None), 1), (dict(w=None), 1), (dict(out=ctypes.c_void_p((1 << 20) + 4)), 1),
+    (dict(eps=-1.0), 1),
+])
+def test_gated_rmsnorm_rejects_bad_arguments(L, kw, expect):
+    assert _gnorm(L, **kw) == expect
+
+
+def test_gated_rmsnorm_empty_is_noop(L):
+    assert _gnorm(L, rows=0, y=None, z=None, w=None, out=None) == 0
+
+
 def test_sizing_helpers_match_printed_figures():
     d = json.load(open(os.path.join(ROOT, "tests", "golden", "pages_sizing.json")))
     for c in d["cases"]:
