@@ -107,9 +107,9 @@ def _softplus(x: np.ndarray) -> np.ndarray:
 
 @dataclasses.dataclass
 class Prefill:
-    """Packed prefill batch. q/k/v are [T_tot, H, d] (uint16 bf16 bits or
-    float32), g/beta [T_tot, H] float32, cu_seqlens [N+1] int32, h0 [N,H,dk,dv]
-    float32 or None."""
+    """Packed prefill batch. q/k are [T_tot, Hk, dk], v [T_tot, H, dv] (uint16
+    bf16 bits or float32), g/beta [T_tot, H] float32, cu_seqlens [N+1] int32,
+    h0 [N,H,dk,dv] float32 or None. Hk = H unless value heads are grouped."""
     name: str
     q: np.ndarray
     k: np.ndarray
@@ -134,6 +134,10 @@ class Prefill:
     @property
     def T_tot(self) -> int:
         return int(self.cu_seqlens[-1])
+
+    @property
+    def Hk(self) -> int:
+        return int(self.q.shape[1])
 
 
 @dataclasses.dataclass
@@ -277,15 +281,18 @@ def decode_step(step: int, N: int = 256, H: int = 16, d: int = 128) -> DecodeSte
 
 def random_prefill(seed: int, lengths, H: int, dk: int, dv: int, dtype: str = "bf16",
                    g_scale: float = 1.0, with_h0: bool = False, h0_std: float = 0.1,
-                   chunk: int = 64, qk_l2norm: bool = True, scale: float = 1.0) -> Prefill:
-    """A small packed prefill problem for parity tests (any shapes)."""
+                   chunk: int = 64, qk_l2norm: bool = True, scale: float = 1.0,
+                   Hk: Optional[int] = None) -> Prefill:
+    """A small packed prefill problem for parity tests (any shapes); Hk < H
+    gives grouped value heads (q, k with Hk heads)."""
+    Hk = H if Hk is None else Hk
     r = np.random.default_rng(np.random.SeedSequence([1000, seed]))
     lengths = np.asarray(lengths, dtype=np.int64)
     cu = np.zeros(len(lengths) + 1, dtype=np.int64)
     cu[1:] = np.cumsum(lengths)
     T_tot = int(cu[-1])
-    q = _normal(r, (T_tot, H, dk))
-    k = _normal(r, (T_tot, H, dk))
+    q = _normal(r, (T_tot, Hk, dk))
+    k = _normal(r, (T_tot, Hk, dk))
     v = _normal(r, (T_tot, H, dv))
     beta = _sigmoid(_normal(r, (T_tot, H)))
     g = (-_softplus(_normal(r, (T_tot, H))) * np.float32(g_scale)).astype(np.float32)

@@ -30,10 +30,10 @@ def lib():
         L = ctypes.CDLL(path)
         vp, i32, f64, i64p = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
         L.gdn_oracle_recurrence_mut.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32,
-                                                i32, f64, i32, f64, vp, i32, vp, vp, i32, i32]
+                                                i32, i32, f64, i32, f64, vp, i32, vp, vp, i32, i32]
         L.gdn_oracle_recurrence_mut.restype = i32
         L.gdn_oracle_chunked.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32, i32,
-                                         f64, i32, f64, vp, i32, vp, vp, i32, i32]
+                                         i32, f64, i32, f64, vp, i32, vp, vp, i32, i32]
         L.gdn_oracle_chunked.restype = i32
         L.gdn_oracle_conv_silu.argtypes = [vp, i32, vp, i32, i64p, i32, i32, i32, vp, i32, vp,
                                            i32, i32, i32, i32, f64, vp, i32]
@@ -65,12 +65,14 @@ def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: floa
                want_o: bool = True, mutation: int = 0):
     """Token-by-token gated delta rule in fp64.
 
-    q,k [T,H,dk], v [T,H,dv] (uint16 bf16 bits when dtype=='bf16', else
+    q,k [T,Hk,dk], v [T,H,dv] (uint16 bf16 bits when dtype=='bf16', else
     float), g/beta [T,H], cu_seqlens [N+1], h0 [N,H,dk,dv] or None.
+    Value head h reads q, k head h // (H // Hk) (grouped value heads; Hk == H
+    is the plain layer).
     Returns (o [T,H,dv] float64 or None, hT [N,H,dk,dv] float64).
     """
-    T, H, dk = q.shape
-    dv = v.shape[2]
+    T, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
     N = cu.shape[0] - 1
     q, dt = _arr(q, dtype)
@@ -82,7 +84,7 @@ def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: floa
     hT = np.empty((N, H, dk, dv), np.float64)
     o = np.empty((T, H, dv), np.float64) if want_o else None
     rc = lib().gdn_oracle_recurrence_mut(
-        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, dk, dv,
+        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, Hk, dk, dv,
         float(scale), int(qk_l2norm), float(eps), _ptr(h0a), h0dt, _ptr(hT), _ptr(o),
         threads or default_threads(), int(mutation))
     if rc != 0:
@@ -95,8 +97,8 @@ def chunked(q, k, v, g, beta, cu_seqlens, *, dtype: str, chunk: int, h0=None,
             threads: Optional[int] = None):
     """fp64 chunkwise (UT-transform) evaluation of the same recurrence; used
     only to check that the chunk algebra equals the token loop."""
-    T, H, dk = q.shape
-    dv = v.shape[2]
+    T, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
     N = cu.shape[0] - 1
     q, dt = _arr(q, dtype)
@@ -108,7 +110,7 @@ def chunked(q, k, v, g, beta, cu_seqlens, *, dtype: str, chunk: int, h0=None,
     hT = np.empty((N, H, dk, dv), np.float64)
     o = np.empty((T, H, dv), np.float64)
     rc = lib().gdn_oracle_chunked(
-        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, dk, dv,
+        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, Hk, dk, dv,
         float(scale), int(qk_l2norm), float(eps), _ptr(h0a), h0dt, _ptr(hT), _ptr(o),
         int(chunk), threads or default_threads())
     if rc != 0:
@@ -167,24 +169,26 @@ def gated_rmsnorm(y, z, w, *, dtype: str, eps: float = 1e-6):
 
 def decode_layer_step(x, conv_w, conv_state, g, beta, state, *, dtype: str, H: int, dk: int,
                       dv: int, z=None, norm_w=None, norm_eps: float = 1e-6, scale: float = 1.0,
-                      qk_l2norm: bool = True, eps: float = 1e-6):
+                      qk_l2norm: bool = True, eps: float = 1e-6, Hk: Optional[int] = None):
     """One decode token of the whole mixer per sequence: the conv update over the
     fused [q | k | v] channels from the conv state (then SiLU and the per-head L2
     norm of q and k), one step of the gated delta rule from `state`, and, when z
     is given, the gated RMSNorm output. Composed from `conv_silu`, `recurrence`
     and `gated_rmsnorm`, each run as documented there.
 
-    x [N, C] (C = 2 H dk + H dv), conv_w [C, K], conv_state [N, C, K-1] in `dtype`
-    encoding; g, beta [N, H]; state [N, H, dk, dv] float.
+    x [N, C] (C = 2 Hk dk + H dv; Hk key heads, default H), conv_w [C, K],
+    conv_state [N, C, K-1] in `dtype` encoding; g, beta [N, H]; state
+    [N, H, dk, dv] float.
     Returns (o [N, H, dv], new conv state [N, C, K-1], new state [N, H, dk, dv]),
     all float64."""
+    Hk = H if Hk is None else Hk
     N, C = x.shape
     cu = np.arange(N + 1, dtype=np.int64)
     y, cs = conv_silu(x, conv_w, cu, dtype=dtype, state_in=conv_state, qk_l2norm=qk_l2norm,
-                      n_qk=2 * H * dk, head_dim=dk, eps=eps, threads=1)
-    q = y[:, :H * dk].reshape(N, H, dk)
-    k = y[:, H * dk:2 * H * dk].reshape(N, H, dk)
-    v = y[:, 2 * H * dk:].reshape(N, H, dv)
+                      n_qk=2 * Hk * dk, head_dim=dk, eps=eps, threads=1)
+    q = y[:, :Hk * dk].reshape(N, Hk, dk)
+    k = y[:, Hk * dk:2 * Hk * dk].reshape(N, Hk, dk)
+    v = y[:, 2 * Hk * dk:].reshape(N, H, dv)
     o, hT = recurrence(q, k, v, np.asarray(g, np.float64), np.asarray(beta, np.float64), cu,
                        dtype="f64", h0=np.asarray(state, np.float64), scale=scale,
                        qk_l2norm=False, threads=1)

@@ -101,7 +101,7 @@ typedef struct {
     const void *g, *beta;
     int gate_dtype;
     const int64_t *cu;
-    int H, dk, dv;
+    int H, Hk, dk, dv; /* H value heads; q, k have Hk heads, each shared by H / Hk value heads */
     double scale;
     int qk_l2norm;
     double eps;
@@ -121,9 +121,10 @@ static void l2_normalise(double *x, int d, double eps) {
 
 static void rec_item(void *vctx, int64_t item) {
     const rec_ctx *c = (const rec_ctx *)vctx;
-    const int H = c->H, dk = c->dk, dv = c->dv;
+    const int H = c->H, Hk = c->Hk, dk = c->dk, dv = c->dv;
     const int64_t n = item / H;
     const int h = (int)(item % H);
+    const int hk = h / (H / Hk); /* the key head this value head reads */
     double *S = (double *)calloc((size_t)dk * dv, sizeof(double)); /* S[i][j], i: key, j: value */
     double *q = (double *)malloc(sizeof(double) * dk);
     double *k = (double *)malloc(sizeof(double) * dk);
@@ -134,7 +135,7 @@ static void rec_item(void *vctx, int64_t item) {
         for (int64_t e = 0; e < (int64_t)dk * dv; ++e) S[e] = load_elem(c->h0, c->h0_dtype, sbase + e);
 
     for (int64_t t = c->cu[n]; t < c->cu[n + 1]; ++t) {
-        const int64_t qk_base = (t * H + h) * (int64_t)dk;
+        const int64_t qk_base = (t * Hk + hk) * (int64_t)dk;
         const int64_t v_base = (t * H + h) * (int64_t)dv;
         for (int i = 0; i < dk; ++i) {
             q[i] = load_elem(c->q, c->dtype, qk_base + i);
@@ -201,19 +202,21 @@ static void rec_item(void *vctx, int64_t item) {
 
 /*
  * Gated delta rule over packed sequences, token by token in fp64.
- *   q,k [T_tot,H,dk], v [T_tot,H,dv] (dtype), g,beta [T_tot,H] (gate_dtype),
+ *   q,k [T_tot,Hk,dk], v [T_tot,H,dv] (dtype), g,beta [T_tot,H] (gate_dtype),
  *   cu_seqlens [N+1], h0 [N,H,dk,dv] (h0_dtype) or NULL for zeros,
  *   hT [N,H,dk,dv] double or NULL, o [T_tot,H,dv] double or NULL.
- * Returns 0, or -1 on a bad argument.
+ * Value head h reads q and k of head h / (H / Hk) (grouped value heads: the
+ * config's linear_num_value_heads may exceed linear_num_key_heads; H == Hk is
+ * the plain layer). Returns 0, or -1 on a bad argument.
  */
 int gdn_oracle_recurrence_mut(const void *q, const void *k, const void *v, int dtype,
                               const void *g, const void *beta, int gate_dtype,
-                              const int64_t *cu_seqlens, int N, int H, int dk, int dv,
+                              const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
                               double scale, int qk_l2norm, double eps,
                               const void *h0, int h0_dtype, double *hT, double *o,
                               int n_threads, int mutation) {
-    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
-    rec_ctx c = {q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, dk, dv, scale,
+    if (N < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
+    rec_ctx c = {q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, Hk, dk, dv, scale,
                  qk_l2norm, eps, h0, h0_dtype, hT, o, mutation};
     run_items(rec_item, &c, (int64_t)N * H, n_threads);
     return 0;
@@ -221,11 +224,12 @@ int gdn_oracle_recurrence_mut(const void *q, const void *k, const void *v, int d
 
 int gdn_oracle_recurrence(const void *q, const void *k, const void *v, int dtype,
                           const void *g, const void *beta, int gate_dtype,
-                          const int64_t *cu_seqlens, int N, int H, int dk, int dv,
+                          const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
                           double scale, int qk_l2norm, double eps,
                           const void *h0, int h0_dtype, double *hT, double *o, int n_threads) {
-    return gdn_oracle_recurrence_mut(q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, N, H, dk,
-                                     dv, scale, qk_l2norm, eps, h0, h0_dtype, hT, o, n_threads, 0);
+    return gdn_oracle_recurrence_mut(q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, N, H, Hk,
+                                     dk, dv, scale, qk_l2norm, eps, h0, h0_dtype, hT, o,
+                                     n_threads, 0);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -321,9 +325,10 @@ typedef struct {
 static void chunk_item(void *vctx, int64_t item) {
     const chunk_ctx *cc = (const chunk_ctx *)vctx;
     const rec_ctx *c = &cc->r;
-    const int H = c->H, dk = c->dk, dv = c->dv, Cs = cc->chunk;
+    const int H = c->H, Hk = c->Hk, dk = c->dk, dv = c->dv, Cs = cc->chunk;
     const int64_t n = item / H;
     const int h = (int)(item % H);
+    const int hk = h / (H / Hk);
     double *S = (double *)calloc((size_t)dk * dv, sizeof(double));
     double *Q = (double *)malloc(sizeof(double) * Cs * dk);
     double *Kc = (double *)malloc(sizeof(double) * Cs * dk);
@@ -345,8 +350,8 @@ static void chunk_item(void *vctx, int64_t item) {
         for (int r = 0; r < L; ++r) {
             const int64_t t = t0 + r;
             for (int i = 0; i < dk; ++i) {
-                Q[r * dk + i] = load_elem(c->q, c->dtype, (t * H + h) * (int64_t)dk + i);
-                Kc[r * dk + i] = load_elem(c->k, c->dtype, (t * H + h) * (int64_t)dk + i);
+                Q[r * dk + i] = load_elem(c->q, c->dtype, (t * Hk + hk) * (int64_t)dk + i);
+                Kc[r * dk + i] = load_elem(c->k, c->dtype, (t * Hk + hk) * (int64_t)dk + i);
             }
             if (c->qk_l2norm) {
                 l2_normalise(Q + r * dk, dk, c->eps);
@@ -421,12 +426,13 @@ static void chunk_item(void *vctx, int64_t item) {
 
 int gdn_oracle_chunked(const void *q, const void *k, const void *v, int dtype,
                        const void *g, const void *beta, int gate_dtype,
-                       const int64_t *cu_seqlens, int N, int H, int dk, int dv,
+                       const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
                        double scale, int qk_l2norm, double eps,
                        const void *h0, int h0_dtype, double *hT, double *o,
                        int chunk, int n_threads) {
-    if (N < 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0 || !cu_seqlens) return -1;
-    chunk_ctx c = {{q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, dk, dv, scale, qk_l2norm,
+    if (N < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || dk <= 0 || dv <= 0 || chunk <= 0 || !cu_seqlens)
+        return -1;
+    chunk_ctx c = {{q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, Hk, dk, dv, scale, qk_l2norm,
                     eps, h0, h0_dtype, hT, o, 0},
                    chunk};
     run_items(chunk_item, &c, (int64_t)N * H, n_threads);

@@ -410,13 +410,15 @@ def test_gated_rmsnorm_gate_is_silu():
     assert np.abs(ratio * np.sqrt(np.mean(y ** 2, axis=-1, keepdims=True)) - y).max() < 1e-12
 
 
-def test_decode_layer_steps_equal_packed_layer():
+@pytest.mark.parametrize("Hk", [2, 1])
+def test_decode_layer_steps_equal_packed_layer(Hk):
     # Token-by-token decode of the whole mixer (conv state and recurrent state
     # carried across calls) equals the packed path: conv over the sequence, then
     # the recurrence over it -- so the conv-state shift and hand-off are right.
+    # Hk = 1 shares one q, k head between both value heads.
     r = _rng(23)
     H, dk, dv, K, T = 2, 4, 3, 4, 7
-    C = 2 * H * dk + H * dv
+    C = 2 * Hk * dk + H * dv
     x = r.normal(size=(T, C))
     cw = r.normal(size=(C, K))
     cs0 = r.normal(size=(1, C, K - 1))
@@ -424,15 +426,15 @@ def test_decode_layer_steps_equal_packed_layer():
     g = -np.abs(r.normal(size=(T, H))) * 0.3
     b = 1.0 / (1.0 + np.exp(-r.normal(size=(T, H))))
     y, cs_ref = oracle.conv_silu(x, cw, [0, T], dtype="f64", state_in=cs0, qk_l2norm=True,
-                                 n_qk=2 * H * dk, head_dim=dk, eps=1e-6)
-    o_ref, h_ref = oracle.recurrence(y[:, :H * dk].reshape(T, H, dk),
-                                     y[:, H * dk:2 * H * dk].reshape(T, H, dk),
-                                     y[:, 2 * H * dk:].reshape(T, H, dv), g, b, [0, T],
+                                 n_qk=2 * Hk * dk, head_dim=dk, eps=1e-6)
+    o_ref, h_ref = oracle.recurrence(y[:, :Hk * dk].reshape(T, Hk, dk),
+                                     y[:, Hk * dk:2 * Hk * dk].reshape(T, Hk, dk),
+                                     y[:, 2 * Hk * dk:].reshape(T, H, dv), g, b, [0, T],
                                      dtype="f64", h0=h0, qk_l2norm=False)
     cs, st = cs0, h0
     for t in range(T):
         o, cs, st = oracle.decode_layer_step(x[t:t + 1], cw, cs, g[t:t + 1], b[t:t + 1], st,
-                                             dtype="f64", H=H, dk=dk, dv=dv)
+                                             dtype="f64", H=H, dk=dk, dv=dv, Hk=Hk)
         assert np.abs(o[0] - o_ref[t]).max() < 1e-12
     assert np.abs(cs - cs_ref).max() < 1e-15 and np.abs(st - h_ref).max() < 1e-12
     # the final conv state is the last K-1 inputs, oldest first
@@ -461,6 +463,45 @@ def test_decode_layer_step_gate_and_input_encoding():
     o_u, _, _ = oracle.decode_layer_step(dec(x), dec(cw), dec(cs0), g, b, st, dtype="f64", H=H,
                                          dk=dk, dv=dv)
     assert np.array_equal(o_f, oracle.gated_rmsnorm(o_u, dec(z), nw, dtype="f64"))
+
+
+# --------------------------------------------------------------------------
+# Grouped value heads: the config's linear_num_value_heads may exceed
+# linear_num_key_heads; each q, k head then serves G consecutive value heads.
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fn", ["recurrence", "chunked"])
+def test_grouped_value_heads_equal_repeated_keys(fn):
+    # Hk key heads shared by G = H / Hk value heads: the result equals the plain
+    # (pinned) rule with every q, k head repeated G times in place
+    r = _rng(26)
+    lens = [37, 0, 70]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, Hk, G, dk, dv = int(cu[-1]), 2, 3, 8, 5
+    H = Hk * G
+    q, k = r.normal(size=(T, Hk, dk)), r.normal(size=(T, Hk, dk))
+    v = r.normal(size=(T, H, dv))
+    g = -0.3 * np.abs(r.normal(size=(T, H))); beta = r.uniform(size=(T, H))
+    h0 = r.normal(size=(len(lens), H, dk, dv))
+    kw = dict(dtype="f64", h0=h0, scale=0.7, threads=2)
+    if fn == "chunked":
+        kw["chunk"] = 16
+    f = getattr(oracle, fn)
+    o, hT = f(q, k, v, g, beta, cu, **kw)
+    o_r, h_r = f(np.repeat(q, G, axis=1), np.repeat(k, G, axis=1), v, g, beta, cu, **kw)
+    assert np.array_equal(o, o_r) and np.array_equal(hT, h_r)
+    # the other conceivable sharing (value head h reading key head h mod Hk)
+    # gives a different result, so the check above tells the two apart
+    o_t, _ = f(np.tile(q, (1, G, 1)), np.tile(k, (1, G, 1)), v, g, beta, cu, **kw)
+    assert np.abs(o_t - o).max() > 1e-3
+
+
+def test_grouped_value_heads_reject_uneven_groups():
+    r = _rng(27)
+    q, k, v = r.normal(size=(4, 2, 3)), r.normal(size=(4, 2, 3)), r.normal(size=(4, 3, 3))
+    g, b = np.zeros((4, 3)), np.zeros((4, 3))
+    with pytest.raises(ValueError):
+        oracle.recurrence(q, k, v, g, b, [0, 4], dtype="f64", threads=1)
 
 
 # --------------------------------------------------------------------------
