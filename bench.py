@@ -508,6 +508,93 @@ def bench_decode_layer(args, dist, pk):
             "gpu_launches": steps}
 
 
+def bench_grouped(args, dist, pk):
+    """Grouped value heads: 32 value heads on 16 q, k heads, d=128. The prefill
+    of 8 sequences x 8192 tokens (fp32 final state), and the whole-mixer decode
+    step for 256 sequences (one two-CTA cluster per q, k head), 100 steps."""
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    P = gi.grouped_prefill()
+    Hv, Hk, N, T = P.H, P.Hk, P.N, P.T_tot
+    bf = lambda a: torch.from_numpy(a.view("int16")).to(dev).view(torch.bfloat16)
+    q, k, v = bf(P.q), bf(P.k), bf(P.v)
+    g, beta = torch.from_numpy(P.g).to(dev), torch.from_numpy(P.beta).to(dev)
+    cu = torch.from_numpy(P.cu_seqlens).to(dev)
+    del P
+    o = torch.empty((T, Hv, D), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((N, Hv, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(N, T, Hv, D, D, CHUNK), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, chunk=CHUNK)
+
+    for _ in range(3):
+        step()
+    gdn.check_device_status(dev)
+    torch.cuda.synchronize()
+    reps = 5
+    total_ms, _ = timed(step, reps, stream)
+    ms = dist.max(total_ms) / reps
+    flops = T * Hv * FLOP_PER_TOKEN_HEAD
+    # q, k once per q, k head; v, o, gates per value head; the final state
+    byts = T * (2 * Hk * D * 2 + Hv * (2 * D * 2 + 8)) + N * Hv * STATE_BYTES
+    pre = {"value": T / (ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": ms,
+           "workload": f"grouped_prefill_{N}x{T // N}_hv{Hv}_hk{Hk}_d128_bf16",
+           "tc_roofline": {"achieved": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                           "peak": pk["bf16_tflops"],
+                           "frac": flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops"]},
+           "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                        "algorithmic_bytes": byts},
+           "gpu_launches": 2 * reps}
+    del q, k, v, g, beta, o, hT
+    torch.cuda.empty_cache()
+
+    Nd, steps, K = 256, 100, 4
+    C = 2 * Hk * D + Hv * D
+    r = np.random.default_rng(8)
+    bfr = lambda a: torch.from_numpy(gi.to_bf16_bits(a.astype(np.float32)).view("int16")).to(dev) \
+        .view(torch.bfloat16)
+    state = torch.from_numpy(gi.decode_state(Nd, Hv, D)).to(dev)
+    conv_state = bfr(r.normal(size=(Nd, C, K - 1)))
+    conv_w = bfr(r.normal(size=(C, K)) * 0.5)
+    norm_w = torch.ones(D, dtype=torch.float32, device=dev)
+    ins = []
+    for _ in range(8):
+        ins.append((bfr(r.normal(size=(Nd, C))), torch.from_numpy(
+            (-np.log1p(np.exp(r.normal(size=(Nd, Hv))))).astype(np.float32)).to(dev),
+            torch.from_numpy((1 / (1 + np.exp(-r.normal(size=(Nd, Hv))))).astype(np.float32)).to(dev),
+            bfr(r.normal(size=(Nd, Hv, D)))))
+    od = torch.empty((Nd, Hv, D), dtype=torch.bfloat16, device=dev)
+    it = iter(range(10 ** 9))
+
+    def dstep():
+        x, gg, bb, z = ins[next(it) % len(ins)]
+        gdn.decode_layer_step(x, conv_w, conv_state, gg, bb, state, H=Hv, Hk=Hk, dk=D, dv=D, z=z,
+                              norm_w=norm_w, out=od)
+
+    for _ in range(5):
+        dstep()
+    gdn.check_device_status(dev)
+    torch.cuda.synchronize()
+    total_ms, _ = timed(dstep, steps, stream)
+    step_ms = dist.max(total_ms) / steps
+    bytes_step = (2 * Nd * Hv * STATE_BYTES + Nd * C * 2 + 2 * Nd * C * (K - 1) * 2
+                  + 2 * Nd * Hv * D * 2 + Nd * Hv * 8 + C * K * 2)
+    dec = {"value": Nd / (step_ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": step_ms,
+           "workload": f"decode_layer_{Nd}_hv{Hv}_hk{Hk}_d128_conv4_gated_{steps}steps",
+           "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
+                        "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                        "algorithmic_bytes": bytes_step},
+           "gpu_launches": steps}
+    return {"prefill": pre, "decode_layer": dec}
+
+
 def bench_gated_norm(args, dist, pk):
     """Gated RMSNorm output over the long-prefill output: 8 x 16384 tokens x 16
     heads, d_v = 128, bf16 (read o and z, write the gated output)."""
@@ -618,6 +705,7 @@ def run_ours(args, dist: Dist):
         extras["varlen"] = bench_varlen(args, dist, pk)
         extras["decode_layer"] = bench_decode_layer(args, dist, pk)
         extras["gated_rmsnorm"] = bench_gated_norm(args, dist, pk)
+        extras["grouped"] = bench_grouped(args, dist, pk)
     clocks.active = False
     clk = clocks.stop()
 
@@ -698,7 +786,8 @@ def main():
 
 
 ONLY = {"decode": bench_decode, "layer": bench_layer, "varlen": bench_varlen,
-        "decode_layer": bench_decode_layer, "gated_rmsnorm": bench_gated_norm}
+        "decode_layer": bench_decode_layer, "gated_rmsnorm": bench_gated_norm,
+        "grouped": bench_grouped}
 
 if __name__ == "__main__":
     main()

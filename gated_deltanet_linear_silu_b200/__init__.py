@@ -56,13 +56,13 @@ def lib() -> ctypes.CDLL:
         L.gdn_conv_silu.restype = i32
         L.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
         L.gdn_prefill_workspace_size.restype = sz
-        L.gdn_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+        L.gdn_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
                                   i64, i64, i64, f32, i32, f32, i32, vp, vp, vp, vp, sz, i32, vp]
         L.gdn_prefill.restype = i32
-        L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, f32, i32, f32,
-                                      vp, vp]
+        L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
+                                      f32, vp, vp]
         L.gdn_decode_layer_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, f32, i32, i32,
-                                            i32, i32, f32, i32, f32, vp, vp]
+                                            i32, i32, i32, f32, i32, f32, vp, vp]
         L.gdn_decode_layer_step.restype = i32
         L.gdn_gated_rmsnorm.argtypes = [vp, vp, vp, i32, i64, i32, f32, vp, vp]
         L.gdn_gated_rmsnorm.restype = i32
@@ -72,7 +72,7 @@ def lib() -> ctypes.CDLL:
         L.gdn_check_device_status.argtypes = [vp]
         L.gdn_check_device_status.restype = i32
         L.gdn_prefill_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32,
-                                          i64, i64, i64, f32, i32, f32, i32, vp, vp, vp, i32, vp]
+                                          i32, i64, i64, i64, f32, i32, f32, i32, vp, vp, vp, i32, vp]
         L.gdn_prefill_noalloc.restype = i32
         L.gdn_prefill_noalloc_max_scratch.argtypes = []
         L.gdn_prefill_noalloc_max_scratch.restype = sz
@@ -158,12 +158,13 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
             cu_seqlens_host: Optional[torch.Tensor] = None, algo: str = "auto",
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None
             ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Chunked gated delta rule. q,k [T,H,dk], v [T,H,dv] (bf16 or fp32; each
-    may be a token-strided view, e.g. a slice of the fused conv output),
-    g,beta [T,H] fp32, cu_seqlens int32 [N+1] (device). Returns (o, hT);
-    final_state may be initial_state itself for an in-place update."""
-    T, H, dk = q.shape
-    dv = v.shape[2]
+    """Chunked gated delta rule. q,k [T,Hk,dk], v [T,H,dv] (bf16 or fp32; each
+    may be a token-strided view, e.g. a slice of the fused conv output; Hk < H
+    groups H / Hk value heads on each q, k head), g,beta [T,H] fp32, cu_seqlens
+    int32 [N+1] (device). Returns (o, hT); final_state may be initial_state
+    itself for an in-place update."""
+    T, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     N = cu_seqlens.shape[0] - 1
     o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device) if out is None else out
     hT = final_state
@@ -179,7 +180,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
         host_cu = cu_seqlens_host.to(torch.int32).contiguous()
     st = lib().gdn_prefill(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
-        None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, dk, dv,
+        None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
         ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(chunk), _ptr(initial_state), _ptr(hT),
         _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill")
@@ -194,14 +195,14 @@ def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
     """gdn_prefill_noalloc: prefill with the library's fixed scratch array
     instead of a workspace; the caller passes every output buffer, so nothing
     is allocated."""
-    T, H, dk = q.shape
-    dv = v.shape[2]
+    T, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     N = cu_seqlens.shape[0] - 1
     ld = [_token_stride(t) for t in (q, k, v)]
     _cuda(g, beta, cu_seqlens, initial_state, final_state, out)
     st = lib().gdn_prefill_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens), None,
-        N, T, H, dk, dv, ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(chunk),
+        N, T, H, Hk, dk, dv, ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(chunk),
         _ptr(initial_state), _ptr(final_state), _ptr(out), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill_noalloc")
 
@@ -220,14 +221,14 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
                 beta: torch.Tensor, state: torch.Tensor, *, scale: float = 1.0,
                 qk_l2norm: bool = True, eps: float = 1e-6, out: Optional[torch.Tensor] = None
                 ) -> torch.Tensor:
-    """One recurrent token per sequence. q,k [N,H,dk], v [N,H,dv], g,beta
+    """One recurrent token per sequence. q,k [N,Hk,dk], v [N,H,dv], g,beta
     [N,H] fp32, state [N,H,dk,dv] fp32 updated in place. Returns o [N,H,dv]."""
-    N, H, dk = q.shape
-    dv = v.shape[2]
+    N, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
     o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device) if out is None else out
     _cuda(q, k, v, g, beta, state, o)
     st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta),
-                               _ptr(state), N, H, dk, dv, float(scale), int(qk_l2norm), float(eps),
+                               _ptr(state), N, H, Hk, dk, dv, float(scale), int(qk_l2norm), float(eps),
                                _ptr(o), _stream(q.device))
     _check(st, "gdn_decode_step")
     return o
@@ -238,18 +239,22 @@ def decode_layer_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: Optiona
                       dv: int, z: Optional[torch.Tensor] = None,
                       norm_w: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
                       scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6,
-                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                      out: Optional[torch.Tensor] = None, Hk: Optional[int] = None) -> torch.Tensor:
     """One decode token of the whole mixer per sequence. x [N, C] fused
-    [q | k | v] projections (C = 2 H dk + H dv), conv_w [C, K], conv_state
-    [N, C, K-1] and state [N, H, dk, dv] fp32 updated in place, g/beta [N, H]
-    fp32, optional gate z [N, H, dv] with norm_w [dv] fp32. Returns o [N, H, dv]."""
+    [q | k | v] projections (C = 2 Hk dk + H dv; Hk q, k heads, default H),
+    conv_w [C, K], conv_state [N, C, K-1] and state [N, H, dk, dv] fp32 updated
+    in place, g/beta [N, H] fp32, optional gate z [N, H, dv] with norm_w [dv]
+    fp32. Returns o [N, H, dv]."""
+    Hk = H if Hk is None else Hk
     N, C = x.shape
     K = conv_w.shape[1]
+    if Hk <= 0 or C != 2 * Hk * dk + H * dv:
+        raise ValueError(f"x has {C} channels; expected 2*Hk*dk + H*dv")
     o = torch.empty((N, H, dv), dtype=x.dtype, device=x.device) if out is None else out
     _cuda(x, conv_w, conv_state, g, beta, state, z, norm_w, o)
     st = lib().gdn_decode_layer_step(_ptr(x), _ptr(conv_w), _ptr(conv_state), K, _dtype_code(x),
                                      _ptr(g), _ptr(beta), _ptr(state), _ptr(z), _ptr(norm_w),
-                                     float(norm_eps), N, H, dk, dv, float(scale), int(qk_l2norm),
+                                     float(norm_eps), N, H, Hk, dk, dv, float(scale), int(qk_l2norm),
                                      float(eps), _ptr(o), _stream(x.device))
     _check(st, "gdn_decode_layer_step")
     return o

@@ -115,11 +115,13 @@ size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, i
 
 gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                          const float* g, const float* beta, const int32_t* cu_seqlens,
-                         const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int dk,
-                         int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale, int qk_l2norm, float eps, int chunk, const float* h0,
-                         float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
-                         void* stream) {
-    if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+                         const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
+                         int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale,
+                         int qk_l2norm, float eps, int chunk, const float* h0, float* hT, void* o,
+                         void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream) {
+    if (Hk == 0) Hk = H;
+    if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0 || Hk < 0 || H % Hk != 0)
+        return GDN_ERR_INVALID_ARG;
     if (N == 0 && T_tot > 0) return GDN_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (!(chunk == 16 || chunk == 32 || chunk == 64)) return GDN_ERR_UNSUPPORTED;
@@ -132,10 +134,10 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
         return GDN_ERR_INVALID_ARG;
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     const int64_t esz = dtype == GDN_BF16 ? 2 : 4;
-    if (ld_q == 0) ld_q = (int64_t)H * dk;
-    if (ld_k == 0) ld_k = (int64_t)H * dk;
+    if (ld_q == 0) ld_q = (int64_t)Hk * dk;
+    if (ld_k == 0) ld_k = (int64_t)Hk * dk;
     if (ld_v == 0) ld_v = (int64_t)H * dv;
-    if (ld_q < (int64_t)H * dk || ld_k < (int64_t)H * dk || ld_v < (int64_t)H * dv ||
+    if (ld_q < (int64_t)Hk * dk || ld_k < (int64_t)Hk * dk || ld_v < (int64_t)H * dv ||
         (ld_q * esz) % 16 != 0 || (ld_k * esz) % 16 != 0 || (ld_v * esz) % 16 != 0)
         return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H * 2 >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
@@ -146,7 +148,7 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
     if (!workspace || ws_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return GDN_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
-    gdn::PrefillArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, dk, dv,
+    gdn::PrefillArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, Hk, dk, dv,
                        ld_q, ld_k, ld_v, scale, qk_l2norm, eps, chunk, h0, hT, o,
                        reinterpret_cast<int32_t*>(ws + wl.order_off),
                        reinterpret_cast<int32_t*>(ws + wl.counter_off), status_ptr()};
@@ -179,9 +181,11 @@ int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_
 }
 
 gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
-                             const float* g, const float* beta, float* state, int N, int H, int dk,
-                             int dv, float scale, int qk_l2norm, float eps, void* o, void* stream) {
-    if (!dtype_ok(dtype) || N < 0 || H <= 0) return GDN_ERR_INVALID_ARG;
+                             const float* g, const float* beta, float* state, int N, int H, int Hk,
+                             int dk, int dv, float scale, int qk_l2norm, float eps, void* o,
+                             void* stream) {
+    if (Hk == 0) Hk = H;
+    if (!dtype_ok(dtype) || N < 0 || H <= 0 || Hk < 0 || H % Hk != 0) return GDN_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (N == 0) return GDN_OK;
     if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
@@ -189,7 +193,7 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dt
         return GDN_ERR_INVALID_ARG;
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
-    gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, dk, dv, scale, qk_l2norm, eps, o,
+    gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, Hk, dk, dv, scale, qk_l2norm, eps, o,
                       nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0.f};
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
 }
@@ -197,10 +201,12 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dt
 gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv_state, int K,
                                    gdn_dtype_t dtype, const float* g, const float* beta, float* state,
                                    const void* z, const float* norm_w, float norm_eps, int N, int H,
-                                   int dk, int dv, float scale, int qk_l2norm, float eps, void* o,
-                                   void* stream) {
-    if (!dtype_ok(dtype) || N < 0 || H <= 0 || K < 1) return GDN_ERR_INVALID_ARG;
-    if (K > 4) return GDN_ERR_UNSUPPORTED;
+                                   int Hk, int dk, int dv, float scale, int qk_l2norm, float eps,
+                                   void* o, void* stream) {
+    if (Hk == 0) Hk = H;
+    if (!dtype_ok(dtype) || N < 0 || H <= 0 || K < 1 || Hk < 0 || H % Hk != 0)
+        return GDN_ERR_INVALID_ARG;
+    if (K > 4 || H / Hk > gdn::kMaxDecodeGroup) return GDN_ERR_UNSUPPORTED;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (N == 0) return GDN_OK;
     if (!x || !conv_w || !g || !beta || !state || !o || (K > 1 && !conv_state))
@@ -212,7 +218,7 @@ gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if (z && !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
-    gdn::DecodeArgs a{nullptr, nullptr, nullptr, dtype == GDN_BF16, g, beta, state, N, H, dk, dv,
+    gdn::DecodeArgs a{nullptr, nullptr, nullptr, dtype == GDN_BF16, g, beta, state, N, H, Hk, dk, dv,
                       scale, qk_l2norm, eps, o, x, conv_w, conv_state, K, z, norm_w, norm_eps};
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
 }

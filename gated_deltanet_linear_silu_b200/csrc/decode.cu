@@ -16,6 +16,14 @@
 // applies SiLU before the recurrent step -- q, k, v never leave the SM. With a
 // gate z the output goes through the gated RMSNorm of 7.6.2 (RMSNorm as in
 // 7.6.3, scale vector as given) on the way out.
+//
+// Grouped value heads (H = G * Hk, the config's linear_num_value_heads over
+// linear_num_key_heads, 7.6.1): value head h reads q, k head h / G. In the
+// whole-mixer step the G CTAs of one group all need the group's q, k conv
+// channels; they run as one thread-block cluster, every CTA computes those
+// channels' conv from the old conv state, and after a cluster barrier (every
+// CTA has read the old state) only the group's first CTA writes the shifted
+// q, k conv state back.
 #include "common.cuh"
 #include "launch.h"
 
@@ -23,6 +31,14 @@ namespace gdn {
 namespace {
 
 __device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// Cluster-wide barrier in two halves (hardware barrier; no spinning in code).
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 template <typename T, int RPT, bool CONV>
 __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
@@ -34,6 +50,8 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
     const int cg = tid % cols4;
     const int rg = tid / cols4;
     const int64_t nh = blockIdx.x;  // n * H + h
+    const int H = a.H, Hk = a.Hk, G = H / Hk;
+    const int n = (int)(nh / H), h = (int)(nh % H), hk = h / G;
 
     float* qs = sm;              // [dk]
     float* ks = qs + dk;         // [dk]
@@ -45,15 +63,14 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
     // the taps and the conv state, a few KB -- are copied to shared memory
     // asynchronously ahead of the state's 64 KB, so they are in when needed and
     // hold no registers meanwhile. Three contiguous channel blocks: q (dk channels
-    // from h*dk), k (dk from H*dk + h*dk), v (dv from 2*H*dk + h*dv).
+    // from hk*dk), k (dk from Hk*dk + hk*dk), v (dv from 2*Hk*dk + h*dv).
     const int nconv = 2 * dk + dv;
     T* cx_s = reinterpret_cast<T*>(vs + dv);          // [nconv]
     T* cw_s = cx_s + nconv;                           // [nconv][K]
     T* cs_s = cw_s + nconv * a.K;                     // [nconv][K-1]
     if constexpr (CONV) {
-        const int H = a.H, K = a.K;
-        const int n = (int)(nh / H), h = (int)(nh % H);
-        const int64_t C = 2 * H * dk + H * dv;
+        const int K = a.K;
+        const int64_t C = 2 * Hk * dk + H * dv;
         const T* x = static_cast<const T*>(a.x) + n * C;
         const T* w = static_cast<const T*>(a.conv_w);
         const T* cs = static_cast<const T*>(a.conv_state) + n * C * (K - 1);
@@ -61,7 +78,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
 #pragma unroll
         for (int b = 0; b < 3; ++b) {
             const int nb = b < 2 ? dk : dv;                       // channels in the block
-            const int64_t ch0 = b == 0 ? h * dk : (b == 1 ? H * dk + h * dk : 2 * H * dk + h * dv);
+            const int64_t ch0 = b == 0 ? hk * dk : (b == 1 ? Hk * dk + hk * dk : 2 * Hk * dk + h * dv);
             const int c0 = b == 0 ? 0 : (b == 1 ? dk : 2 * dk);  // first local channel
             for (int p = tid; p < nb / E; p += blockDim.x) cp_async_16(cx_s + c0 + p * E, x + ch0 + p * E);
             for (int p = tid; p < nb * K / E; p += blockDim.x)
@@ -84,12 +101,12 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
         // causal conv of this head's q, k, v channels against the conv state
         // (window: the K-1 stored inputs, oldest first, then x); the state shifts
         // by one and takes x as its newest entry
-        const int H = a.H, K = a.K;
-        const int n = (int)(nh / H), h = (int)(nh % H);
-        const int64_t C = 2 * H * dk + H * dv;
+        const int K = a.K;
+        const int64_t C = 2 * Hk * dk + H * dv;
         T* cs = static_cast<T*>(a.conv_state) + n * C * (K - 1);
         cp_async_wait_all_groups();
         __syncthreads();
+        if (G > 1) cluster_arrive_release();  // this CTA's copy of the old conv state is in
         for (int c = tid; c < nconv; c += blockDim.x) {
             const float xt = Elem<T>::load(cx_s, c);
             float acc;
@@ -122,13 +139,16 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
             else vs[c - 2 * dk] = y;
         }
         __syncthreads();
-        // the shifted conv state back to global memory, 16 bytes per store
+        if (G > 1) cluster_wait_acquire();  // every CTA of the group has read the old state
+        // the shifted conv state back to global memory, 16 bytes per store (the
+        // shared q, k channels by the group's first CTA only)
         if (K > 1) {
             constexpr int E = 16 / (int)sizeof(T);
 #pragma unroll
             for (int b = 0; b < 3; ++b) {
+                if (b < 2 && h % G != 0) continue;
                 const int nb = b < 2 ? dk : dv;
-                const int64_t ch0 = b == 0 ? h * dk : (b == 1 ? H * dk + h * dk : 2 * H * dk + h * dv);
+                const int64_t ch0 = b == 0 ? hk * dk : (b == 1 ? Hk * dk + hk * dk : 2 * Hk * dk + h * dv);
                 const int c0 = b == 0 ? 0 : (b == 1 ? dk : 2 * dk);
                 for (int p = tid; p < nb * (K - 1) / E; p += blockDim.x)
                     *reinterpret_cast<uint4*>(cs + ch0 * (K - 1) + p * E) =
@@ -138,8 +158,8 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
         __syncthreads();
         v4 = *reinterpret_cast<const float4*>(vs + 4 * cg);
     } else {
-        const T* qg = static_cast<const T*>(a.q) + nh * dk;
-        const T* kg = static_cast<const T*>(a.k) + nh * dk;
+        const T* qg = static_cast<const T*>(a.q) + ((int64_t)n * Hk + hk) * dk;
+        const T* kg = static_cast<const T*>(a.k) + ((int64_t)n * Hk + hk) * dk;
         for (int i = tid; i < dk; i += blockDim.x) {
             qs[i] = Elem<T>::load(qg, i);
             ks[i] = Elem<T>::load(kg, i);
@@ -247,6 +267,22 @@ cudaError_t launch_rpt(const DecodeArgs& a, cudaStream_t s) {
     if (a.x)  // conv inputs: x, taps, conv state of the head's channels
         smem += (size_t)(2 * a.dk + a.dv) * (2 * a.K) * (a.is_bf16 ? 2 : 4);
     const int64_t blocks = (int64_t)a.N * a.H;
+    const int G = a.H / a.Hk;
+    if (a.x && G > 1) {  // one cluster per group of value heads sharing a q, k head
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)blocks);
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = G;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, decode_step_kernel<T, RPT, true>, a);
+    }
     if (a.x)
         decode_step_kernel<T, RPT, true><<<(unsigned)blocks, threads, smem, s>>>(a);
     else

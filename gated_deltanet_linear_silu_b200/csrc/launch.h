@@ -33,13 +33,13 @@ struct DecodeArgs {
     const float* g;
     const float* beta;
     float* state;
-    int N, H, dk, dv;
+    int N, H, Hk, dk, dv;  // H value heads; q, k have Hk heads, head h reads h / (H / Hk)
     float scale;
     int qk_l2norm;
     float eps;
     void* o;
     // whole-mixer step (x != nullptr): q, k, v come from the conv update of x
-    const void* x;        // [N, C] fused projections, C = 2*H*dk + H*dv
+    const void* x;        // [N, C] fused projections, C = 2*Hk*dk + H*dv
     const void* conv_w;   // [C, K]
     void* conv_state;     // [N, C, K-1], updated in place
     int K;
@@ -49,6 +49,9 @@ struct DecodeArgs {
     float norm_eps;
 };
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
+// Largest value-head group (H / Hk) of the whole-mixer decode step: one
+// thread-block cluster per group, 8 being the portable cluster size.
+constexpr int kMaxDecodeGroup = 8;
 
 struct GatedNormArgs {
     const void* y;
@@ -72,7 +75,7 @@ struct PrefillArgs {
     const int32_t* cu;
     int N;
     int64_t T_tot;
-    int H, dk, dv;
+    int H, Hk, dk, dv;         // H value heads; q, k have Hk heads, head h reads h / (H / Hk)
     int64_t ld_q, ld_k, ld_v;  // elements between consecutive tokens of q, k, v
     float scale;
     int qk_l2norm;

@@ -55,7 +55,7 @@ size_t gdn_prefill_noalloc_max_scratch(void) { return kNoallocScratchBytes; }
 gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                                  const float* g, const float* beta, const int32_t* cu_seqlens,
                                  const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H,
-                                 int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v,
+                                 int Hk, int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v,
                                  float scale, int qk_l2norm, float eps, int chunk,
                                  const float* h0, float* hT, void* o, gdn_algo_t algo,
                                  void* stream) {
@@ -67,7 +67,7 @@ gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v, gd
         scratch = scratch_on_current_device();
         if (!scratch) return GDN_ERR_CUDA;
     }
-    return gdn_prefill(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, dk, dv,
+    return gdn_prefill(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv,
                        ld_q, ld_k, ld_v, scale, qk_l2norm, eps, chunk, h0, hT, o, scratch, kNoallocScratchBytes,
                        algo, stream);
 }

@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
         if (unit >= total_units) break;
         const int vt = (int)(unit % n_vt);
         const int h = (int)((unit / n_vt) % H);
+        const int hk = h / (H / a.Hk);  // the q, k head this value head reads
         const int n = a.order[unit / ((int64_t)n_vt * H)];
         const int64_t start = a.cu[n], end = a.cu[n + 1];
         if (!(n >= 0 && n < a.N && start >= 0 && start <= end && end <= a.T_tot)) {
@@ -146,8 +147,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
                 const int r = e / dk, i = e % dk;
                 float qv = 0.f, kv = 0.f;
                 if (r < L) {
-                    qv = Elem<T>::load(q, (c0 + r) * a.ld_q + h * dk + i);
-                    kv = Elem<T>::load(k, (c0 + r) * a.ld_k + h * dk + i);
+                    qv = Elem<T>::load(q, (c0 + r) * a.ld_q + hk * dk + i);
+                    kv = Elem<T>::load(k, (c0 + r) * a.ld_k + hk * dk + i);
                 }
                 Qs[r * ldk + i] = qv;
                 Ks[r * ldk + i] = kv;

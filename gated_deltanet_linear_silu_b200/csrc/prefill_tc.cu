@@ -213,14 +213,14 @@ __device__ __forceinline__ int64_t next_nonempty(const PrefillArgs& a, int64_t u
 }
 
 __device__ __forceinline__ void issue_tiles(uint8_t* stage, uint64_t* bar, const CUtensorMap* mq,
-                                            const CUtensorMap* mk, const CUtensorMap* mv, int h,
-                                            int64_t c0) {
+                                            const CUtensorMap* mk, const CUtensorMap* mv, int hk,
+                                            int h, int64_t c0) {
     mbar_arrive_expect_tx(bar, kStageBytes);
     const int t = (int)c0;
-    tma_load_3d(stage + kQb0, mq, bar, 0, h, t);
-    tma_load_3d(stage + kQb1, mq, bar, 64, h, t);
-    tma_load_3d(stage + kKb0, mk, bar, 0, h, t);
-    tma_load_3d(stage + kKb1, mk, bar, 64, h, t);
+    tma_load_3d(stage + kQb0, mq, bar, 0, hk, t);
+    tma_load_3d(stage + kQb1, mq, bar, 64, hk, t);
+    tma_load_3d(stage + kKb0, mk, bar, 0, hk, t);
+    tma_load_3d(stage + kKb1, mk, bar, 64, hk, t);
     tma_load_3d(stage + kVb0, mv, bar, 0, h, t);
     tma_load_3d(stage + kVb1, mv, bar, 64, h, t);
 }
@@ -311,6 +311,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     const PrefillArgs& a = P.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
+    const int group = H / a.Hk;  // value heads per q, k head
     const int64_t total = (int64_t)a.N * H;
 
     uint8_t* sWT = sm + kOffWT;
@@ -693,7 +694,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         uint32_t issued = 0, issued_par = 0;  // for the bounded drain at exit
         auto fill = [&](const Item& f, int s, int use) {
             if (stid != kRefill) return;
-            issue_tiles(S.stage(s), &full[s], &map_q, &map_k, &map_v, f.U.h, f.c0);
+            issue_tiles(S.stage(s), &full[s], &map_q, &map_k, &map_v, f.U.h / group, f.U.h, f.c0);
             issued |= 1u << s;
             issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(use & 1) << s);
         };
@@ -985,7 +986,7 @@ bool prefill_tc_supported(const PrefillArgs& a) {
 
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     CUtensorMap mq, mk, mv, mo;
-    if (!make_map(&mq, a.q, a.H, a.T_tot, a.ld_q, true) || !make_map(&mk, a.k, a.H, a.T_tot, a.ld_k, true) ||
+    if (!make_map(&mq, a.q, a.Hk, a.T_tot, a.ld_q, true) || !make_map(&mk, a.k, a.Hk, a.T_tot, a.ld_k, true) ||
         !make_map(&mv, a.v, a.H, a.T_tot, a.ld_v, true) ||
         !make_map(&mo, a.o, a.H, a.T_tot, (int64_t)a.H * kD, false))
         return cudaErrorInvalidValue;

@@ -26,6 +26,9 @@ token mixer (Qwen3.5 linear-attention layer shapes, "7.6 Qwen3.5" config table:
                    g = -softplus(N(0,1)); 100 steps.
 * ``varlen``       64 lengths ~ U[256, 32768] (inclusive), packed; q/k/v/beta/g
                    as ``long_prefill``; initial state ~ N(0, 0.1) fp32.
+* ``grouped``      grouped value heads (the config table lists the value-head
+                   and key-head counts separately): 8 x 8192 tokens, 32 value
+                   heads on 16 q/k heads, d=128, draws as ``long_prefill``.
 
 q and k are drawn raw; the per-head L2 normalisation the workloads call for is
 part of the computed path (both sides apply it), not of the data. The gate
@@ -47,6 +50,7 @@ LAYER_0P8B = 1
 LONG_PREFILL = 2
 DECODE = 3
 VARLEN = 4
+GROUPED = 5
 
 WORKLOAD_NAMES = {
     TINY_FP32: "tiny_fp32",
@@ -54,6 +58,7 @@ WORKLOAD_NAMES = {
     LONG_PREFILL: "long_prefill",
     DECODE: "decode",
     VARLEN: "varlen",
+    GROUPED: "grouped",
 }
 
 # Tensor tags of the seed tree (stable: changing one changes every draw).
@@ -204,10 +209,12 @@ def layer_0p8b(T: int = 4096, emb: int = 1024, H: int = 16, d: int = 128) -> Lay
 
 
 def sequence_tensors(workload: int, n: int, T: int, H: int, d: int,
-                     g_scale: float) -> dict:
-    """q/k/v (bf16 bits), beta, g of sequence n of a packed prefill workload."""
-    q = to_bf16_bits(_normal(rng(workload, "q", n), (T, H, d)))
-    k = to_bf16_bits(_normal(rng(workload, "k", n), (T, H, d)))
+                     g_scale: float, Hk: Optional[int] = None) -> dict:
+    """q/k/v (bf16 bits), beta, g of sequence n of a packed prefill workload
+    (q, k with Hk heads, default H)."""
+    Hk = H if Hk is None else Hk
+    q = to_bf16_bits(_normal(rng(workload, "q", n), (T, Hk, d)))
+    k = to_bf16_bits(_normal(rng(workload, "k", n), (T, Hk, d)))
     v = to_bf16_bits(_normal(rng(workload, "v", n), (T, H, d)))
     beta = _sigmoid(_normal(rng(workload, "beta", n), (T, H)))
     g = (-_softplus(_normal(rng(workload, "g", n), (T, H))) * np.float32(g_scale)).astype(np.float32)
@@ -219,19 +226,20 @@ def varlen_lengths(N: int = 64, lo: int = 256, hi: int = 32768) -> np.ndarray:
 
 
 def _packed(workload: int, name: str, lengths, H: int, d: int, g_scale: float,
-            h0: Optional[np.ndarray]) -> Prefill:
+            h0: Optional[np.ndarray], Hk: Optional[int] = None) -> Prefill:
+    Hk = H if Hk is None else Hk
     lengths = np.asarray(lengths, dtype=np.int64)
     cu = np.zeros(len(lengths) + 1, dtype=np.int64)
     cu[1:] = np.cumsum(lengths)
     T_tot = int(cu[-1])
-    q = np.empty((T_tot, H, d), np.uint16)
+    q = np.empty((T_tot, Hk, d), np.uint16)
     k = np.empty_like(q)
-    v = np.empty_like(q)
+    v = np.empty((T_tot, H, d), np.uint16)
     beta = np.empty((T_tot, H), np.float32)
     g = np.empty_like(beta)
 
     def fill(n):  # numpy releases the GIL while drawing, so sequences fill in parallel
-        s = sequence_tensors(workload, n, int(lengths[n]), H, d, g_scale)
+        s = sequence_tensors(workload, n, int(lengths[n]), H, d, g_scale, Hk)
         a, b = int(cu[n]), int(cu[n + 1])
         q[a:b], k[a:b], v[a:b], beta[a:b], g[a:b] = s["q"], s["k"], s["v"], s["beta"], s["g"]
 
@@ -242,6 +250,10 @@ def _packed(workload: int, name: str, lengths, H: int, d: int, g_scale: float,
 
 def long_prefill(N: int = 8, T: int = 16384, H: int = 16, d: int = 128) -> Prefill:
     return _packed(LONG_PREFILL, "long_prefill", [T] * N, H, d, 0.1, None)
+
+
+def grouped_prefill(N: int = 8, T: int = 8192, H: int = 32, Hk: int = 16, d: int = 128) -> Prefill:
+    return _packed(GROUPED, "grouped", [T] * N, H, d, 0.1, None, Hk)
 
 
 def initial_state(workload: int, n: int, H: int, dk: int, dv: int, std: float = 0.1) -> np.ndarray:

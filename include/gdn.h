@@ -30,6 +30,15 @@
  *       a separate projection of the layer input; 7.6.3: RMSNorm(x) =
  *       x / sqrt(mean(x^2) + eps) times a per-feature scale (stored there as
  *       1 + w, zero-centred).
+ *   [V] same page, 7.6.1 (config table): the value-head and key-head counts of
+ *       the linear-attention layers are separate settings
+ *       (linear_num_value_heads, linear_num_key_heads).
+ *
+ * Heads: H is the number of value heads (v, g, beta, the recurrent state and
+ * the output have H heads); q and k have Hk heads, Hk dividing H, and value
+ * head h reads q, k head h / (H / Hk) -- each q, k head serves H / Hk
+ * consecutive value heads ([V]; the grouping order is this library's reading).
+ * Hk = 0 means Hk = H, the plain layer.
  *
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
@@ -134,7 +143,7 @@ GDN_API size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, i
  * triangular solve, inter-chunk state passing); the result equals the token
  * loop up to rounding.
  *
- *   q, k            [T_tot, H, dk]  dtype
+ *   q, k            [T_tot, Hk, dk] dtype   (Hk = 0: Hk = H; see "Heads" above)
  *   v               [T_tot, H, dv]  dtype
  *   g, beta         [T_tot, H]      fp32    g = log(alpha) <= 0 expected
  *   cu_seqlens      [N+1]           int32   device prefix offsets
@@ -144,7 +153,7 @@ GDN_API size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, i
  *   hT              [N, H, dk, dv]  fp32    nullable final state; may alias h0
  *   o               [T_tot, H, dv]  dtype   output (dense)
  *   ld_q, ld_k, ld_v                        elements from one token of q, k, v
- *                                           to the next; 0 = dense (H*dk, H*dk,
+ *                                           to the next; 0 = dense (Hk*dk, Hk*dk,
  *                                           H*dv). Larger strides let q, k and v
  *                                           be views into one fused [T_tot, C]
  *                                           buffer, e.g. the conv output. Each
@@ -153,12 +162,13 @@ GDN_API size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, i
  *   workspace       ws_bytes >= gdn_prefill_workspace_size(...)
  * A sequence of length 0 writes hT = h0 (or zeros) and no output.
  * Supported: dk, dv in {16, 32, ..., 128}; chunk in {16, 32, 64}.
+ * Hk < 0 or H not a multiple of Hk: GDN_ERR_INVALID_ARG.
  * Except for hT == h0, no two buffers may overlap.
  */
 GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                          const float* g, const float* beta,
                          const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
-                         int N, int64_t T_tot, int H, int dk, int dv,
+                         int N, int64_t T_tot, int H, int Hk, int dk, int dv,
                          int64_t ld_q, int64_t ld_k, int64_t ld_v,
                          float scale, int qk_l2norm, float eps, int chunk,
                          const float* h0, float* hT, void* o,
@@ -188,7 +198,7 @@ GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gd
 GDN_API gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v,
                                          gdn_dtype_t dtype, const float* g, const float* beta,
                                          const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
-                                         int N, int64_t T_tot, int H, int dk, int dv,
+                                         int N, int64_t T_tot, int H, int Hk, int dk, int dv,
                                          int64_t ld_q, int64_t ld_k, int64_t ld_v,
                                          float scale, int qk_l2norm, float eps, int chunk,
                                          const float* h0, float* hT, void* o, gdn_algo_t algo,
@@ -208,7 +218,7 @@ GDN_API int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chu
  * Same per-token rule as gdn_prefill; `state` is read and overwritten in
  * place with the post-token state.
  *
- *   q, k     [N, H, dk]       dtype
+ *   q, k     [N, Hk, dk]      dtype   (Hk = 0: Hk = H; see "Heads" above)
  *   v        [N, H, dv]       dtype
  *   g, beta  [N, H]           fp32
  *   state    [N, H, dk, dv]   fp32   in/out
@@ -217,13 +227,13 @@ GDN_API int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chu
  */
 GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                              const float* g, const float* beta, float* state,
-                             int N, int H, int dk, int dv, float scale, int qk_l2norm,
+                             int N, int H, int Hk, int dk, int dv, float scale, int qk_l2norm,
                              float eps, void* o, void* stream);
 
 /*
  * The whole mixer for one decode token per sequence, in one kernel. [C] [R] [G] [P]
  *
- * For each sequence n the fused channels x[n] = [q | k | v] (C = 2*H*dk + H*dv,
+ * For each sequence n the fused channels x[n] = [q | k | v] (C = 2*Hk*dk + H*dv,
  * head-major inside each block) go through the causal conv against the
  * sequence's conv state (the K-1 previous inputs, oldest first):
  *   y_c = w[c, K-1] * x[n, c] + sum_{j<K-1} w[c, j] * conv_state[n, c, j]
@@ -241,12 +251,14 @@ GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v
  *   z           [N, H, dv]        dtype   nullable: no gate
  *   norm_w      [dv]              fp32    required when z is given
  *   o           [N, H, dv]        dtype   output
- * Supported: dk, dv in {16, 32, ..., 128}. No buffer may overlap another.
+ * Supported: dk, dv in {16, 32, ..., 128}; H / Hk <= 8 (the CTAs of one
+ * value-head group run as one thread-block cluster; larger groups return
+ * GDN_ERR_UNSUPPORTED). No buffer may overlap another.
  */
 GDN_API gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv_state, int K,
                                            gdn_dtype_t dtype, const float* g, const float* beta,
                                            float* state, const void* z, const float* norm_w,
-                                           float norm_eps, int N, int H, int dk, int dv,
+                                           float norm_eps, int N, int H, int Hk, int dk, int dv,
                                            float scale, int qk_l2norm, float eps, void* o,
                                            void* stream);
 

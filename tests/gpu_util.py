@@ -61,9 +61,10 @@ def prefill_oracle(P, h0=None):
 def oracle_unit(P, n: int, h: int):
     """Oracle on one (sequence, head) of a packed problem: (o [T_n, dv], hT [dk, dv])."""
     a, b = int(P.cu_seqlens[n]), int(P.cu_seqlens[n + 1])
-    sl = lambda x: np.ascontiguousarray(x[a:b, h:h + 1])
+    sl = lambda x, i=h: np.ascontiguousarray(x[a:b, i:i + 1])
+    hk = h // (P.H // P.Hk)  # the q, k head of value head h
     h0 = None if P.h0 is None else P.h0[n:n + 1, h:h + 1]
-    o, hT = oracle.recurrence(sl(P.q), sl(P.k), sl(P.v), sl(P.g), sl(P.beta), [0, b - a],
+    o, hT = oracle.recurrence(sl(P.q, hk), sl(P.k, hk), sl(P.v), sl(P.g), sl(P.beta), [0, b - a],
                               dtype=P.dtype, h0=h0, scale=P.scale, qk_l2norm=P.qk_l2norm,
                               eps=P.eps, threads=1)
     return o[:, 0], hT[0, 0]

@@ -125,6 +125,41 @@ def test_prefill_token_strided_views_equal_dense(algo):
     assert np.array_equal(host(o), o_d) and np.array_equal(host(hT), h_d)
 
 
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("H,Hk", [(6, 3), (8, 2)])
+def test_prefill_grouped_value_heads(algo, H, Hk):
+    """H value heads on Hk q, k heads (value head h reads q, k head h // (H // Hk)),
+    ragged lengths with an empty sequence and an initial state."""
+    P = gi.random_prefill(15, [1, 130, 0, 64, 77], H=H, Hk=Hk, dk=128, dv=128, with_h0=True)
+    o, hT = prefill_gpu(P, algo=algo)
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_BF16
+    assert err(hT, h_ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_prefill_grouped_value_heads_from_fused_buffer(algo):
+    """Grouped heads read in place from one fused [T, 2 Hk dk + H dv (+pad)] buffer
+    (the conv output's layout) give the dense result bit for bit."""
+    H, Hk, d = 4, 2, 128
+    P = gi.random_prefill(16, [70, 129, 64], H=H, Hk=Hk, dk=d, dv=d, with_h0=True)
+    o_d, h_d = prefill_gpu(P, algo=algo)
+    T = P.T_tot
+    widths = [Hk * d, Hk * d, H * d]
+    ld = sum(widths) + 32
+    fused = torch.zeros((T, ld), dtype=torch.bfloat16, device=DEV)
+    views, c0 = [], 0
+    for a, wdt, nh in zip((P.q, P.k, P.v), widths, (Hk, Hk, H)):
+        fused[:, c0:c0 + wdt] = dev_tensor(a, "bf16").view(T, wdt)
+        views.append(fused[:, c0:c0 + wdt].view(T, nh, d))
+        c0 += wdt
+    o, hT = gdn.prefill(*views, dev_tensor(P.g, "f32"), dev_tensor(P.beta, "f32"),
+                        torch.from_numpy(P.cu_seqlens).to(DEV),
+                        initial_state=dev_tensor(P.h0, "f32"), algo=algo)
+    gdn.check_device_status(DEV)
+    assert np.array_equal(host(o), o_d) and np.array_equal(host(hT), h_d)
+
+
 def test_chunk_sizes_agree():
     P = gi.random_prefill(4, [100, 37], H=2, dk=32, dv=32, dtype="f32", with_h0=True)
     outs = [prefill_gpu(P, chunk=c) for c in (16, 32, 64)]
@@ -205,6 +240,25 @@ def test_decode_step_matches_oracle(kind, dk, dv):
                                      scale=0.9)
     assert err(host(o), o_ref) <= tol(kind)
     assert err(host(state), s_ref) <= TOL_F32  # the state never passes through bf16
+
+
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+def test_decode_step_grouped_value_heads(kind):
+    r = np.random.default_rng(9)
+    N, H, Hk, dk, dv = 5, 6, 2, 128, 128
+    q, k = r.normal(size=(N, Hk, dk)).astype(np.float32), r.normal(size=(N, Hk, dk)).astype(np.float32)
+    v = r.normal(size=(N, H, dv)).astype(np.float32)
+    if kind == "bf16":
+        q, k, v = gi.to_bf16_bits(q), gi.to_bf16_bits(k), gi.to_bf16_bits(v)
+    g = -np.abs(r.normal(size=(N, H))).astype(np.float32)
+    beta = r.uniform(size=(N, H)).astype(np.float32)
+    s0 = r.normal(0, 0.1, size=(N, H, dk, dv)).astype(np.float32)
+    state = dev_tensor(s0, "f32")
+    o = gdn.decode_step(dev_tensor(q, kind), dev_tensor(k, kind), dev_tensor(v, kind),
+                        dev_tensor(g, "f32"), dev_tensor(beta, "f32"), state)
+    o_ref, s_ref = oracle.recurrence(q, k, v, g, beta, np.arange(N + 1), dtype=kind, h0=s0)
+    assert err(host(o), o_ref) <= tol(kind)
+    assert err(host(state), s_ref) <= TOL_F32
 
 
 def test_decode_workload_full_100_steps():
@@ -325,6 +379,46 @@ def test_decode_layer_step_matches_oracle(kind, gate, K):
     assert err(host(st_d), st_o) <= tol
     assert np.array_equal(host(cs_d), (gi.bf16_bits_to_f32(cs_o) if kind == "bf16" else cs_o)
                           .astype(np.float32))  # a pure shift: bit exact
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_decode_layer_step_grouped_value_heads(kind, G):
+    """G value heads per q, k head: the G CTAs of a group run as one cluster and
+    share the q, k conv channels; three tokens in a row check that the shared
+    conv state is shifted exactly once per token."""
+    r = np.random.default_rng(34 + G)
+    N, Hk, dk, dv, K = 5, 2, 128, 128, 4
+    H = G * Hk
+    C = 2 * Hk * dk + H * dv
+    to = (lambda a: gi.to_bf16_bits(a.astype(np.float32))) if kind == "bf16" else (
+        lambda a: a.astype(np.float32))
+    cw = to(r.normal(size=(C, K)) * 0.5)
+    cs = to(r.normal(size=(N, C, K - 1)))
+    st = (r.normal(size=(N, H, dk, dv)) * 0.1).astype(np.float32)
+    nw = (1.0 + 0.1 * r.normal(size=dv)).astype(np.float32)
+    cs_d, st_d = dev_tensor(cs, kind), torch.from_numpy(st).to(DEV)
+    cs_o, st_o = cs, st.astype(np.float64)
+    worst = 0.0
+    for t in range(3):
+        x = to(r.normal(size=(N, C)))
+        z = to(r.normal(size=(N, H, dv)))
+        g = (-np.log1p(np.exp(r.normal(size=(N, H))))).astype(np.float32)
+        b = (1.0 / (1.0 + np.exp(-r.normal(size=(N, H))))).astype(np.float32)
+        o = gdn.decode_layer_step(dev_tensor(x, kind), dev_tensor(cw, kind), cs_d,
+                                  torch.from_numpy(g).to(DEV), torch.from_numpy(b).to(DEV), st_d,
+                                  H=H, Hk=Hk, dk=dk, dv=dv, z=dev_tensor(z, kind),
+                                  norm_w=torch.from_numpy(nw).to(DEV))
+        o_ref, cs_n, st_o = oracle.decode_layer_step(x, cw, cs_o, g, b, st_o, dtype=kind, H=H,
+                                                     Hk=Hk, dk=dk, dv=dv, z=z, norm_w=nw)
+        cs_o = to(cs_n) if kind == "bf16" else cs_n
+        worst = max(worst, err(host(o), o_ref))
+    gdn.check_device_status(DEV)
+    tol_ = TOL_BF16 if kind == "bf16" else TOL_F32
+    assert worst <= tol_
+    assert err(host(st_d), st_o) <= tol_
+    assert np.array_equal(host(cs_d), (gi.bf16_bits_to_f32(cs_o) if kind == "bf16" else cs_o)
+                          .astype(np.float32))
 
 
 def test_decode_layer_step_equals_separate_kernels():
