@@ -33,8 +33,11 @@ namespace {
 __device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
 // Cluster-wide barrier in two halves (hardware barrier; no spinning in code).
-__device__ __forceinline__ void cluster_arrive_release() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+// The arrive is relaxed: what it has to order are reads of the conv state that
+// have already completed (cp.async waited, the data is in shared memory), and
+// a release would also wait for the state loads still in flight.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -106,7 +109,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
         T* cs = static_cast<T*>(a.conv_state) + n * C * (K - 1);
         cp_async_wait_all_groups();
         __syncthreads();
-        if (G > 1) cluster_arrive_release();  // this CTA's copy of the old conv state is in
+        if (G > 1) cluster_arrive_relaxed();  // this CTA's copy of the old conv state is in
         for (int c = tid; c < nconv; c += blockDim.x) {
             const float xt = Elem<T>::load(cx_s, c);
             float acc;
