@@ -590,6 +590,8 @@ def bench_grouped(args, dist, pk):
            "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
                         "peak": pk["hbm_gbs"], "unit": "GB/s",
                         "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                        "traffic": profiled_traffic("decode_layer_grouped_kernel", ["decode.cu"],
+                                                    Nd * Hv),
                         "algorithmic_bytes": bytes_step},
            "gpu_launches": steps}
     return {"prefill": pre, "decode_layer": dec}

@@ -43,8 +43,10 @@ __device__ __forceinline__ void cluster_wait_acquire() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Two CTAs of 256 threads per SM (128 registers a thread): the state streams
+// from HBM, so the kernel needs both CTAs' loads in flight.
 template <typename T, int RPT, bool CONV>
-__global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(256, 2) decode_step_kernel(DecodeArgs a) {
     extern __shared__ float sm[];
     const int dk = a.dk, dv = a.dv;
     const int cols4 = dv >> 2;
@@ -53,8 +55,6 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
     const int cg = tid % cols4;
     const int rg = tid / cols4;
     const int64_t nh = blockIdx.x;  // n * H + h
-    const int H = a.H, Hk = a.Hk, G = H / Hk;
-    const int n = (int)(nh / H), h = (int)(nh % H), hk = h / G;
 
     float* qs = sm;              // [dk]
     float* ks = qs + dk;         // [dk]
@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
     T* cw_s = cx_s + nconv;                           // [nconv][K]
     T* cs_s = cw_s + nconv * a.K;                     // [nconv][K-1]
     if constexpr (CONV) {
-        const int K = a.K;
+        const int H = a.H, Hk = a.Hk, G = H / Hk, K = a.K;
+        const int n = (int)(nh / H), h = (int)(nh % H), hk = h / G;
         const int64_t C = 2 * Hk * dk + H * dv;
         const T* x = static_cast<const T*>(a.x) + n * C;
         const T* w = static_cast<const T*>(a.conv_w);
@@ -104,7 +105,8 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
         // causal conv of this head's q, k, v channels against the conv state
         // (window: the K-1 stored inputs, oldest first, then x); the state shifts
         // by one and takes x as its newest entry
-        const int K = a.K;
+        const int H = a.H, Hk = a.Hk, G = H / Hk, K = a.K;
+        const int n = (int)(nh / H), h = (int)(nh % H), hk = h / G;
         const int64_t C = 2 * Hk * dk + H * dv;
         T* cs = static_cast<T*>(a.conv_state) + n * C * (K - 1);
         cp_async_wait_all_groups();
@@ -161,8 +163,9 @@ __global__ void __launch_bounds__(256) decode_step_kernel(DecodeArgs a) {
         __syncthreads();
         v4 = *reinterpret_cast<const float4*>(vs + 4 * cg);
     } else {
-        const T* qg = static_cast<const T*>(a.q) + ((int64_t)n * Hk + hk) * dk;
-        const T* kg = static_cast<const T*>(a.k) + ((int64_t)n * Hk + hk) * dk;
+        const int n = (int)(nh / a.H), hk = (int)(nh % a.H) / (a.H / a.Hk);
+        const T* qg = static_cast<const T*>(a.q) + ((int64_t)n * a.Hk + hk) * dk;
+        const T* kg = static_cast<const T*>(a.k) + ((int64_t)n * a.Hk + hk) * dk;
         for (int i = tid; i < dk; i += blockDim.x) {
             qs[i] = Elem<T>::load(qg, i);
             ks[i] = Elem<T>::load(kg, i);
