@@ -30,10 +30,11 @@ def lib():
         L = ctypes.CDLL(path)
         vp, i32, f64, i64p = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
         L.gdn_oracle_recurrence_mut.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32,
-                                                i32, i32, f64, i32, f64, vp, i32, vp, vp, i32, i32]
+                                                i32, i32, f64, i32, f64, i32, vp, i32, vp, vp, i32,
+                                                i32]
         L.gdn_oracle_recurrence_mut.restype = i32
         L.gdn_oracle_chunked.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32, i32,
-                                         i32, f64, i32, f64, vp, i32, vp, vp, i32, i32]
+                                         i32, f64, i32, f64, i32, vp, i32, vp, vp, i32, i32]
         L.gdn_oracle_chunked.restype = i32
         L.gdn_oracle_conv_silu.argtypes = [vp, i32, vp, i32, i64p, i32, i32, i32, vp, i32, vp,
                                            i32, i32, i32, i32, f64, vp, i32]
@@ -62,8 +63,13 @@ def _ptr(a: Optional[np.ndarray]):
 
 def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: float = 1.0,
                qk_l2norm: bool = True, eps: float = 1e-6, threads: Optional[int] = None,
-               want_o: bool = True, mutation: int = 0):
+               want_o: bool = True, mutation: int = 0, undecayed: bool = False):
     """Token-by-token gated delta rule in fp64.
+
+    Default order (Qwen3.5-MoE source walkthrough, 4.3): decay the state, then
+    read kv_mem = S^T k. undecayed=True takes the order of "7.6 Qwen3.5:
+    linear-attention hybrid", 7.6.2: kv_mem is read from S_{t-1} before the
+    decay, S_t = alpha S_{t-1} + k [beta (v - S_{t-1}^T k)]^T.
 
     q,k [T,Hk,dk], v [T,H,dv] (uint16 bf16 bits when dtype=='bf16', else
     float), g/beta [T,H], cu_seqlens [N+1], h0 [N,H,dk,dv] or None.
@@ -85,8 +91,8 @@ def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: floa
     o = np.empty((T, H, dv), np.float64) if want_o else None
     rc = lib().gdn_oracle_recurrence_mut(
         _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, Hk, dk, dv,
-        float(scale), int(qk_l2norm), float(eps), _ptr(h0a), h0dt, _ptr(hT), _ptr(o),
-        threads or default_threads(), int(mutation))
+        float(scale), int(qk_l2norm), float(eps), int(undecayed), _ptr(h0a), h0dt, _ptr(hT),
+        _ptr(o), threads or default_threads(), int(mutation))
     if rc != 0:
         raise ValueError("oracle recurrence: bad arguments")
     return o, hT
@@ -94,7 +100,7 @@ def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: floa
 
 def chunked(q, k, v, g, beta, cu_seqlens, *, dtype: str, chunk: int, h0=None,
             scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6,
-            threads: Optional[int] = None):
+            threads: Optional[int] = None, undecayed: bool = False):
     """fp64 chunkwise (UT-transform) evaluation of the same recurrence; used
     only to check that the chunk algebra equals the token loop."""
     T, Hk, dk = q.shape
@@ -111,8 +117,8 @@ def chunked(q, k, v, g, beta, cu_seqlens, *, dtype: str, chunk: int, h0=None,
     o = np.empty((T, H, dv), np.float64)
     rc = lib().gdn_oracle_chunked(
         _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, Hk, dk, dv,
-        float(scale), int(qk_l2norm), float(eps), _ptr(h0a), h0dt, _ptr(hT), _ptr(o),
-        int(chunk), threads or default_threads())
+        float(scale), int(qk_l2norm), float(eps), int(undecayed), _ptr(h0a), h0dt, _ptr(hT),
+        _ptr(o), int(chunk), threads or default_threads())
     if rc != 0:
         raise ValueError("oracle chunked: bad arguments")
     return o, hT
@@ -169,7 +175,8 @@ def gated_rmsnorm(y, z, w, *, dtype: str, eps: float = 1e-6):
 
 def decode_layer_step(x, conv_w, conv_state, g, beta, state, *, dtype: str, H: int, dk: int,
                       dv: int, z=None, norm_w=None, norm_eps: float = 1e-6, scale: float = 1.0,
-                      qk_l2norm: bool = True, eps: float = 1e-6, Hk: Optional[int] = None):
+                      qk_l2norm: bool = True, eps: float = 1e-6, Hk: Optional[int] = None,
+                      undecayed: bool = False):
     """One decode token of the whole mixer per sequence: the conv update over the
     fused [q | k | v] channels from the conv state (then SiLU and the per-head L2
     norm of q and k), one step of the gated delta rule from `state`, and, when z
@@ -191,7 +198,7 @@ def decode_layer_step(x, conv_w, conv_state, g, beta, state, *, dtype: str, H: i
     v = y[:, 2 * Hk * dk:].reshape(N, H, dv)
     o, hT = recurrence(q, k, v, np.asarray(g, np.float64), np.asarray(beta, np.float64), cu,
                        dtype="f64", h0=np.asarray(state, np.float64), scale=scale,
-                       qk_l2norm=False, threads=1)
+                       qk_l2norm=False, threads=1, undecayed=undecayed)
     if z is not None:  # o is already fp64; z arrives in the inputs' encoding
         o = gated_rmsnorm(o, _to_f64(z, dtype), norm_w, dtype="f64", eps=norm_eps)
     return o, cs, hT

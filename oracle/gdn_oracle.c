@@ -19,6 +19,10 @@
  *   [S] Same page as [R], section 8.2: the prefill keeps the last K conv inputs
  *       as the conv state (left-padded when the sequence is shorter than K),
  *       and the recurrent state is carried from call to call.
+ *   [U] "7.6 Qwen3.5: linear-attention hybrid", 7.6.2, the recurrence as that
+ *       page writes it: S_t = alpha_t S_{t-1} + k_t [beta_t (v_t - S_{t-1}^T k_t)]^T,
+ *       i.e. the memory is read from the state before the decay. Selected by
+ *       `undecayed`; [R]'s decay-first order is the default.
  * Readings where the pages are silent (all listed in the design notes):
  *   SiLU follows the conv; L2(x) = x / sqrt(sum x^2 + eps); `scale` multiplies
  *   the normalised q; the conv state exposes the K-1 most recent inputs
@@ -105,6 +109,7 @@ typedef struct {
     double scale;
     int qk_l2norm;
     double eps;
+    int undecayed; /* 1: read kv_mem from the state before the decay ([U]) */
     const void *h0;
     int h0_dtype;
     double *hT, *o;
@@ -150,8 +155,9 @@ static void rec_item(void *vctx, int64_t item) {
         const double beta = load_elem(c->beta, c->gate_dtype, t * H + h);
         const double alpha = exp(g);
 
-        /* mutation 1 (pin check only): read the memory before the decay */
-        if (c->mutation == 1)
+        /* [U]: kv_mem_j = sum_i S_{t-1}[i][j] k_i, before the decay.
+         * (mutation 1, pin check only: the same read planted in the default rule) */
+        if (c->undecayed || c->mutation == 1)
             for (int j = 0; j < dv; ++j) {
                 double acc = 0.0;
                 for (int i = 0; i < dk; ++i) acc += S[i * dv + j] * k[i];
@@ -162,8 +168,8 @@ static void rec_item(void *vctx, int64_t item) {
         if (c->mutation != 3)
             for (int64_t e = 0; e < (int64_t)dk * dv; ++e) S[e] *= alpha;
 
-        /* kv_mem_j = sum_i S[i][j] k_i  (reduction over the key axis) */
-        if (c->mutation != 1)
+        /* [R]: kv_mem_j = sum_i S[i][j] k_i  (reduction over the key axis) */
+        if (!c->undecayed && c->mutation != 1)
             for (int j = 0; j < dv; ++j) {
                 double acc = 0.0;
                 for (int i = 0; i < dk; ++i) {
@@ -207,17 +213,18 @@ static void rec_item(void *vctx, int64_t item) {
  *   hT [N,H,dk,dv] double or NULL, o [T_tot,H,dv] double or NULL.
  * Value head h reads q and k of head h / (H / Hk) (grouped value heads: the
  * config's linear_num_value_heads may exceed linear_num_key_heads; H == Hk is
- * the plain layer). Returns 0, or -1 on a bad argument.
+ * the plain layer). undecayed = 1 selects the [U] order (read, then decay).
+ * Returns 0, or -1 on a bad argument.
  */
 int gdn_oracle_recurrence_mut(const void *q, const void *k, const void *v, int dtype,
                               const void *g, const void *beta, int gate_dtype,
                               const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
-                              double scale, int qk_l2norm, double eps,
+                              double scale, int qk_l2norm, double eps, int undecayed,
                               const void *h0, int h0_dtype, double *hT, double *o,
                               int n_threads, int mutation) {
     if (N < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
     rec_ctx c = {q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, Hk, dk, dv, scale,
-                 qk_l2norm, eps, h0, h0_dtype, hT, o, mutation};
+                 qk_l2norm, eps, undecayed, h0, h0_dtype, hT, o, mutation};
     run_items(rec_item, &c, (int64_t)N * H, n_threads);
     return 0;
 }
@@ -225,10 +232,10 @@ int gdn_oracle_recurrence_mut(const void *q, const void *k, const void *v, int d
 int gdn_oracle_recurrence(const void *q, const void *k, const void *v, int dtype,
                           const void *g, const void *beta, int gate_dtype,
                           const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
-                          double scale, int qk_l2norm, double eps,
+                          double scale, int qk_l2norm, double eps, int undecayed,
                           const void *h0, int h0_dtype, double *hT, double *o, int n_threads) {
     return gdn_oracle_recurrence_mut(q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, N, H, Hk,
-                                     dk, dv, scale, qk_l2norm, eps, h0, h0_dtype, hT, o,
+                                     dk, dv, scale, qk_l2norm, eps, undecayed, h0, h0_dtype, hT, o,
                                      n_threads, 0);
 }
 
@@ -334,6 +341,7 @@ static void chunk_item(void *vctx, int64_t item) {
     double *Kc = (double *)malloc(sizeof(double) * Cs * dk);
     double *V = (double *)malloc(sizeof(double) * Cs * dv);
     double *gam = (double *)malloc(sizeof(double) * Cs);
+    double *grow = (double *)malloc(sizeof(double) * Cs);
     double *bet = (double *)malloc(sizeof(double) * Cs);
     double *A = (double *)malloc(sizeof(double) * Cs * Cs);
     double *Tm = (double *)malloc(sizeof(double) * Cs * Cs);
@@ -363,14 +371,18 @@ static void chunk_item(void *vctx, int64_t item) {
             gam[r] = acc_g; /* gamma_r = sum_{i<=r} g_i */
             bet[r] = load_elem(c->beta, c->gate_dtype, t * H + h);
         }
-        /* A[r][j] = beta_r exp(gamma_r - gamma_j) k_r.k_j for j < r */
+        /* Decay of the row whose delta is being solved for: token r reads the
+         * state after gamma_r of decay ([R]), or before its own decay, i.e. after
+         * gamma_{r-1} = gamma_r - g_r ([U]; gamma_{-1} = 0). */
+        for (int r = 0; r < L; ++r) grow[r] = c->undecayed ? (r > 0 ? gam[r - 1] : 0.0) : gam[r];
+        /* A[r][j] = beta_r exp(grow_r - gamma_j) k_r.k_j for j < r */
         for (int r = 0; r < L; ++r)
             for (int j = 0; j < L; ++j) {
                 double a = 0.0;
                 if (j < r) {
                     double dot = 0.0;
                     for (int i = 0; i < dk; ++i) dot += Kc[r * dk + i] * Kc[j * dk + i];
-                    a = bet[r] * exp(gam[r] - gam[j]) * dot;
+                    a = bet[r] * exp(grow[r] - gam[j]) * dot;
                 }
                 A[r * Cs + j] = a;
             }
@@ -382,11 +394,11 @@ static void chunk_item(void *vctx, int64_t item) {
                     for (int m = j; m < r; ++m) s -= A[r * Cs + m] * Tm[m * Cs + j];
                 Tm[r * Cs + j] = (j <= r) ? s : 0.0;
             }
-        /* W = Tm diag(beta e^gamma) K ; U = Tm diag(beta) V - W S */
+        /* W = Tm diag(beta e^grow) K ; U = Tm diag(beta) V - W S */
         for (int r = 0; r < L; ++r) {
             for (int i = 0; i < dk; ++i) {
                 double s = 0.0;
-                for (int m = 0; m <= r; ++m) s += Tm[r * Cs + m] * bet[m] * exp(gam[m]) * Kc[m * dk + i];
+                for (int m = 0; m <= r; ++m) s += Tm[r * Cs + m] * bet[m] * exp(grow[m]) * Kc[m * dk + i];
                 W[r * dk + i] = s;
             }
             for (int j = 0; j < dv; ++j) {
@@ -420,20 +432,20 @@ static void chunk_item(void *vctx, int64_t item) {
         memcpy(S, Sn, sizeof(double) * (size_t)dk * dv);
     }
     if (c->hT) memcpy(c->hT + sbase, S, sizeof(double) * (size_t)dk * dv);
-    free(S); free(Q); free(Kc); free(V); free(gam); free(bet); free(A); free(Tm);
+    free(S); free(Q); free(Kc); free(V); free(gam); free(grow); free(bet); free(A); free(Tm);
     free(W); free(U); free(Sn);
 }
 
 int gdn_oracle_chunked(const void *q, const void *k, const void *v, int dtype,
                        const void *g, const void *beta, int gate_dtype,
                        const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
-                       double scale, int qk_l2norm, double eps,
+                       double scale, int qk_l2norm, double eps, int undecayed,
                        const void *h0, int h0_dtype, double *hT, double *o,
                        int chunk, int n_threads) {
     if (N < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || dk <= 0 || dv <= 0 || chunk <= 0 || !cu_seqlens)
         return -1;
     chunk_ctx c = {{q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, Hk, dk, dv, scale, qk_l2norm,
-                    eps, h0, h0_dtype, hT, o, 0},
+                    eps, undecayed, h0, h0_dtype, hT, o, 0},
                    chunk};
     run_items(chunk_item, &c, (int64_t)N * H, n_threads);
     return 0;

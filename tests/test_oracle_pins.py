@@ -115,13 +115,17 @@ def pin_decay_first(rec):
     return np.abs(hT[0, 0].T @ kk - ref).max()
 
 
-def _unrolled(q, k, v, alpha, beta, S0):
+def _unrolled(q, k, v, alpha, beta, S0, undecayed=False):
     """Transposed orientation P = S^T ([d_v, d_k]); P_t = P_0 prod B_j +
-    sum_i b_i v_i k_i^T prod_{j>i} B_j with B_j = a_j (I - b_j k_j k_j^T),
-    every product formed explicitly left to right. Returns (o [T,dv], P_T)."""
+    sum_i b_i v_i k_i^T prod_{j>i} B_j with B_j = a_j (I - b_j k_j k_j^T)
+    (or B_j = a_j I - b_j k_j k_j^T for the read-before-decay order), every
+    product formed explicitly left to right. Returns (o [T,dv], P_T)."""
     T, dk = k.shape
     I = np.eye(dk)
-    B = [alpha[j] * (I - beta[j] * np.outer(k[j], k[j])) for j in range(T)]
+    if undecayed:
+        B = [alpha[j] * I - beta[j] * np.outer(k[j], k[j]) for j in range(T)]
+    else:
+        B = [alpha[j] * (I - beta[j] * np.outer(k[j], k[j])) for j in range(T)]
     outs, P = [], None
     for t in range(1, T + 1):
         P = S0.T.copy()
@@ -502,6 +506,99 @@ def test_grouped_value_heads_reject_uneven_groups():
     g, b = np.zeros((4, 3)), np.zeros((4, 3))
     with pytest.raises(ValueError):
         oracle.recurrence(q, k, v, g, b, [0, 4], dtype="f64", threads=1)
+
+
+# --------------------------------------------------------------------------
+# The order "7.6 Qwen3.5: linear-attention hybrid", 7.6.2 writes: the memory
+# is read from S_{t-1} before the decay, S_t = a S_{t-1} + k [b (v - S_{t-1}^T k)]^T,
+# i.e. S_t = (a I - b k k^T) S_{t-1} + b k v^T (the oracle's undecayed=True).
+# --------------------------------------------------------------------------
+
+def test_undecayed_brute_force():
+    for seed, (T, dk, dv) in enumerate([(1, 1, 1), (3, 2, 3), (6, 4, 4), (5, 3, 2)]):
+        r = _rng(200 + seed)
+        q, k = r.normal(size=(T, dk)), r.normal(size=(T, dk))
+        v = r.normal(size=(T, dv))
+        g = -np.abs(r.normal(size=T)); beta = r.uniform(size=T)
+        S0 = r.normal(size=(dk, dv))
+        o_ref, P = _unrolled(_unit(q) * 0.7, _unit(k), v, np.exp(g), beta, S0, undecayed=True)
+        o, hT = _rec()(q[:, None], k[:, None], v[:, None], g[:, None], beta[:, None], [0, T],
+                       h0=S0[None, None], scale=0.7, eps=0.0, undecayed=True)
+        assert np.abs(o[:, 0] - o_ref).max() < 1e-12 and np.abs(hT[0, 0] - P.T).max() < 1e-12
+
+
+def test_undecayed_unit_key_one_step():
+    # for unit k: S_1^T k = (a - b) S_0^T k + b v (the decay-first order gives a (1 - b) S_0^T k + b v)
+    r = _rng(210)
+    dk = dv = 5
+    h0 = r.normal(size=(1, 1, dk, dv))
+    kk = _unit(r.normal(size=dk)); vv = r.normal(size=dv)
+    a, b = 0.5, 0.3
+    _, hT = _rec()(kk[None, None], kk[None, None], vv[None, None], [[math.log(a)]], [[b]], [0, 1],
+                   h0=h0, qk_l2norm=False, undecayed=True)
+    assert np.abs(hT[0, 0].T @ kk - ((a - b) * (h0[0, 0].T @ kk) + b * vv)).max() < 1e-13
+
+
+def test_undecayed_equals_reparametrised_default():
+    # (a I - b k k^T) S + b k v^T = a (I - (b/a) k k^T) S + (b/a) k (a v)^T: the read-before-decay
+    # order with (beta, v) is the decay-first order with (beta / alpha, alpha v)
+    r = _rng(211)
+    T, H, dk, dv = 40, 2, 6, 4
+    q, k, v = r.normal(size=(T, H, dk)), r.normal(size=(T, H, dk)), r.normal(size=(T, H, dv))
+    g = -0.5 * np.abs(r.normal(size=(T, H))); beta = r.uniform(size=(T, H))
+    h0 = r.normal(size=(1, H, dk, dv))
+    a = np.exp(g)
+    o1, h1 = _rec()(q, k, v, g, beta, [0, T], h0=h0, undecayed=True)
+    o2, h2 = _rec()(q, k, v * a[..., None], g, beta / a, [0, T], h0=h0)
+    assert np.abs(o1 - o2).max() < 1e-12 * np.abs(o1).max()
+    assert np.abs(h1 - h2).max() < 1e-12 * np.abs(h1).max()
+    # with no decay the two orders coincide exactly; with decay they differ
+    o3, _ = _rec()(q, k, v, np.zeros_like(g), beta, [0, T], h0=h0, undecayed=True)
+    o4, _ = _rec()(q, k, v, np.zeros_like(g), beta, [0, T], h0=h0)
+    assert np.array_equal(o3, o4)
+    o5, _ = _rec()(q, k, v, g, beta, [0, T], h0=h0)
+    assert np.abs(o5 - o1).max() > 1e-2
+
+
+@pytest.mark.parametrize("chunk", [1, 4, 16, 64])
+def test_undecayed_chunked_evaluator_equals_token_loop(chunk):
+    # chunk form of the read-before-decay order: row decay e^{gamma_{r-1}} in A and W
+    r = _rng(212)
+    lens = [70, 3, 64, 129, 1]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    H, dk, dv = 2, 8, 6
+    T = int(cu[-1])
+    q, k, v = r.normal(size=(T, H, dk)), r.normal(size=(T, H, dk)), r.normal(size=(T, H, dv))
+    g = -0.3 * np.abs(r.normal(size=(T, H))); beta = r.uniform(size=(T, H))
+    g[5:9] = -9.0  # strong decay inside a chunk
+    h0 = r.normal(size=(len(lens), H, dk, dv))
+    kw = dict(dtype="f64", h0=h0, scale=0.8, threads=2, undecayed=True)
+    o1, h1 = oracle.recurrence(q, k, v, g, beta, cu, **kw)
+    o2, h2 = oracle.chunked(q, k, v, g, beta, cu, chunk=chunk, **kw)
+    assert np.abs(o1 - o2).max() <= 1e-12 * np.abs(o1).max()
+    assert np.abs(h1 - h2).max() <= 1e-12 * np.abs(h1).max()
+
+
+def test_undecayed_decode_layer_steps_equal_packed_layer():
+    r = _rng(213)
+    H, dk, dv, K, T = 2, 4, 3, 4, 6
+    C = 2 * H * dk + H * dv
+    x, cw = r.normal(size=(T, C)), r.normal(size=(C, K))
+    cs0, h0 = r.normal(size=(1, C, K - 1)), r.normal(size=(1, H, dk, dv)) * 0.3
+    g = -np.abs(r.normal(size=(T, H))) * 0.3
+    b = 1.0 / (1.0 + np.exp(-r.normal(size=(T, H))))
+    y, _ = oracle.conv_silu(x, cw, [0, T], dtype="f64", state_in=cs0, qk_l2norm=True,
+                            n_qk=2 * H * dk, head_dim=dk, eps=1e-6)
+    o_ref, h_ref = oracle.recurrence(y[:, :H * dk].reshape(T, H, dk),
+                                     y[:, H * dk:2 * H * dk].reshape(T, H, dk),
+                                     y[:, 2 * H * dk:].reshape(T, H, dv), g, b, [0, T],
+                                     dtype="f64", h0=h0, qk_l2norm=False, undecayed=True)
+    cs, st = cs0, h0
+    for t in range(T):
+        o, cs, st = oracle.decode_layer_step(x[t:t + 1], cw, cs, g[t:t + 1], b[t:t + 1], st,
+                                             dtype="f64", H=H, dk=dk, dv=dv, undecayed=True)
+        assert np.abs(o[0] - o_ref[t]).max() < 1e-12
+    assert np.abs(st - h_ref).max() < 1e-12
 
 
 # --------------------------------------------------------------------------
