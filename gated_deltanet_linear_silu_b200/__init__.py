@@ -57,12 +57,13 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
         L.gdn_prefill_workspace_size.restype = sz
         L.gdn_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
-                                  i64, i64, i64, f32, i32, f32, i32, vp, vp, vp, vp, sz, i32, vp]
+                                  i64, i64, i64, f32, i32, f32, i32, i32, vp, vp, vp, vp, sz, i32,
+                                  vp]
         L.gdn_prefill.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
-                                      f32, vp, vp]
+                                      f32, i32, vp, vp]
         L.gdn_decode_layer_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, f32, i32, i32,
-                                            i32, i32, i32, f32, i32, f32, vp, vp]
+                                            i32, i32, i32, f32, i32, f32, i32, vp, vp]
         L.gdn_decode_layer_step.restype = i32
         L.gdn_gated_rmsnorm.argtypes = [vp, vp, vp, i32, i64, i32, f32, vp, vp]
         L.gdn_gated_rmsnorm.restype = i32
@@ -72,7 +73,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_check_device_status.argtypes = [vp]
         L.gdn_check_device_status.restype = i32
         L.gdn_prefill_noalloc.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32,
-                                          i32, i64, i64, i64, f32, i32, f32, i32, vp, vp, vp, i32, vp]
+                                          i32, i64, i64, i64, f32, i32, f32, i32, i32, vp, vp, vp,
+                                          i32, vp]
         L.gdn_prefill_noalloc.restype = i32
         L.gdn_prefill_noalloc_max_scratch.argtypes = []
         L.gdn_prefill_noalloc_max_scratch.restype = sz
@@ -156,13 +158,14 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
             output_final_state: bool = True, final_state: Optional[torch.Tensor] = None,
             scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6, chunk: int = 64,
             cu_seqlens_host: Optional[torch.Tensor] = None, algo: str = "auto",
-            workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None
-            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+            undecayed: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked gated delta rule. q,k [T,Hk,dk], v [T,H,dv] (bf16 or fp32; each
     may be a token-strided view, e.g. a slice of the fused conv output; Hk < H
     groups H / Hk value heads on each q, k head), g,beta [T,H] fp32, cu_seqlens
     int32 [N+1] (device). Returns (o, hT); final_state may be initial_state
-    itself for an in-place update."""
+    itself for an in-place update. undecayed=True reads each token's memory
+    from the state before its decay (the 7.6.2 order)."""
     T, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
     N = cu_seqlens.shape[0] - 1
@@ -181,7 +184,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     st = lib().gdn_prefill(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
         None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
-        ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(chunk), _ptr(initial_state), _ptr(hT),
+        ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(undecayed), int(chunk),
+        _ptr(initial_state), _ptr(hT),
         _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill")
     return o, hT
@@ -191,7 +195,8 @@ def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
                     beta: torch.Tensor, cu_seqlens: torch.Tensor, *,
                     initial_state: Optional[torch.Tensor] = None, final_state: torch.Tensor,
                     out: torch.Tensor, scale: float = 1.0, qk_l2norm: bool = True,
-                    eps: float = 1e-6, chunk: int = 64, algo: str = "auto") -> None:
+                    eps: float = 1e-6, chunk: int = 64, algo: str = "auto",
+                    undecayed: bool = False) -> None:
     """gdn_prefill_noalloc: prefill with the library's fixed scratch array
     instead of a workspace; the caller passes every output buffer, so nothing
     is allocated."""
@@ -202,7 +207,8 @@ def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
     _cuda(g, beta, cu_seqlens, initial_state, final_state, out)
     st = lib().gdn_prefill_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens), None,
-        N, T, H, Hk, dk, dv, ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(chunk),
+        N, T, H, Hk, dk, dv, ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps),
+        int(undecayed), int(chunk),
         _ptr(initial_state), _ptr(final_state), _ptr(out), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill_noalloc")
 
@@ -219,8 +225,8 @@ def selected_algo(dtype: str, dk: int, dv: int, chunk: int = 64, algo: str = "au
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                 beta: torch.Tensor, state: torch.Tensor, *, scale: float = 1.0,
-                qk_l2norm: bool = True, eps: float = 1e-6, out: Optional[torch.Tensor] = None
-                ) -> torch.Tensor:
+                qk_l2norm: bool = True, eps: float = 1e-6, out: Optional[torch.Tensor] = None,
+                undecayed: bool = False) -> torch.Tensor:
     """One recurrent token per sequence. q,k [N,Hk,dk], v [N,H,dv], g,beta
     [N,H] fp32, state [N,H,dk,dv] fp32 updated in place. Returns o [N,H,dv]."""
     N, Hk, dk = q.shape
@@ -229,7 +235,7 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     _cuda(q, k, v, g, beta, state, o)
     st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta),
                                _ptr(state), N, H, Hk, dk, dv, float(scale), int(qk_l2norm), float(eps),
-                               _ptr(o), _stream(q.device))
+                               int(undecayed), _ptr(o), _stream(q.device))
     _check(st, "gdn_decode_step")
     return o
 
@@ -239,7 +245,8 @@ def decode_layer_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: Optiona
                       dv: int, z: Optional[torch.Tensor] = None,
                       norm_w: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
                       scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6,
-                      out: Optional[torch.Tensor] = None, Hk: Optional[int] = None) -> torch.Tensor:
+                      out: Optional[torch.Tensor] = None, Hk: Optional[int] = None,
+                      undecayed: bool = False) -> torch.Tensor:
     """One decode token of the whole mixer per sequence. x [N, C] fused
     [q | k | v] projections (C = 2 Hk dk + H dv; Hk q, k heads, default H),
     conv_w [C, K], conv_state [N, C, K-1] and state [N, H, dk, dv] fp32 updated
@@ -255,7 +262,7 @@ def decode_layer_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: Optiona
     st = lib().gdn_decode_layer_step(_ptr(x), _ptr(conv_w), _ptr(conv_state), K, _dtype_code(x),
                                      _ptr(g), _ptr(beta), _ptr(state), _ptr(z), _ptr(norm_w),
                                      float(norm_eps), N, H, Hk, dk, dv, float(scale), int(qk_l2norm),
-                                     float(eps), _ptr(o), _stream(x.device))
+                                     float(eps), int(undecayed), _ptr(o), _stream(x.device))
     _check(st, "gdn_decode_layer_step")
     return o
 

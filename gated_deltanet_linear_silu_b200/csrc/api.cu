@@ -117,8 +117,9 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
                          const float* g, const float* beta, const int32_t* cu_seqlens,
                          const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
                          int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale,
-                         int qk_l2norm, float eps, int chunk, const float* h0, float* hT, void* o,
-                         void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream) {
+                         int qk_l2norm, float eps, int undecayed, int chunk, const float* h0,
+                         float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
+                         void* stream) {
     if (Hk == 0) Hk = H;
     if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0 || Hk < 0 || H % Hk != 0)
         return GDN_ERR_INVALID_ARG;
@@ -133,6 +134,7 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
         !aligned16(hT))
         return GDN_ERR_INVALID_ARG;
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if (undecayed != 0 && undecayed != 1) return GDN_ERR_INVALID_ARG;
     const int64_t esz = dtype == GDN_BF16 ? 2 : 4;
     if (ld_q == 0) ld_q = (int64_t)Hk * dk;
     if (ld_k == 0) ld_k = (int64_t)Hk * dk;
@@ -149,7 +151,7 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
         return GDN_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     gdn::PrefillArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, Hk, dk, dv,
-                       ld_q, ld_k, ld_v, scale, qk_l2norm, eps, chunk, h0, hT, o,
+                       ld_q, ld_k, ld_v, scale, qk_l2norm, eps, undecayed, chunk, h0, hT, o,
                        reinterpret_cast<int32_t*>(ws + wl.order_off),
                        reinterpret_cast<int32_t*>(ws + wl.counter_off), status_ptr()};
     if (!a.status) return GDN_ERR_CUDA;
@@ -182,10 +184,11 @@ int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_
 
 gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                              const float* g, const float* beta, float* state, int N, int H, int Hk,
-                             int dk, int dv, float scale, int qk_l2norm, float eps, void* o,
-                             void* stream) {
+                             int dk, int dv, float scale, int qk_l2norm, float eps, int undecayed,
+                             void* o, void* stream) {
     if (Hk == 0) Hk = H;
     if (!dtype_ok(dtype) || N < 0 || H <= 0 || Hk < 0 || H % Hk != 0) return GDN_ERR_INVALID_ARG;
+    if (undecayed != 0 && undecayed != 1) return GDN_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (N == 0) return GDN_OK;
     if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
@@ -193,7 +196,7 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dt
         return GDN_ERR_INVALID_ARG;
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
-    gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, Hk, dk, dv, scale, qk_l2norm, eps, o,
+    gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, Hk, dk, dv, scale, qk_l2norm, eps, undecayed, o,
                       nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0.f};
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
 }
@@ -202,10 +205,11 @@ gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv
                                    gdn_dtype_t dtype, const float* g, const float* beta, float* state,
                                    const void* z, const float* norm_w, float norm_eps, int N, int H,
                                    int Hk, int dk, int dv, float scale, int qk_l2norm, float eps,
-                                   void* o, void* stream) {
+                                   int undecayed, void* o, void* stream) {
     if (Hk == 0) Hk = H;
     if (!dtype_ok(dtype) || N < 0 || H <= 0 || K < 1 || Hk < 0 || H % Hk != 0)
         return GDN_ERR_INVALID_ARG;
+    if (undecayed != 0 && undecayed != 1) return GDN_ERR_INVALID_ARG;
     if (K > 4 || H / Hk > gdn::kMaxDecodeGroup) return GDN_ERR_UNSUPPORTED;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (N == 0) return GDN_OK;
@@ -219,7 +223,7 @@ gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv
     if (z && !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
     gdn::DecodeArgs a{nullptr, nullptr, nullptr, dtype == GDN_BF16, g, beta, state, N, H, Hk, dk, dv,
-                      scale, qk_l2norm, eps, o, x, conv_w, conv_state, K, z, norm_w, norm_eps};
+                      scale, qk_l2norm, eps, undecayed, o, x, conv_w, conv_state, K, z, norm_w, norm_eps};
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
 }
 

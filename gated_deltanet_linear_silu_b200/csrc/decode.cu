@@ -222,12 +222,14 @@ __global__ void __launch_bounds__(256, 2) decode_step_kernel(DecodeArgs a) {
     }
     const float inv_k = scal[0], qsc = scal[1], kq = scal[2];
 
-    // 4. delta, output, state update.
+    // 4. delta, output, state update. The memory is alpha a (decay first) or a
+    // (read from the state before the decay).
+    const float mk = a.undecayed ? inv_k : alpha * inv_k;
     float4 d;
-    d.x = beta * (v4.x - alpha * inv_k * A.x);
-    d.y = beta * (v4.y - alpha * inv_k * A.y);
-    d.z = beta * (v4.z - alpha * inv_k * A.z);
-    d.w = beta * (v4.w - alpha * inv_k * A.w);
+    d.x = beta * (v4.x - mk * A.x);
+    d.y = beta * (v4.y - mk * A.y);
+    d.z = beta * (v4.z - mk * A.z);
+    d.w = beta * (v4.w - mk * A.w);
     // output: the rg == 0 threads, all in warp 0 (dv / 4 <= 32 columns groups)
     if (tid < 32) {
         float4 o = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -37,6 +37,7 @@ struct DecodeArgs {
     float scale;
     int qk_l2norm;
     float eps;
+    int undecayed;  // 1: the memory is read from the state before the decay
     void* o;
     // whole-mixer step (x != nullptr): q, k, v come from the conv update of x
     const void* x;        // [N, C] fused projections, C = 2*Hk*dk + H*dv
@@ -80,6 +81,7 @@ struct PrefillArgs {
     float scale;
     int qk_l2norm;
     float eps;
+    int undecayed;  // 1: each token reads the state before its own decay (gamma_{r-1} row decay)
     int chunk;
     const float* h0;
     float* hT;

@@ -56,7 +56,7 @@ gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v, gd
                                  const float* g, const float* beta, const int32_t* cu_seqlens,
                                  const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H,
                                  int Hk, int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v,
-                                 float scale, int qk_l2norm, float eps, int chunk,
+                                 float scale, int qk_l2norm, float eps, int undecayed, int chunk,
                                  const float* h0, float* hT, void* o, gdn_algo_t algo,
                                  void* stream) {
     if (N < 0) return GDN_ERR_INVALID_ARG;
@@ -68,7 +68,8 @@ gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v, gd
         if (!scratch) return GDN_ERR_CUDA;
     }
     return gdn_prefill(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv,
-                       ld_q, ld_k, ld_v, scale, qk_l2norm, eps, chunk, h0, hT, o, scratch, kNoallocScratchBytes,
+                       ld_q, ld_k, ld_v, scale, qk_l2norm, eps, undecayed, chunk, h0, hT, o, scratch,
+                       kNoallocScratchBytes,
                        algo, stream);
 }
 

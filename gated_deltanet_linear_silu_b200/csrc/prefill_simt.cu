@@ -186,9 +186,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
                 }
             }
             __syncthreads();
-            // 3. A = strict_tril(beta_r e^{gamma_r - gamma_j} K K^T);  P = tril(e^{..} Q K^T).
+            // 3. A = strict_tril(beta_r e^{grow_r - gamma_j} K K^T);  P = tril(e^{..} Q K^T).
+            // The row decay grow_r is gamma_r, or gamma_{r-1} (gamma_{-1} = 0) when
+            // token r reads the state before its own decay.
+            const bool und = a.undecayed != 0;
             gemm(C, C, dk, Ks, ldk, 1, Ks, 1, ldk, [&](int r, int j, float x) {
-                Am[r * ldc + j] = j < r ? bet[r] * expf(gam[r] - gam[j]) * x : 0.f;
+                const float gr = und ? (r > 0 ? gam[r - 1] : 0.f) : gam[r];
+                Am[r * ldc + j] = j < r ? bet[r] * expf(gr - gam[j]) * x : 0.f;
             });
             gemm(C, C, dk, Qs, ldk, 1, Ks, 1, ldk, [&](int r, int j, float x) {
                 Pm[r * ldc + j] = j <= r ? expf(gam[r] - gam[j]) * x : 0.f;
@@ -210,11 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(PrefillArgs a
                 }
             }
             __syncthreads();
-            // 5. T1 = T diag(beta e^gamma) (into Am), T2 = T diag(beta) (in place).
+            // 5. T1 = T diag(beta e^grow) (into Am), T2 = T diag(beta) (in place).
             for (int e = tid; e < C * C; e += kThreads) {
                 const int r = e / C, m = e % C;
                 const float t = Tm[r * ldc + m];
-                Am[r * ldc + m] = t * bet[m] * expf(gam[m]);
+                const float gm = und ? (m > 0 ? gam[m - 1] : 0.f) : gam[m];
+                Am[r * ldc + m] = t * bet[m] * expf(gm);
                 Tm[r * ldc + m] = t * bet[m];
             }
             __syncthreads();

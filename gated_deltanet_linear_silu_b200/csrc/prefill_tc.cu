@@ -438,6 +438,10 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
                 }
+                if (a.undecayed) {  // A's row decay then reaches back to gamma_{-1} = 0
+                    mx = fmaxf(mx, 0.f);
+                    mn = fminf(mn, 0.f);
+                }
                 constexpr float kLog2e = 1.4426950408889634f;
                 *reinterpret_cast<float2*>(vec + r) =
                     make_float2(ex2((mx - g0) * kLog2e), ex2((mx - g1) * kLog2e));
@@ -490,7 +494,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 if (rb >= cb) {
                     tmem_ld32(tmem + lane_off + kRA + 64 + 32 * half, x);  // columns = k rows
                     tmem_wait_ld();
-                    const float gr = gam[r];
+                    // row decay: gamma_r, or for A rows with the read-before-decay
+                    // order gamma_{r-1} (gamma_{-1} = 0)
+                    const float gr = (!is_p && a.undecayed) ? (r > 0 ? gam[r - 1] : 0.f) : gam[r];
                     const float fr = is_p ? rq[r] : bet[r] * rk[r];
                     const int lim = (is_p && rb == cb) ? r : 64;  // keep j <= lim
                     if (vec[65] != 0.f) {
@@ -622,7 +628,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 float x[32];
 #pragma unroll
                 for (int r = 0; r < 32; ++r) x[r] = sT[(32 * hf + r) * kLdA + j];
-                const float f = which == 0 ? bet[j] * expf(gam[j]) * rk[j] : bet[j];
+                const float gj = a.undecayed ? (j > 0 ? gam[j - 1] : 0.f) : gam[j];
+                const float f = which == 0 ? bet[j] * expf(gj) * rk[j] : bet[j];
                 store_half_row(which == 0 ? sT1 : sT2, j, hf, x, f);
             }
             fence_proxy_async();

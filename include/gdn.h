@@ -33,6 +33,11 @@
  *   [V] same page, 7.6.1 (config table): the value-head and key-head counts of
  *       the linear-attention layers are separate settings
  *       (linear_num_value_heads, linear_num_key_heads).
+ *   [U] same page, 7.6.2, the recurrence as that page writes it:
+ *         S_t = alpha_t S_{t-1} + k_t [beta_t (v_t - S_{t-1}^T k_t)]^T,
+ *       the memory read from the state BEFORE the decay. Calls that take
+ *       `undecayed` run this order when it is 1, [R]'s decay-first order
+ *       (the default) when it is 0; any other value is GDN_ERR_INVALID_ARG.
  *
  * Heads: H is the number of value heads (v, g, beta, the recurrent state and
  * the output have H heads); q and k have Hk heads, Hk dividing H, and value
@@ -138,7 +143,8 @@ GDN_API size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, i
  *                                        qk_l2norm, else identity)
  *   S <- exp(g_t) S;  delta = beta_t (v_t - S^T k^);  S <- S + k^ delta^T;
  *   o_t = S^T q^
- * and the final S is written to hT[n, h]. The kernels evaluate this in chunks
+ * (with undecayed = 1: delta = beta_t (v_t - S^T k^) from S before the
+ * decay, [U]) and the final S is written to hT[n, h]. The kernels evaluate this in chunks
  * of `chunk` tokens (cumulative decay, UT transform with a unit lower
  * triangular solve, inter-chunk state passing); the result equals the token
  * loop up to rounding.
@@ -170,7 +176,7 @@ GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gd
                          const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
                          int N, int64_t T_tot, int H, int Hk, int dk, int dv,
                          int64_t ld_q, int64_t ld_k, int64_t ld_v,
-                         float scale, int qk_l2norm, float eps, int chunk,
+                         float scale, int qk_l2norm, float eps, int undecayed, int chunk,
                          const float* h0, float* hT, void* o,
                          void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream);
 
@@ -200,7 +206,8 @@ GDN_API gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const voi
                                          const int32_t* cu_seqlens, const int32_t* cu_seqlens_host,
                                          int N, int64_t T_tot, int H, int Hk, int dk, int dv,
                                          int64_t ld_q, int64_t ld_k, int64_t ld_v,
-                                         float scale, int qk_l2norm, float eps, int chunk,
+                                         float scale, int qk_l2norm, float eps, int undecayed,
+                                         int chunk,
                                          const float* h0, float* hT, void* o, gdn_algo_t algo,
                                          void* stream);
 
@@ -215,8 +222,8 @@ GDN_API int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chu
 
 /*
  * One recurrent step for N independent sequences (one token each). [R], [P]
- * Same per-token rule as gdn_prefill; `state` is read and overwritten in
- * place with the post-token state.
+ * Same per-token rule as gdn_prefill (undecayed selects [U]'s order); `state`
+ * is read and overwritten in place with the post-token state.
  *
  *   q, k     [N, Hk, dk]      dtype   (Hk = 0: Hk = H; see "Heads" above)
  *   v        [N, H, dv]       dtype
@@ -228,7 +235,7 @@ GDN_API int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chu
 GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                              const float* g, const float* beta, float* state,
                              int N, int H, int Hk, int dk, int dv, float scale, int qk_l2norm,
-                             float eps, void* o, void* stream);
+                             float eps, int undecayed, void* o, void* stream);
 
 /*
  * The whole mixer for one decode token per sequence, in one kernel. [C] [R] [G] [P]
@@ -239,7 +246,8 @@ GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v
  *   y_c = w[c, K-1] * x[n, c] + sum_{j<K-1} w[c, j] * conv_state[n, c, j]
  * after which conv_state[n, c] shifts by one and takes x[n, c] as its newest
  * entry; then SiLU, the L2 norm of q and k (when qk_l2norm), and the recurrent
- * step of gdn_decode_step on state[n]. When z is given the output is gated:
+ * step of gdn_decode_step on state[n] (undecayed as there). When z is given
+ * the output is gated:
  *   o = y / sqrt(mean(y^2) + norm_eps) * norm_w * SiLU(z)   per (n, head),
  * norm_w applied as given (a zero-centred scale w is passed as 1 + w).
  *
@@ -259,8 +267,8 @@ GDN_API gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, vo
                                            gdn_dtype_t dtype, const float* g, const float* beta,
                                            float* state, const void* z, const float* norm_w,
                                            float norm_eps, int N, int H, int Hk, int dk, int dv,
-                                           float scale, int qk_l2norm, float eps, void* o,
-                                           void* stream);
+                                           float scale, int qk_l2norm, float eps, int undecayed,
+                                           void* o, void* stream);
 
 /*
  * Gated RMSNorm output over rows of dv features (a row = one (token, head)). [G]

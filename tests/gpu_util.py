@@ -37,7 +37,7 @@ def tol(kind: str) -> float:
     return TOL_BF16 if kind == "bf16" else TOL_F32
 
 
-def prefill_gpu(P, *, algo="auto", chunk=None, h0=None, give_host_cu=True):
+def prefill_gpu(P, *, algo="auto", chunk=None, h0=None, give_host_cu=True, undecayed=False):
     kind = P.dtype
     q, k, v = (dev_tensor(a, kind) for a in (P.q, P.k, P.v))
     g, beta = dev_tensor(P.g, "f32"), dev_tensor(P.beta, "f32")
@@ -46,16 +46,17 @@ def prefill_gpu(P, *, algo="auto", chunk=None, h0=None, give_host_cu=True):
     h0d = None if h0 is None else dev_tensor(h0, "f32")
     o, hT = gdn.prefill(q, k, v, g, beta, cu, initial_state=h0d, scale=P.scale,
                         qk_l2norm=P.qk_l2norm, eps=P.eps, chunk=chunk or P.chunk, algo=algo,
+                        undecayed=undecayed,
                         cu_seqlens_host=torch.from_numpy(P.cu_seqlens.astype(np.int32))
                         if give_host_cu else None)
     gdn.check_device_status(DEV)
     return host(o), host(hT)
 
 
-def prefill_oracle(P, h0=None):
+def prefill_oracle(P, h0=None, undecayed=False):
     h0 = P.h0 if h0 is None else h0
     return oracle.recurrence(P.q, P.k, P.v, P.g, P.beta, P.cu_seqlens, dtype=P.dtype, h0=h0,
-                             scale=P.scale, qk_l2norm=P.qk_l2norm, eps=P.eps)
+                             scale=P.scale, qk_l2norm=P.qk_l2norm, eps=P.eps, undecayed=undecayed)
 
 
 def oracle_unit(P, n: int, h: int):

@@ -64,7 +64,7 @@ FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails
 
 def _prefill(L, **kw):
     args = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, g=FAKE, beta=FAKE, cu=FAKE, cu_host=None, N=1,
-                T=64, H=2, Hk=0, dk=128, dv=128, ldq=0, ldk=0, ldv=0, scale=1.0, l2=1, eps=1e-6, chunk=64, h0=None, hT=None,
+                T=64, H=2, Hk=0, dk=128, dv=128, ldq=0, ldk=0, ldv=0, scale=1.0, l2=1, eps=1e-6, und=0, chunk=64, h0=None, hT=None,
                 o=FAKE, ws=FAKE, ws_bytes=1 << 20, algo=0, stream=None)
     args.update(kw)
     return L.gdn_prefill(*args.values())
@@ -80,6 +80,7 @@ def _prefill(L, **kw):
     # grouped value heads: Hk must divide H; dense strides follow Hk for q, k
     (dict(Hk=-1), 1), (dict(H=6, Hk=4), 1), (dict(H=4, Hk=2, ldq=255), 1),
     (dict(H=4, Hk=2, ldv=256), 1),
+    (dict(und=2), 1), (dict(und=-1), 1),     # the order flag is 0 or 1
 ])
 def test_prefill_rejects_bad_arguments(L, kw, expect):
     assert _prefill(L, **kw) == expect
@@ -114,7 +115,7 @@ def test_conv_rejects_bad_arguments(L, kw, expect):
 
 def _decode(L, **kw):
     args = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, g=FAKE, beta=FAKE, state=FAKE, N=4, H=2, Hk=0, dk=128,
-                dv=128, scale=1.0, l2=1, eps=1e-6, o=FAKE, stream=None)
+                dv=128, scale=1.0, l2=1, eps=1e-6, und=0, o=FAKE, stream=None)
     args.update(kw)
     return L.gdn_decode_step(*args.values())
 
@@ -122,7 +123,7 @@ def _decode(L, **kw):
 @pytest.mark.parametrize("kw,expect", [
     (dict(dt=2), 1), (dict(dk=8), 2), (dict(dv=130), 2), (dict(state=None), 1),
     (dict(state=ctypes.c_void_p((1 << 20) + 8)), 1), (dict(H=-1), 1),
-    (dict(Hk=-2), 1), (dict(H=4, Hk=3), 1), (dict(Hk=4), 1),
+    (dict(Hk=-2), 1), (dict(H=4, Hk=3), 1), (dict(Hk=4), 1), (dict(und=3), 1),
 ])
 def test_decode_rejects_bad_arguments(L, kw, expect):
     assert _decode(L, **kw) == expect
@@ -141,7 +142,7 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 
 def _layer_step(L, **kw):
     args = dict(x=FAKE, cw=FAKE, cs=FAKE, K=4, dt=1, g=FAKE, beta=FAKE, st=FAKE, z=None, nw=None,
-                neps=1e-6, N=2, H=16, Hk=0, dk=128, dv=128, scale=1.0, l2=1, eps=1e-6, o=FAKE,
+                neps=1e-6, N=2, H=16, Hk=0, dk=128, dv=128, scale=1.0, l2=1, eps=1e-6, und=0, o=FAKE,
                 stream=None)
     args.update(kw)
     return L.gdn_decode_layer_step(*args.values())
@@ -155,6 +156,7 @@ def _layer_step(L, **kw):
     (dict(cs=ctypes.c_void_p((1 << 20) + 2)), 1), (dict(eps=float("nan")), 1),
     (dict(Hk=3), 1), (dict(Hk=-1), 1),
     (dict(Hk=1), 2),                         # 16 value heads per q, k head: above the cluster limit
+    (dict(und=7), 1),
 ])
 def test_decode_layer_step_rejects_bad_arguments(L, kw, expect):
     assert _layer_step(L, **kw) == expect

@@ -160,6 +160,31 @@ def test_prefill_grouped_value_heads_from_fused_buffer(algo):
     assert np.array_equal(host(o), o_d) and np.array_equal(host(hT), h_d)
 
 
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("g_scale", [1.0, 4.0])
+def test_prefill_undecayed_read(algo, g_scale):
+    """The 7.6.2 order (memory read from the state before the decay): ragged
+    sequences with an initial state; g_scale 4 takes chunks past the factored-decay
+    range, so both epilogue paths run."""
+    P = gi.random_prefill(17, [1, 63, 64, 65, 0, 200, 130], H=3, dk=128, dv=128, with_h0=True,
+                          g_scale=g_scale)
+    o, hT = prefill_gpu(P, algo=algo, undecayed=True)
+    o_ref, h_ref = prefill_oracle(P, undecayed=True)
+    assert err(o, o_ref) <= TOL_BF16
+    assert err(hT, h_ref) <= TOL_BF16
+    o_std, _ = prefill_oracle(P)
+    assert err(o_std, o_ref) > 2 * TOL_BF16  # the two orders are told apart at this tolerance
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_prefill_undecayed_read_fp32(chunk):
+    P = gi.random_prefill(18, [100, 37, 1], H=2, dk=64, dv=48, dtype="f32", with_h0=True,
+                          chunk=chunk)
+    o, hT = prefill_gpu(P, undecayed=True)
+    o_ref, h_ref = prefill_oracle(P, undecayed=True)
+    assert err(o, o_ref) <= TOL_F32 and err(hT, h_ref) <= TOL_F32
+
+
 def test_chunk_sizes_agree():
     P = gi.random_prefill(4, [100, 37], H=2, dk=32, dv=32, dtype="f32", with_h0=True)
     outs = [prefill_gpu(P, chunk=c) for c in (16, 32, 64)]
@@ -257,6 +282,26 @@ def test_decode_step_grouped_value_heads(kind):
     o = gdn.decode_step(dev_tensor(q, kind), dev_tensor(k, kind), dev_tensor(v, kind),
                         dev_tensor(g, "f32"), dev_tensor(beta, "f32"), state)
     o_ref, s_ref = oracle.recurrence(q, k, v, g, beta, np.arange(N + 1), dtype=kind, h0=s0)
+    assert err(host(o), o_ref) <= tol(kind)
+    assert err(host(state), s_ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("kind", ["f32", "bf16"])
+def test_decode_step_undecayed_read(kind):
+    r = np.random.default_rng(10)
+    N, H, dk, dv = 5, 3, 128, 64
+    q, k = r.normal(size=(N, H, dk)).astype(np.float32), r.normal(size=(N, H, dk)).astype(np.float32)
+    v = r.normal(size=(N, H, dv)).astype(np.float32)
+    if kind == "bf16":
+        q, k, v = gi.to_bf16_bits(q), gi.to_bf16_bits(k), gi.to_bf16_bits(v)
+    g = -np.abs(r.normal(size=(N, H))).astype(np.float32)
+    beta = r.uniform(size=(N, H)).astype(np.float32)
+    s0 = r.normal(0, 0.1, size=(N, H, dk, dv)).astype(np.float32)
+    state = dev_tensor(s0, "f32")
+    o = gdn.decode_step(dev_tensor(q, kind), dev_tensor(k, kind), dev_tensor(v, kind),
+                        dev_tensor(g, "f32"), dev_tensor(beta, "f32"), state, undecayed=True)
+    o_ref, s_ref = oracle.recurrence(q, k, v, g, beta, np.arange(N + 1), dtype=kind, h0=s0,
+                                     undecayed=True)
     assert err(host(o), o_ref) <= tol(kind)
     assert err(host(state), s_ref) <= TOL_F32
 
@@ -419,6 +464,37 @@ def test_decode_layer_step_grouped_value_heads(kind, G):
     assert err(host(st_d), st_o) <= tol_
     assert np.array_equal(host(cs_d), (gi.bf16_bits_to_f32(cs_o) if kind == "bf16" else cs_o)
                           .astype(np.float32))
+
+
+@pytest.mark.parametrize("kind", ["bf16", "f32"])
+def test_decode_layer_step_undecayed_read(kind):
+    r = np.random.default_rng(45)
+    N, H, Hk, dk, dv, K = 4, 4, 2, 128, 128, 4
+    C = 2 * Hk * dk + H * dv
+    to = (lambda a: gi.to_bf16_bits(a.astype(np.float32))) if kind == "bf16" else (
+        lambda a: a.astype(np.float32))
+    cw, cs = to(r.normal(size=(C, K)) * 0.5), to(r.normal(size=(N, C, K - 1)))
+    st = (r.normal(size=(N, H, dk, dv)) * 0.1).astype(np.float32)
+    nw = (1.0 + 0.1 * r.normal(size=dv)).astype(np.float32)
+    cs_d, st_d = dev_tensor(cs, kind), torch.from_numpy(st).to(DEV)
+    cs_o, st_o = cs, st.astype(np.float64)
+    worst = 0.0
+    for t in range(3):
+        x, z = to(r.normal(size=(N, C))), to(r.normal(size=(N, H, dv)))
+        g = (-np.log1p(np.exp(r.normal(size=(N, H))))).astype(np.float32)
+        b = (1.0 / (1.0 + np.exp(-r.normal(size=(N, H))))).astype(np.float32)
+        o = gdn.decode_layer_step(dev_tensor(x, kind), dev_tensor(cw, kind), cs_d,
+                                  torch.from_numpy(g).to(DEV), torch.from_numpy(b).to(DEV), st_d,
+                                  H=H, Hk=Hk, dk=dk, dv=dv, z=dev_tensor(z, kind),
+                                  norm_w=torch.from_numpy(nw).to(DEV), undecayed=True)
+        o_ref, cs_n, st_o = oracle.decode_layer_step(x, cw, cs_o, g, b, st_o, dtype=kind, H=H,
+                                                     Hk=Hk, dk=dk, dv=dv, z=z, norm_w=nw,
+                                                     undecayed=True)
+        cs_o = to(cs_n) if kind == "bf16" else cs_n
+        worst = max(worst, err(host(o), o_ref))
+    gdn.check_device_status(DEV)
+    tol_ = TOL_BF16 if kind == "bf16" else TOL_F32
+    assert worst <= tol_ and err(host(st_d), st_o) <= tol_
 
 
 def test_decode_layer_step_equals_separate_kernels():

@@ -56,7 +56,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         hT = torch.empty_like(hT_ref)
         stream = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
         st = L.gdn_prefill_noalloc(_p(q), _p(k), _p(v), gdn.GDN_BF16, _p(g), _p(beta), _p(cu), None,
-                                   N, T, H, 0, dk, dv, 0, 0, 0, 1.0, 1, 1e-6, 64, _p(h0), _p(hT),
+                                   N, T, H, 0, dk, dv, 0, 0, 0, 1.0, 1, 1e-6, 0, 64, _p(h0), _p(hT),
                                    _p(o), 0, stream)
         assert st == 0, gdn.STATUS.get(st, st)
         gdn.check_device_status(DEV)
@@ -71,6 +71,6 @@ def test_noalloc_rejects_problems_larger_than_its_scratch():
     too_many = cap // 4  # the schedule needs 4 bytes per sequence plus a header
     fake = ctypes.c_void_p(1 << 20)
     st = L.gdn_prefill_noalloc(fake, fake, fake, gdn.GDN_BF16, fake, fake, fake, None, too_many,
-                               too_many, 1, 0, 128, 128, 0, 0, 0, 1.0, 1, 1e-6, 64, None, None, fake, 0,
+                               too_many, 1, 0, 128, 128, 0, 0, 0, 1.0, 1, 1e-6, 0, 64, None, None, fake, 0,
                                None)
     assert st == 3  # GDN_ERR_WORKSPACE, before anything is launched
