@@ -597,6 +597,83 @@ def bench_grouped(args, dist, pk):
     return {"prefill": pre, "decode_layer": dec}
 
 
+def bench_undecayed(args, dist, pk):
+    """The read-before-decay order (memory read from the state before the decay)
+    on the headline prefill workload (8 x 16384 tokens, 16 heads, d=128) and on
+    the decode workload (256 x 16 heads, 100 in-place steps)."""
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    P = gi.long_prefill(SEQS, SEQ_LEN, H, D)
+    T = P.T_tot
+    bf = lambda a: torch.from_numpy(a.view("int16")).to(dev).view(torch.bfloat16)
+    q, k, v = bf(P.q), bf(P.k), bf(P.v)
+    g, beta = torch.from_numpy(P.g).to(dev), torch.from_numpy(P.beta).to(dev)
+    cu = torch.from_numpy(P.cu_seqlens).to(dev)
+    del P
+    o = torch.empty_like(v)
+    hT = torch.empty((SEQS, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(SEQS, T, H, D, D, CHUNK), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, chunk=CHUNK,
+                    undecayed=True)
+
+    for _ in range(3):
+        step()
+    gdn.check_device_status(dev)
+    torch.cuda.synchronize()
+    reps = 5
+    total_ms, _ = timed(step, reps, stream)
+    ms = dist.max(total_ms) / reps
+    flops = T * H * FLOP_PER_TOKEN_HEAD
+    byts = T * H * BYTES_PER_TOKEN_HEAD + SEQS * H * STATE_BYTES
+    pre = {"value": T / (ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": ms,
+           "workload": f"long_prefill_{SEQS}x{SEQ_LEN}_h16_d128_bf16_undecayed",
+           "tc_roofline": {"achieved": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                           "peak": pk["bf16_tflops"],
+                           "frac": flops / (ms * 1e-3) / 1e12 / pk["bf16_tflops"]},
+           "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                        "algorithmic_bytes": byts},
+           "gpu_launches": 2 * reps}
+    del q, k, v, g, beta, o, hT
+    torch.cuda.empty_cache()
+
+    N, steps = 256, 100
+    state = torch.from_numpy(gi.decode_state(N, H, D)).to(dev)
+    ins = []
+    for s_ in range(8):
+        Dd = gi.decode_step(s_, N, H, D)
+        ins.append((bf(Dd.q), bf(Dd.k), bf(Dd.v), torch.from_numpy(Dd.g).to(dev),
+                    torch.from_numpy(Dd.beta).to(dev)))
+    od = torch.empty((N, H, D), dtype=torch.bfloat16, device=dev)
+    it = iter(range(10 ** 9))
+
+    def dstep():
+        qq, kk, vv, gg, bb = ins[next(it) % len(ins)]
+        gdn.decode_step(qq, kk, vv, gg, bb, state, out=od, undecayed=True)
+
+    for _ in range(5):
+        dstep()
+    torch.cuda.synchronize()
+    total_ms, _ = timed(dstep, steps, stream)
+    step_ms = dist.max(total_ms) / steps
+    bytes_step = N * H * (2 * STATE_BYTES + 4 * D * 2 + 8)
+    dec = {"value": N / (step_ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": step_ms,
+           "workload": f"decode_{N}x16_d128_{steps}steps_undecayed",
+           "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
+                        "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                        "algorithmic_bytes": bytes_step},
+           "gpu_launches": steps}
+    return {"prefill": pre, "decode": dec}
+
+
 def bench_gated_norm(args, dist, pk):
     """Gated RMSNorm output over the long-prefill output: 8 x 16384 tokens x 16
     heads, d_v = 128, bf16 (read o and z, write the gated output)."""
@@ -708,6 +785,7 @@ def run_ours(args, dist: Dist):
         extras["decode_layer"] = bench_decode_layer(args, dist, pk)
         extras["gated_rmsnorm"] = bench_gated_norm(args, dist, pk)
         extras["grouped"] = bench_grouped(args, dist, pk)
+        extras["undecayed"] = bench_undecayed(args, dist, pk)
     clocks.active = False
     clk = clocks.stop()
 
@@ -789,7 +867,7 @@ def main():
 
 ONLY = {"decode": bench_decode, "layer": bench_layer, "varlen": bench_varlen,
         "decode_layer": bench_decode_layer, "gated_rmsnorm": bench_gated_norm,
-        "grouped": bench_grouped}
+        "grouped": bench_grouped, "undecayed": bench_undecayed}
 
 if __name__ == "__main__":
     main()
