@@ -300,6 +300,10 @@ struct Smem {
     // [256,320) rq, [320,384) rk (written by the prep group)
 };
 
+// kUndecayed: each token reads the state before its own decay (row decay
+// gamma_{r-1} in A and W). A template parameter, so the default order's code is
+// not touched by the option.
+template <bool kUndecayed>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap map_q,
                   const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
@@ -438,7 +442,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
                 }
-                if (a.undecayed) {  // A's row decay then reaches back to gamma_{-1} = 0
+                if (kUndecayed) {  // A's row decay then reaches back to gamma_{-1} = 0
                     mx = fmaxf(mx, 0.f);
                     mn = fminf(mn, 0.f);
                 }
@@ -496,7 +500,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                     tmem_wait_ld();
                     // row decay: gamma_r, or for A rows with the read-before-decay
                     // order gamma_{r-1} (gamma_{-1} = 0)
-                    const float gr = (!is_p && a.undecayed) ? (r > 0 ? gam[r - 1] : 0.f) : gam[r];
+                    const float gr = (kUndecayed && !is_p) ? (r > 0 ? gam[r - 1] : 0.f) : gam[r];
                     const float fr = is_p ? rq[r] : bet[r] * rk[r];
                     const int lim = (is_p && rb == cb) ? r : 64;  // keep j <= lim
                     if (vec[65] != 0.f) {
@@ -628,7 +632,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 float x[32];
 #pragma unroll
                 for (int r = 0; r < 32; ++r) x[r] = sT[(32 * hf + r) * kLdA + j];
-                const float gj = a.undecayed ? (j > 0 ? gam[j - 1] : 0.f) : gam[j];
+                const float gj = kUndecayed ? (j > 0 ? gam[j - 1] : 0.f) : gam[j];
                 const float f = which == 0 ? bet[j] * expf(gj) * rk[j] : bet[j];
                 store_half_row(which == 0 ? sT1 : sT2, j, hf, x, f);
             }
@@ -997,7 +1001,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
         !make_map(&mv, a.v, a.H, a.T_tot, a.ld_v, true) ||
         !make_map(&mo, a.o, a.H, a.T_tot, (int64_t)a.H * kD, false))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kernel = a.undecayed ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemAlloc);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
@@ -1006,7 +1011,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sms ? units : sms);
     TcParams p{a};
-    prefill_tc_kernel<<<grid, kThreads, kSmemAlloc, s>>>(p, mq, mk, mv, mo);
+    kernel<<<grid, kThreads, kSmemAlloc, s>>>(p, mq, mk, mv, mo);
     return cudaGetLastError();
 }
 
