@@ -674,6 +674,53 @@ def bench_undecayed(args, dist, pk):
     return {"prefill": pre, "decode": dec}
 
 
+def bench_backward(args, dist, pk):
+    """Gradients of the recurrence (fp32 CUDA cores, token by token): 8 sequences x
+    4096 tokens, 16 heads, d=128, bf16 q/k/v, fp32 dO and dS_T."""
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    N, T1 = SEQS, 4096
+    P = gi.long_prefill(N, T1, H, D)
+    T = P.T_tot
+    bf = lambda a: torch.from_numpy(a.view("int16")).to(dev).view(torch.bfloat16)
+    q, k, v = bf(P.q), bf(P.k), bf(P.v)
+    g, beta = torch.from_numpy(P.g).to(dev), torch.from_numpy(P.beta).to(dev)
+    cu = torch.from_numpy(P.cu_seqlens).to(dev)
+    host_cu = torch.from_numpy(P.cu_seqlens)
+    del P
+    r = np.random.default_rng(9)
+    do = torch.from_numpy(r.standard_normal((T, H, D), dtype=np.float32)).to(dev)
+    dhT = torch.from_numpy(r.standard_normal((N, H, D, D), dtype=np.float32)).to(dev)
+    ws = torch.empty(gdn.lib().gdn_backward_workspace_size(N, T, H, D, D), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        gdn.backward(q, k, v, g, beta, cu, do, dhT=dhT, cu_seqlens_host=host_cu, workspace=ws)
+
+    for _ in range(3):
+        step()
+    gdn.check_device_status(dev)
+    torch.cuda.synchronize()
+    reps = 3
+    total_ms, _ = timed(step, reps, stream)
+    ms = dist.max(total_ms) / reps
+    # read q, k, v (bf16), g, beta, dO (fp32), dS_T; write dq, dk, dv (fp32), dg, dbeta, dh0
+    per_th = 3 * D * 2 + 8 + D * 4 + 3 * D * 4 + 8
+    byts = T * H * per_th + 2 * N * H * STATE_BYTES
+    return {"value": T / (ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": ms,
+            "workload": f"backward_{N}x{T1}_h16_d128_bf16_inputs_fp32_grads",
+            "roofline": {"bound": "hbm", "achieved": byts / (ms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": byts / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "algorithmic_bytes": byts,
+                         "note": "token-sequential fp32 kernel: bound by per-token barriers, "
+                                 "not by HBM"},
+            "gpu_launches": reps}
+
+
 def bench_gated_norm(args, dist, pk):
     """Gated RMSNorm output over the long-prefill output: 8 x 16384 tokens x 16
     heads, d_v = 128, bf16 (read o and z, write the gated output)."""
@@ -786,6 +833,7 @@ def run_ours(args, dist: Dist):
         extras["gated_rmsnorm"] = bench_gated_norm(args, dist, pk)
         extras["grouped"] = bench_grouped(args, dist, pk)
         extras["undecayed"] = bench_undecayed(args, dist, pk)
+        extras["backward"] = bench_backward(args, dist, pk)
     clocks.active = False
     clk = clocks.stop()
 
@@ -867,7 +915,7 @@ def main():
 
 ONLY = {"decode": bench_decode, "layer": bench_layer, "varlen": bench_varlen,
         "decode_layer": bench_decode_layer, "gated_rmsnorm": bench_gated_norm,
-        "grouped": bench_grouped, "undecayed": bench_undecayed}
+        "grouped": bench_grouped, "undecayed": bench_undecayed, "backward": bench_backward}
 
 if __name__ == "__main__":
     main()

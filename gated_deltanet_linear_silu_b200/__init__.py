@@ -80,6 +80,11 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill_noalloc_max_scratch.restype = sz
         L.gdn_prefill_selected_algo.argtypes = [i32, i32, i32, i32, i32]
         L.gdn_prefill_selected_algo.restype = i32
+        L.gdn_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+        L.gdn_backward_workspace_size.restype = sz
+        L.gdn_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                   f32, i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.gdn_backward.restype = i32
         L.gdn_version.argtypes = []
         L.gdn_version.restype = i32
         _lib = L
@@ -265,6 +270,41 @@ def decode_layer_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: Optiona
                                      float(eps), int(undecayed), _ptr(o), _stream(x.device))
     _check(st, "gdn_decode_layer_step")
     return o
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+             beta: torch.Tensor, cu_seqlens: torch.Tensor, do: torch.Tensor, *,
+             initial_state: Optional[torch.Tensor] = None, dhT: Optional[torch.Tensor] = None,
+             scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6,
+             cu_seqlens_host: Optional[torch.Tensor] = None, want_dh0: bool = True,
+             workspace: Optional[torch.Tensor] = None):
+    """Gradients of the recurrence for upstream gradients do [T, H, dv] (fp32)
+    and dhT [N, H, dk, dv] (fp32, optional). q, k [T, Hk, dk] and v [T, H, dv]
+    dense (bf16 or fp32). Returns (dq, dk, dv, dg, dbeta, dh0), fp32; dh0 is
+    None unless want_dh0."""
+    T, Hk, dk = q.shape
+    H, dv = v.shape[1], v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dkt = torch.empty((T, Hk, dk), **f32), torch.empty((T, Hk, dk), **f32)
+    dvt, dg, db = torch.empty((T, H, dv), **f32), torch.empty((T, H), **f32), torch.empty((T, H), **f32)
+    dh0 = torch.empty((N, H, dk, dv), **f32) if want_dh0 else None
+    ws_bytes = int(lib().gdn_backward_workspace_size(N, T, H, dk, dv))
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    _cuda(q, k, v, g, beta, cu_seqlens, do, initial_state, dhT, workspace)
+    host_cu = None
+    if cu_seqlens_host is not None:
+        host_cu = cu_seqlens_host.to(torch.int32).contiguous()
+    st = lib().gdn_backward(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+        None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
+        float(scale), int(qk_l2norm), float(eps), _ptr(initial_state), _ptr(do), _ptr(dhT),
+        _ptr(dq), _ptr(dkt), _ptr(dvt), _ptr(dg), _ptr(db), _ptr(dh0), _ptr(workspace),
+        workspace.numel(), _stream(dev))
+    _check(st, "gdn_backward")
+    return dq, dkt, dvt, dg, db, dh0
 
 
 def gated_rmsnorm(y: torch.Tensor, z: torch.Tensor, w: torch.Tensor, *, eps: float = 1e-6,

@@ -227,6 +227,47 @@ gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t gdn_backward_workspace_size(int N, int64_t T_tot, int H, int dk, int dv) {
+    if (N < 0 || T_tot < 0 || H <= 0 || dk <= 0 || dv <= 0) return 0;
+    const size_t b = gdn::backward_workspace_floats(N, T_tot, H, dk, dv) * sizeof(float);
+    return (b + 255) / 256 * 256 + 256;
+}
+
+gdn_status_t gdn_backward(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                          const float* g, const float* beta, const int32_t* cu_seqlens,
+                          const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
+                          int dk, int dv, float scale, int qk_l2norm, float eps, const float* h0,
+                          const float* dO, const float* dhT, float* dq, float* dk_out,
+                          float* dv_out, float* dg, float* dbeta, float* dh0, void* workspace,
+                          size_t ws_bytes, void* stream) {
+    if (Hk == 0) Hk = H;
+    if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0 || Hk < 0 || H % Hk != 0)
+        return GDN_ERR_INVALID_ARG;
+    if (N == 0 && T_tot > 0) return GDN_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (N > 0 && !cu_seqlens) return GDN_ERR_INVALID_ARG;
+    if (T_tot > 0 && (!q || !k || !v || !g || !beta || !dO || !dq || !dk_out || !dv_out || !dg ||
+                      !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(h0) || !aligned16(dhT) || !aligned16(dh0) || !aligned16(q) || !aligned16(k) ||
+        !aligned16(v))
+        return GDN_ERR_INVALID_ARG;
+    if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)N * H >= (int64_t)1 << 31 || T_tot >= ((int64_t)1 << 31)) return GDN_ERR_UNSUPPORTED;
+    if (gdn_status_t st = check_host_seqlens(cu_seqlens_host, N, T_tot)) return st;
+    if (N == 0) return GDN_OK;
+    const size_t need = gdn_backward_workspace_size(N, T_tot, H, dk, dv);
+    if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GDN_ERR_WORKSPACE;
+    const int64_t slots = 2 * (int64_t)N + (T_tot + gdn::kCk - 1) / gdn::kCk + 1;
+    float* ws = static_cast<float*>(workspace);
+    gdn::BackwardArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, Hk, dk, dv,
+                        scale, qk_l2norm, eps, h0, dO, dhT, dq, dk_out, dv_out, dg, dbeta, dh0,
+                        ws, ws + slots * H * (int64_t)dk * dv, slots, status_ptr()};
+    if (!a.status) return GDN_ERR_CUDA;
+    return from_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
+}
+
 gdn_status_t gdn_gated_rmsnorm(const void* y, const void* z, const float* w, gdn_dtype_t dtype,
                                int64_t rows, int dv, float eps, void* out, void* stream) {
     if (!dtype_ok(dtype) || rows < 0) return GDN_ERR_INVALID_ARG;

@@ -54,6 +54,39 @@ cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
 // thread-block cluster per group, 8 being the portable cluster size.
 constexpr int kMaxDecodeGroup = 8;
 
+// Backward of the recurrence (fp32, one CTA per (sequence, value head)).
+constexpr int kCk = 16;  // tokens between state checkpoints
+struct BackwardArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    int is_bf16;
+    const float* g;
+    const float* beta;
+    const int32_t* cu;
+    int N;
+    int64_t T_tot;
+    int H, Hk, dk, dv;
+    float scale;
+    int qk_l2norm;
+    float eps;
+    const float* h0;    // [N, H, dk, dv] or null
+    const float* dO;    // [T, H, dv]
+    const float* dhT;   // [N, H, dk, dv] or null
+    float* dq_out;      // [T, Hk, dk]
+    float* dk_out;      // [T, Hk, dk]
+    float* dv_out;      // [T, H, dv]
+    float* dg;          // [T, H]
+    float* dbeta;       // [T, H]
+    float* dh0;         // [N, H, dk, dv] or null
+    float* ws_ckpt;     // ck_slots x H checkpoints of dk x dv
+    float* ws_buf;      // N x H x kCk states of dk x dv
+    int64_t ck_slots;
+    int* status;
+};
+size_t backward_workspace_floats(int N, int64_t T_tot, int H, int dk, int dv);
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s);
+
 struct GatedNormArgs {
     const void* y;
     const void* z;

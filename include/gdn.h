@@ -13,6 +13,7 @@
  *                    from the conv state, SiLU, L2 norm, the recurrent step
  *                    and (optionally) the gated RMSNorm output, in one kernel.
  *   gdn_gated_rmsnorm  the gated RMSNorm output for prefill outputs.
+ *   gdn_backward     gradients of the recurrence (q, k, v, g, beta, h0).
  *
  * Sources (page title, section):
  *   [R] "Qwen3.5-MoE source walkthrough", 4.3 Qwen3_5MoeGatedDeltaNet: the
@@ -269,6 +270,45 @@ GDN_API gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, vo
                                            float norm_eps, int N, int H, int Hk, int dk, int dv,
                                            float scale, int qk_l2norm, float eps, int undecayed,
                                            void* o, void* stream);
+
+/*
+ * Bytes of device workspace gdn_backward needs (a multiple of 256): state
+ * checkpoints every 16 tokens plus 16 recomputed states per (sequence, head),
+ * 4 * dk * dv * (H * (2N + ceil(T_tot / 16) + 1) + 16 N H) bytes, rounded up.
+ */
+GDN_API size_t gdn_backward_workspace_size(int N, int64_t T_tot, int H, int dk, int dv);
+
+/*
+ * Gradients of the recurrence gdn_prefill computes (decay-first order, [R]),
+ * for upstream gradients dO of the output and dhT of the final state. fp32
+ * arithmetic on CUDA cores, one CTA per (sequence, value head), token by
+ * token: a forward pass stores the state every 16 tokens in the workspace,
+ * then each block of 16 tokens, last first, recomputes its states and is
+ * swept in reverse. Gradients flow through the L2 norms (when qk_l2norm) and
+ * the query scale; the q, k gradients of a q/k head shared by several value
+ * heads are the sums over them.
+ *
+ *   q, k           [T_tot, Hk, dk]  dtype   (dense; Hk = 0: Hk = H)
+ *   v              [T_tot, H, dv]   dtype
+ *   g, beta        [T_tot, H]       fp32
+ *   cu_seqlens     [N+1] int32 device (cu_seqlens_host: nullable host copy)
+ *   h0             [N, H, dk, dv]   fp32    nullable initial state
+ *   dO             [T_tot, H, dv]   fp32    gradient of the output
+ *   dhT            [N, H, dk, dv]   fp32    nullable gradient of the final state
+ *   dq, dk         [T_tot, Hk, dk]  fp32    out
+ *   dv             [T_tot, H, dv]   fp32    out
+ *   dg, dbeta      [T_tot, H]       fp32    out
+ *   dh0            [N, H, dk, dv]   fp32    nullable out
+ *   workspace      ws_bytes >= gdn_backward_workspace_size(...), 256-byte aligned
+ * Supported: dk, dv in {16, 32, ..., 128}. Outputs must not overlap inputs.
+ */
+GDN_API gdn_status_t gdn_backward(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                                  const float* g, const float* beta, const int32_t* cu_seqlens,
+                                  const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H,
+                                  int Hk, int dk, int dv, float scale, int qk_l2norm, float eps,
+                                  const float* h0, const float* dO, const float* dhT, float* dq,
+                                  float* dk_out, float* dv_out, float* dg, float* dbeta,
+                                  float* dh0, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Gated RMSNorm output over rows of dv features (a row = one (token, head)). [G]

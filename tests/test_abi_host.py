@@ -168,6 +168,36 @@ def test_decode_layer_step_k1_needs_no_conv_state_and_empty_is_noop(L):
     assert _layer_step(L, K=1, cs=None, st=None) == 1
 
 
+def _bwd(L, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, dt=1, g=FAKE, beta=FAKE, cu=FAKE, cu_host=None, N=1, T=64,
+                H=2, Hk=0, dk=128, dv=128, scale=1.0, l2=1, eps=1e-6, h0=None, dO=FAKE, dhT=None,
+                dq=FAKE, dkk=FAKE, dvv=FAKE, dg=FAKE, db=FAKE, dh0=None, ws=FAKE, ws_bytes=1 << 20,
+                stream=None)
+    args.update(kw)
+    return L.gdn_backward(*args.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=4), 1), (dict(N=-1), 1), (dict(H=0), 1), (dict(H=6, Hk=4), 1), (dict(Hk=-1), 1),
+    (dict(N=0, T=3), 1), (dict(dk=40), 2), (dict(dv=144), 2), (dict(cu=None), 1),
+    (dict(dO=None), 1), (dict(dq=None), 1), (dict(db=None), 1),
+    (dict(h0=ctypes.c_void_p((1 << 20) + 4)), 1), (dict(eps=float("nan")), 1),
+    (dict(ws=None), 3), (dict(ws_bytes=1024), 3), (dict(ws=ctypes.c_void_p((1 << 20) + 64)), 3),
+])
+def test_backward_rejects_bad_arguments(L, kw, expect):
+    assert _bwd(L, **kw) == expect
+
+
+def test_backward_workspace_size_formula(L):
+    # checkpoints every 16 tokens + 16 recomputed states per (sequence, head)
+    N, T, H, dk, dv = 3, 100, 2, 64, 32
+    floats = ((2 * N + (T + 15) // 16 + 1) * H + N * H * 16) * dk * dv
+    got = L.gdn_backward_workspace_size(N, T, H, dk, dv)
+    assert got % 256 == 0 and floats * 4 <= got <= floats * 4 + 512
+    assert _bwd(L, N=0, T=0, q=None, k=None, v=None, dO=None, dq=None, dkk=None, dvv=None,
+                dg=None, db=None, cu=None) == 0  # empty batch: nothing to do
+
+
 def _gnorm(L, **kw):
     args = dict(y=FAKE, z=FAKE, w=FAKE, dt=1, rows=10, dv=128, eps=1e-6, out=FAKE, stream=None)
     args.update(kw)

@@ -528,6 +528,59 @@ def test_decode_layer_step_equals_separate_kernels():
 
 
 # ----------------------------------------------------------------------------
+# backward
+# ----------------------------------------------------------------------------
+
+def _backward_case(P, seed, with_dhT):
+    from oracle import backward as ob
+    r = np.random.default_rng(seed)
+    T, N = P.T_tot, P.N
+    do = r.normal(size=(T, P.H, P.dv)).astype(np.float32)
+    dhT = r.normal(size=(N, P.H, P.dk, P.dv)).astype(np.float32) if with_dhT else None
+    dec = (lambda a: gi.bf16_bits_to_f32(a).astype(np.float64)) if P.dtype == "bf16" else (
+        lambda a: np.asarray(a, np.float64))
+    ref = ob.recurrence_backward(dec(P.q), dec(P.k), dec(P.v), P.g, P.beta, P.cu_seqlens, do, dhT,
+                                 h0=P.h0, scale=P.scale, qk_l2norm=P.qk_l2norm, eps=P.eps)
+    got = gdn.backward(dev_tensor(P.q, P.dtype), dev_tensor(P.k, P.dtype), dev_tensor(P.v, P.dtype),
+                       dev_tensor(P.g, "f32"), dev_tensor(P.beta, "f32"),
+                       torch.from_numpy(P.cu_seqlens.astype(np.int32)).to(DEV),
+                       dev_tensor(do, "f32"),
+                       initial_state=None if P.h0 is None else dev_tensor(P.h0, "f32"),
+                       dhT=None if dhT is None else dev_tensor(dhT, "f32"), scale=P.scale,
+                       qk_l2norm=P.qk_l2norm, eps=P.eps,
+                       cu_seqlens_host=torch.from_numpy(P.cu_seqlens.astype(np.int32)))
+    gdn.check_device_status(DEV)
+    return [host(x) for x in got], ref
+
+
+@pytest.mark.parametrize("kind,H,Hk,dk,dv,with_h0,with_dhT", [
+    ("bf16", 2, 2, 128, 128, True, True),
+    ("f32", 4, 2, 64, 48, False, True),
+    ("f32", 3, 3, 32, 128, True, False),
+])
+def test_backward_matches_oracle(kind, H, Hk, dk, dv, with_h0, with_dhT):
+    """Gradients of q, k, v, g, beta and h0 against autograd of the fp64 oracle:
+    ragged sequences (an empty one, one shorter than a checkpoint block, one spanning
+    several blocks), grouped heads, with and without initial state and final-state
+    gradient. The inputs are the same values on both sides; the kernel computes in fp32."""
+    P = gi.random_prefill(19, [40, 0, 7, 35], H=H, Hk=Hk, dk=dk, dv=dv, dtype=kind,
+                          with_h0=with_h0, scale=0.9)
+    got, ref = _backward_case(P, 20, with_dhT)
+    for name, a_, b_ in zip(["dq", "dk", "dv", "dg", "dbeta", "dh0"], got, ref):
+        assert err(a_, b_) <= TOL_F32, name
+
+
+def test_backward_without_l2norm():
+    P = gi.random_prefill(21, [33, 18], H=2, dk=16, dv=16, dtype="f32", with_h0=True,
+                          qk_l2norm=False)
+    P.q *= 0.25
+    P.k *= 0.25
+    got, ref = _backward_case(P, 22, True)
+    for name, a_, b_ in zip(["dq", "dk", "dv", "dg", "dbeta", "dh0"], got, ref):
+        assert err(a_, b_) <= TOL_F32, name
+
+
+# ----------------------------------------------------------------------------
 # full-size workloads
 # ----------------------------------------------------------------------------
 
