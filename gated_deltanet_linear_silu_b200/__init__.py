@@ -118,6 +118,19 @@ def _cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _check_heads(q, k, v, g, beta):
+    """Shapes the C ABI cannot see: q, k [T, Hk, dk] alike, v [T, H, dv],
+    g, beta [T, H], H a multiple of Hk."""
+    T, Hk, dk = q.shape
+    if tuple(k.shape) != (T, Hk, dk) or v.dim() != 3 or v.shape[0] != T:
+        raise ValueError("q and k must be [T, Hk, dk] and v [T, H, dv]")
+    H = v.shape[1]
+    if H % Hk != 0:
+        raise ValueError(f"{H} value heads cannot share {Hk} q/k heads evenly")
+    if tuple(g.shape) != (T, H) or tuple(beta.shape) != (T, H):
+        raise ValueError("g and beta must be [T, H]")
+
+
 def _token_stride(t: torch.Tensor) -> int:
     """Elements between consecutive tokens of a [T, H, d] tensor whose rows
     may be views into a wider fused buffer (each row itself dense)."""
@@ -171,6 +184,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     int32 [N+1] (device). Returns (o, hT); final_state may be initial_state
     itself for an in-place update. undecayed=True reads each token's memory
     from the state before its decay (the 7.6.2 order)."""
+    _check_heads(q, k, v, g, beta)
     T, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
     N = cu_seqlens.shape[0] - 1
@@ -205,6 +219,7 @@ def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
     """gdn_prefill_noalloc: prefill with the library's fixed scratch array
     instead of a workspace; the caller passes every output buffer, so nothing
     is allocated."""
+    _check_heads(q, k, v, g, beta)
     T, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
     N = cu_seqlens.shape[0] - 1
@@ -234,6 +249,7 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
                 undecayed: bool = False) -> torch.Tensor:
     """One recurrent token per sequence. q,k [N,Hk,dk], v [N,H,dv], g,beta
     [N,H] fp32, state [N,H,dk,dv] fp32 updated in place. Returns o [N,H,dv]."""
+    _check_heads(q, k, v, g, beta)
     N, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
     o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device) if out is None else out
@@ -282,6 +298,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     and dhT [N, H, dk, dv] (fp32, optional). q, k [T, Hk, dk] and v [T, H, dv]
     dense (bf16 or fp32). Returns (dq, dk, dv, dg, dbeta, dh0), fp32; dh0 is
     None unless want_dh0."""
+    _check_heads(q, k, v, g, beta)
     T, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
     N = cu_seqlens.shape[0] - 1

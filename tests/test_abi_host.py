@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import gated_deltanet_linear_silu_b200 as gdn
 from gated_deltanet_linear_silu_b200 import build as gbuild
@@ -131,6 +132,21 @@ def test_decode_rejects_bad_arguments(L, kw, expect):
 
 def test_decode_empty_batch_is_noop(L):
     assert _decode(L, N=0, q=None, k=None, v=None, state=None, o=None) == 0
+
+
+@pytest.mark.parametrize("shapes", [
+    ((8, 2, 16), (8, 1, 16), (8, 2, 16), (8, 2)),   # k unlike q
+    ((8, 2, 16), (8, 2, 16), (8, 3, 16), (8, 3)),   # 3 value heads on 2 q/k heads
+    ((8, 2, 16), (8, 2, 16), (7, 2, 16), (8, 2)),   # v has another token count
+    ((8, 2, 16), (8, 2, 16), (8, 4, 16), (8, 2)),   # gates not per value head
+])
+def test_binding_rejects_head_shapes_the_abi_cannot_see(shapes):
+    q, k, v, gg = (torch.zeros(s_) for s_ in shapes)
+    cu = torch.tensor([0, 8], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        gdn.prefill(q, k, v, gg, gg, cu)
+    with pytest.raises(ValueError):
+        gdn.backward(q, k, v, gg, gg, cu, torch.zeros(8, v.shape[1], 16))
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
