@@ -682,7 +682,7 @@ def bench_backward(args, dist, pk):
     import gated_deltanet_linear_silu_b200 as gdn
     import gdn_inputs as gi
     dev = torch.device("cuda", dist.local)
-    N, T1 = SEQS, 4096
+    N, T1 = SEQS, min(4096, SEQ_LEN)  # --seq-len below 4096 gives a smaller profiling case
     P = gi.long_prefill(N, T1, H, D)
     T = P.T_tot
     bf = lambda a: torch.from_numpy(a.view("int16")).to(dev).view(torch.bfloat16)

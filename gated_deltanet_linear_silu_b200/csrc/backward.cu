@@ -51,7 +51,8 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
     float* dbt = dmm + dv;       // [dv] ddelta (v - m)
     float* red = dbt + dv;       // [RG][dv]
     float* redr = red + RG * dv; // [dk][cols4]
-    float* scal = redr + dk * cols4;  // [16]: a, beta, |q|, |k|, delta.do, k^.dk^, q~.dq~, <dS', Sp>
+    float* scal = redr + dk * cols4;  // [16]: a, beta, |q|, |k|, delta.do, k^.dk^, q~.dq~, <dS', Sp>,
+                                      //       g, beta as loaded
 
     const int64_t start = a.cu[n], end = a.cu[n + 1];
     const int64_t ck_base = 2 * (int64_t)n + (start + kCk - 1) / kCk;  // first checkpoint slot
@@ -76,6 +77,10 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
     // Token t's k^ (and q~, do when `full`), v, a, beta into shared memory.
     auto load_token = [&](int64_t t, bool full) {
         __syncthreads();  // the previous token's values are no longer read
+        if (tid == 0) {  // the gates travel with the vectors (one round trip per token)
+            scal[8] = a.g[t * H + h];
+            scal[9] = a.beta[t * H + h];
+        }
         for (int i = tid; i < dk; i += blockDim.x) {
             kh[i] = Elem<T>::load(k, (t * Hk + hk) * dk + i);
             if (full) qn[i] = Elem<T>::load(q, (t * Hk + hk) * dk + i);
@@ -94,8 +99,8 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
             sk = warp_sum(sk);
             sq = warp_sum(sq);
             if (lane == 0) {
-                scal[0] = expf(a.g[t * H + h]);
-                scal[1] = a.beta[t * H + h];
+                scal[0] = expf(scal[8]);
+                scal[1] = scal[9];
                 scal[2] = a.qk_l2norm ? sqrtf(sq + a.eps) : 1.f;
                 scal[3] = a.qk_l2norm ? sqrtf(sk + a.eps) : 1.f;
             }
