@@ -26,6 +26,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
+ABI_VERSION = 200  # gdn_version() of the C ABI these argument lists describe
 
 GDN_F32, GDN_BF16 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tensor": 2}
@@ -87,6 +88,9 @@ def lib() -> ctypes.CDLL:
         L.gdn_backward.restype = i32
         L.gdn_version.argtypes = []
         L.gdn_version.restype = i32
+        if L.gdn_version() != ABI_VERSION:  # argument lists differ between versions
+            raise RuntimeError(f"{LIB_PATH} has ABI {L.gdn_version()}, this binding needs "
+                               f"{ABI_VERSION}: rebuild with `python -m gated_deltanet_linear_silu_b200.build`")
         _lib = L
     return _lib
 

@@ -51,7 +51,7 @@ gdn_status_t check_host_seqlens(const int32_t* cu, int N, int64_t T_tot) {
 
 extern "C" {
 
-int gdn_version(void) { return 100; }  // 0.1.0
+int gdn_version(void) { return 200; }  // 0.2.0: Hk, undecayed, gdn_backward
 
 const char* gdn_status_string(gdn_status_t s) {
     switch (s) {

@@ -333,7 +333,9 @@ GDN_API const char* gdn_status_string(gdn_status_t status);
  */
 GDN_API gdn_status_t gdn_check_device_status(void* stream);
 
-/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH (0.2.0: q/k head count Hk,
+ * the `undecayed` order, gdn_backward). Argument lists change between minor
+ * versions; a binding checks the version before calling anything else. */
 GDN_API int gdn_version(void);
 
 #ifdef __cplusplus
