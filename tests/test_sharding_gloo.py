@@ -20,19 +20,19 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _problem():
+def _problem(Hk=2):
     import gdn_inputs as gi
-    return gi.random_prefill(41, [50, 3, 0, 120, 77, 9, 64], H=2, dk=8, dv=8, dtype="f32",
+    return gi.random_prefill(41, [50, 3, 0, 120, 77, 9, 64], H=2, Hk=Hk, dk=8, dv=8, dtype="f32",
                              with_h0=True)
 
 
-def _rank_main(rank, world, port, q):
+def _rank_main(rank, world, port, q, Hk=2):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         import oracle
-        P = _problem()
+        P = _problem(Hk)
         lens = np.diff(P.cu_seqlens)
         mine = assign_sequences(lens, world)[rank]
         tok, cu = shard_tokens(P.cu_seqlens, mine)
@@ -46,20 +46,21 @@ def _rank_main(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_sequence_sharding_matches_unsharded():
+@pytest.mark.parametrize("Hk", [2, 1], ids=["plain", "grouped_heads"])
+def test_sequence_sharding_matches_unsharded(Hk):
     import oracle
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, Hk)) for r in range(world)]
     for p in procs:
         p.start()
     payload = q.get(timeout=120)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    P = _problem()
+    P = _problem(Hk)
     o_ref, h_ref = oracle.recurrence(P.q, P.k, P.v, P.g, P.beta, P.cu_seqlens, dtype=P.dtype,
                                      h0=P.h0, threads=1)
     o = np.full_like(o_ref, np.nan)
