@@ -1,7 +1,8 @@
 """Pins for the oracle's gradients (oracle/backward.py): its torch forward is
 checked against the C oracle's token loop, and its gradients against central
 finite differences of that forward (every input element of a tiny problem) and
-against the closed form of the beta = 0 case."""
+against the closed form of the beta = 0 case; the chunk-form gradient evaluator
+is checked against those gradients."""
 import numpy as np
 import pytest
 
@@ -90,3 +91,30 @@ def test_beta0_closed_form_gradients():
     ref_dg = np.array([contrib[t:].sum() + final for t in range(T)])
     assert np.abs(dg[:, 0] - ref_dg).max() < 1e-12
     assert np.abs(dk_).max() < 1e-15  # k enters only through beta-weighted terms
+
+
+@pytest.mark.parametrize("lens,H,Hk,l2,chunk,g_scale", [
+    ([37, 0, 9, 70], 2, 1, True, 16, 0.5),   # ragged, empty, grouped heads
+    ([33], 1, 1, False, 4, 0.2),              # no L2 norm
+    ([20, 65], 2, 2, True, 64, 3.0),          # strong decay across a full chunk
+    ([19], 1, 1, True, 1, 1.0),               # chunk of one token
+])
+def test_chunked_backward_equals_autograd(lens, H, Hk, l2, chunk, g_scale):
+    # the chunk-level gradient algebra (what a tensor-core backward evaluates)
+    # against autograd of the token loop
+    r = _rng(30 + chunk)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T, N, dk, dv = int(cu[-1]), len(lens), 6, 5
+    q, k = r.normal(size=(T, Hk, dk)), r.normal(size=(T, Hk, dk))
+    if not l2:
+        q, k = 0.3 * q, 0.3 * k
+    v = r.normal(size=(T, H, dv))
+    g = -g_scale * np.abs(r.normal(size=(T, H)))
+    beta = r.uniform(size=(T, H))
+    h0, dhT = r.normal(size=(N, H, dk, dv)), r.normal(size=(N, H, dk, dv))
+    do = r.normal(size=(T, H, dv))
+    kw = dict(h0=h0, scale=0.8, qk_l2norm=l2)
+    ref = ob.recurrence_backward(q, k, v, g, beta, cu, do, dhT, **kw)
+    got = ob.chunked_backward(q, k, v, g, beta, cu, do, dhT, chunk=chunk, **kw)
+    for name, a_, b_ in zip(["dq", "dk", "dv", "dg", "dbeta", "dh0"], got, ref):
+        assert np.abs(a_ - b_).max() <= 1e-12 * max(np.abs(b_).max(), 1.0), name
