@@ -182,8 +182,8 @@ GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gd
                          void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream);
 
 /*
- * gdn_prefill without a caller-supplied workspace. There is no counterpart of
- * this call in the paper: it exists for callers that cannot allocate device
+ * gdn_prefill without a caller-supplied workspace. The sources describe no
+ * counterpart of this call: it exists for callers that cannot allocate device
  * memory where they run the mixer -- a runtime whose memory planner reserved
  * the whole device arena at start-up, or a serving loop that must not call
  * cudaMalloc/cudaFree (which can synchronise the device) once it is running.
