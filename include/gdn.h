@@ -1,7 +1,8 @@
 /*
  * gdn.h -- C ABI of libgdn.so: the Gated DeltaNet token mixer on NVIDIA B200
- * (sm_100a). Three operations, as the Qwen3.5 linear-attention layer uses
- * them:
+ * (sm_100a). The conv stage, the chunked prefill and the recurrent decode
+ * step as the Qwen3.5 linear-attention layer uses them, plus the fused decode
+ * step of the whole mixer, the gated output and the gradients:
  *
  *   gdn_conv_silu    causal depthwise conv1d + SiLU over the fused q/k/v
  *                    channels, optional per-head L2 norm of q and k, with a
