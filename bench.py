@@ -872,9 +872,43 @@ def run_ours(args, dist: Dist):
     }
     if cpu:
         line["cpu_baseline"] = cpu
-    line.update(extras)
+    # Details first, the headline keys and a compact summary of every workload
+    # last: readers that keep only the end of the output still see all numbers.
+    out = dict(extras)
+    out.update(line)
+    out["summary"] = summarize(line, extras)
     if dist.rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(out), flush=True)
+
+
+def summarize(line, extras):
+    """One short object: per workload its time and its roofline fraction(s)."""
+    def r(x, n=4):
+        return None if not isinstance(x, (int, float)) else round(float(x), n)
+
+    def obj(d, t_key="ms_per_step"):
+        o = {"ms": r(d.get(t_key, d.get("ms")))}
+        if "roofline" in d:
+            o["hbm"] = r(d["roofline"]["frac"], 3)
+        if "tc_roofline" in d:
+            o["tc"] = r(d["tc_roofline"]["frac"], 3)
+        if "conv" in d:
+            o["conv_ms"] = r(d["conv"]["ms"])
+            o["conv_hbm"] = r(d["conv"]["roofline"]["frac"], 3)
+        return o
+
+    s = {"prefill": {"ms": r(line["ms_per_step"]), "hbm": r(line["roofline"]["frac"], 3),
+                     "tc": r(line["tc_roofline"]["frac"], 3)}}
+    for name in ("decode", "decode_layer", "layer", "varlen", "gated_rmsnorm", "backward"):
+        if name in extras:
+            s[name] = obj(extras[name])
+    if "decode" in extras and isinstance(extras["decode"].get("ms_per_step_graph"), float):
+        s["decode"]["ms_graph"] = r(extras["decode"]["ms_per_step_graph"])
+    if "grouped" in extras:
+        s["grouped"] = {k: obj(v) for k, v in extras["grouped"].items()}
+    if "undecayed" in extras:
+        s["undecayed"] = {k: obj(v) for k, v in extras["undecayed"].items()}
+    return s
 
 
 def main():

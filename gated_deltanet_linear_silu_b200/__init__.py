@@ -26,7 +26,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
-ABI_VERSION = 200  # gdn_version() of the C ABI these argument lists describe
+ABI_VERSION = 201  # gdn_version() of the C ABI these argument lists describe
 
 GDN_F32, GDN_BF16 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tensor": 2}
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
                                    f32, i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_backward.restype = i32
+        L.gdn_set_wait_limit_ns.argtypes = [i64]
+        L.gdn_set_wait_limit_ns.restype = None
         L.gdn_version.argtypes = []
         L.gdn_version.restype = i32
         if L.gdn_version() != ABI_VERSION:  # argument lists differ between versions
@@ -101,6 +103,12 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def _stream(dev: torch.device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _on(dev: torch.device):
+    """The C ABI works on the current device (its status word and the no-alloc
+    scratch array are per device): make the tensors' device current."""
+    return torch.cuda.device(dev)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -164,9 +172,10 @@ def conv_silu(x: torch.Tensor, w: torch.Tensor, cu_seqlens: torch.Tensor, *,
     if st_out is None and return_state:
         st_out = torch.empty((N, C, K - 1), dtype=x.dtype, device=x.device)
     _cuda(x, w, cu_seqlens, conv_state, st_out, y)
-    st = lib().gdn_conv_silu(_ptr(x), _dtype_code(x), _ptr(w), _ptr(cu_seqlens), N, T, C, K,
-                             _ptr(conv_state), _ptr(st_out), int(qk_l2norm), int(n_qk_channels),
-                             int(head_dim), float(eps), _ptr(y), _stream(x.device))
+    with _on(x.device):
+        st = lib().gdn_conv_silu(_ptr(x), _dtype_code(x), _ptr(w), _ptr(cu_seqlens), N, T, C, K,
+                                 _ptr(conv_state), _ptr(st_out), int(qk_l2norm), int(n_qk_channels),
+                                 int(head_dim), float(eps), _ptr(y), _stream(x.device))
     _check(st, "gdn_conv_silu")
     return y, st_out
 
@@ -204,12 +213,13 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     host_cu = None
     if cu_seqlens_host is not None:
         host_cu = cu_seqlens_host.to(torch.int32).contiguous()
-    st = lib().gdn_prefill(
-        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
-        None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
-        ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(undecayed), int(chunk),
-        _ptr(initial_state), _ptr(hT),
-        _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
+    with _on(q.device):
+        st = lib().gdn_prefill(
+            _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+            None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
+            ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(undecayed), int(chunk),
+            _ptr(initial_state), _ptr(hT),
+            _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill")
     return o, hT
 
@@ -229,11 +239,12 @@ def prefill_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.
     N = cu_seqlens.shape[0] - 1
     ld = [_token_stride(t) for t in (q, k, v)]
     _cuda(g, beta, cu_seqlens, initial_state, final_state, out)
-    st = lib().gdn_prefill_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens), None,
-        N, T, H, Hk, dk, dv, ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps),
-        int(undecayed), int(chunk),
-        _ptr(initial_state), _ptr(final_state), _ptr(out), ALGOS[algo], _stream(q.device))
+    with _on(q.device):
+        st = lib().gdn_prefill_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens), None,
+            N, T, H, Hk, dk, dv, ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps),
+            int(undecayed), int(chunk),
+            _ptr(initial_state), _ptr(final_state), _ptr(out), ALGOS[algo], _stream(q.device))
     _check(st, "gdn_prefill_noalloc")
 
 
@@ -258,9 +269,10 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     H, dv = v.shape[1], v.shape[2]
     o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device) if out is None else out
     _cuda(q, k, v, g, beta, state, o)
-    st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta),
-                               _ptr(state), N, H, Hk, dk, dv, float(scale), int(qk_l2norm), float(eps),
-                               int(undecayed), _ptr(o), _stream(q.device))
+    with _on(q.device):
+        st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta),
+                                   _ptr(state), N, H, Hk, dk, dv, float(scale), int(qk_l2norm), float(eps),
+                                   int(undecayed), _ptr(o), _stream(q.device))
     _check(st, "gdn_decode_step")
     return o
 
@@ -284,10 +296,11 @@ def decode_layer_step(x: torch.Tensor, conv_w: torch.Tensor, conv_state: Optiona
         raise ValueError(f"x has {C} channels; expected 2*Hk*dk + H*dv")
     o = torch.empty((N, H, dv), dtype=x.dtype, device=x.device) if out is None else out
     _cuda(x, conv_w, conv_state, g, beta, state, z, norm_w, o)
-    st = lib().gdn_decode_layer_step(_ptr(x), _ptr(conv_w), _ptr(conv_state), K, _dtype_code(x),
-                                     _ptr(g), _ptr(beta), _ptr(state), _ptr(z), _ptr(norm_w),
-                                     float(norm_eps), N, H, Hk, dk, dv, float(scale), int(qk_l2norm),
-                                     float(eps), int(undecayed), _ptr(o), _stream(x.device))
+    with _on(x.device):
+        st = lib().gdn_decode_layer_step(_ptr(x), _ptr(conv_w), _ptr(conv_state), K, _dtype_code(x),
+                                         _ptr(g), _ptr(beta), _ptr(state), _ptr(z), _ptr(norm_w),
+                                         float(norm_eps), N, H, Hk, dk, dv, float(scale), int(qk_l2norm),
+                                         float(eps), int(undecayed), _ptr(o), _stream(x.device))
     _check(st, "gdn_decode_layer_step")
     return o
 
@@ -318,12 +331,13 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     host_cu = None
     if cu_seqlens_host is not None:
         host_cu = cu_seqlens_host.to(torch.int32).contiguous()
-    st = lib().gdn_backward(
-        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
-        None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
-        float(scale), int(qk_l2norm), float(eps), _ptr(initial_state), _ptr(do), _ptr(dhT),
-        _ptr(dq), _ptr(dkt), _ptr(dvt), _ptr(dg), _ptr(db), _ptr(dh0), _ptr(workspace),
-        workspace.numel(), _stream(dev))
+    with _on(dev):
+        st = lib().gdn_backward(
+            _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+            None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
+            float(scale), int(qk_l2norm), float(eps), _ptr(initial_state), _ptr(do), _ptr(dhT),
+            _ptr(dq), _ptr(dkt), _ptr(dvt), _ptr(dg), _ptr(db), _ptr(dh0), _ptr(workspace),
+            workspace.numel(), _stream(dev))
     _check(st, "gdn_backward")
     return dq, dkt, dvt, dg, db, dh0
 
@@ -335,16 +349,24 @@ def gated_rmsnorm(y: torch.Tensor, z: torch.Tensor, w: torch.Tensor, *, eps: flo
     dv = y.shape[-1]
     o = torch.empty_like(y) if out is None else out
     _cuda(y, z, w, o)
-    st = lib().gdn_gated_rmsnorm(_ptr(y), _ptr(z), _ptr(w), _dtype_code(y), y.numel() // dv, dv,
-                                 float(eps), _ptr(o), _stream(y.device))
+    with _on(y.device):
+        st = lib().gdn_gated_rmsnorm(_ptr(y), _ptr(z), _ptr(w), _dtype_code(y), y.numel() // dv, dv,
+                                     float(eps), _ptr(o), _stream(y.device))
     _check(st, "gdn_gated_rmsnorm")
     return o
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Diagnostic: limit of the tensor-core prefill's bounded hand-off waits
+    (ns; negative restores the 2 s default, 0 makes them give up at once)."""
+    lib().gdn_set_wait_limit_ns(int(ns))
 
 
 def check_device_status(device: Optional[torch.device] = None) -> None:
     """Synchronise and raise if a kernel skipped work (bad cu_seqlens, timeout)."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
-    _check(lib().gdn_check_device_status(_stream(dev)), "device status")
+    with _on(dev):
+        _check(lib().gdn_check_device_status(_stream(dev)), "device status")
 
 
 def state_bytes(n_layers: int, heads: int, dk: int, dv: int, elem_bytes: int = 4) -> int:

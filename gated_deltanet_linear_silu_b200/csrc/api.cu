@@ -1,6 +1,7 @@
 // C ABI of libgdn (declared in include/gdn.h): argument validation on the
 // host, workspace carving, kernel dispatch. No allocation, no host sync except
 // in gdn_check_device_status.
+#include <atomic>
 #include <mutex>
 
 #include "../../include/gdn.h"
@@ -33,6 +34,10 @@ int* status_ptr() {
     return g_status_ptr[dev];
 }
 
+// Process-wide limit of the tensor-core prefill's bounded hand-off waits
+// (gdn_set_wait_limit_ns); negative: the default.
+std::atomic<int64_t> g_wait_limit_ns{-1};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool head_dim_ok(int d) { return d >= 16 && d <= 128 && d % 16 == 0; }
 bool dtype_ok(gdn_dtype_t t) { return t == GDN_F32 || t == GDN_BF16; }
@@ -49,9 +54,19 @@ gdn_status_t check_host_seqlens(const int32_t* cu, int N, int64_t T_tot) {
 
 }  // namespace
 
+namespace gdn {
+uint64_t wait_limit_ns() {
+    const int64_t v = g_wait_limit_ns.load(std::memory_order_relaxed);
+    return v < 0 ? kDefaultWaitNs : static_cast<uint64_t>(v);
+}
+}  // namespace gdn
+
 extern "C" {
 
-int gdn_version(void) { return 200; }  // 0.2.0: Hk, undecayed, gdn_backward
+// 0.2.1: gdn_set_wait_limit_ns; 0.2.0: Hk, undecayed, gdn_backward
+int gdn_version(void) { return 201; }
+
+void gdn_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns < 0 ? -1 : ns, std::memory_order_relaxed); }
 
 const char* gdn_status_string(gdn_status_t s) {
     switch (s) {
@@ -153,7 +168,8 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
     gdn::PrefillArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, Hk, dk, dv,
                        ld_q, ld_k, ld_v, scale, qk_l2norm, eps, undecayed, chunk, h0, hT, o,
                        reinterpret_cast<int32_t*>(ws + wl.order_off),
-                       reinterpret_cast<int32_t*>(ws + wl.counter_off), status_ptr()};
+                       reinterpret_cast<int32_t*>(ws + wl.counter_off), status_ptr(),
+                       gdn::wait_limit_ns()};
     if (!a.status) return GDN_ERR_CUDA;
     const bool tc_ok = gdn::prefill_tc_supported(a);
     if (algo == GDN_ALGO_TENSOR && !tc_ok) return GDN_ERR_UNSUPPORTED;

@@ -123,7 +123,14 @@ struct PrefillArgs {
     int32_t* order;    // [N] sequences, longest first
     int32_t* counter;  // [1] work counter of the persistent kernels
     int* status;
+    // Limit of each bounded hand-off wait inside the tensor-core kernel (ns);
+    // 0: a wait whose phase is not complete at its first probe gives up.
+    uint64_t wait_ns;
 };
+// Default limit of the bounded hand-off waits (2 s) and the process-wide
+// setting (gdn_set_wait_limit_ns).
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+uint64_t wait_limit_ns();
 
 struct WorkspaceLayout {
     size_t counter_off, order_off, total;

@@ -59,9 +59,9 @@ gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v, gd
                                  float scale, int qk_l2norm, float eps, int undecayed, int chunk,
                                  const float* h0, float* hT, void* o, gdn_algo_t algo,
                                  void* stream) {
-    if (N < 0) return GDN_ERR_INVALID_ARG;
-    if (gdn_prefill_workspace_size(N, T_tot, H, dk, dv, chunk) > kNoallocScratchBytes)
-        return GDN_ERR_WORKSPACE;  // problem needs more scratch than the fixed array holds
+    // The fixed array stands in for the caller's workspace: gdn_prefill checks
+    // every argument first and returns GDN_ERR_WORKSPACE only for a valid
+    // problem whose schedule does not fit (more than 16320 sequences).
     void* scratch = nullptr;
     if (N > 0) {
         scratch = scratch_on_current_device();
@@ -69,8 +69,7 @@ gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const void* v, gd
     }
     return gdn_prefill(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv,
                        ld_q, ld_k, ld_v, scale, qk_l2norm, eps, undecayed, chunk, h0, hT, o, scratch,
-                       kNoallocScratchBytes,
-                       algo, stream);
+                       kNoallocScratchBytes, algo, stream);
 }
 
 }  // extern "C"

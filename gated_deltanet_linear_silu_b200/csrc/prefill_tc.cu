@@ -67,7 +67,7 @@ constexpr int kStateThreads = 128;
 constexpr int kThreads = kPrepThreads + kStateThreads;
 constexpr int kStateWarp0 = kPrepThreads / 32;               // 8
 constexpr int kBarPrep = 1, kBarState = 2;                   // named barrier ids
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
+constexpr uint64_t kWaitNs = kDefaultWaitNs;  // drains: a quarter of this
 
 // Shared memory map (bytes from a 1024-aligned base).
 constexpr uint32_t kBox = 8192;                   // 64 rows x 128 B (64 bf16)
@@ -279,14 +279,16 @@ __device__ __forceinline__ bool item_next(const PrefillArgs& a, int64_t total, I
     return true;
 }
 
-// Bounded wait that also gives up once another group has aborted.
+// Bounded wait that also gives up once another group has aborted. limit 0:
+// only a phase already complete at the first (non-blocking) probe passes.
 __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
-                                                   volatile int* abort_flag) {
+                                                   volatile int* abort_flag, uint64_t limit) {
+    if (limit == 0) return mbar_test_wait(bar, parity);
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitNs) return false;
+        if (globaltimer_ns() - t0 > limit) return false;
     }
     return true;
 }
@@ -396,7 +398,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 if (r + 1 < L) { gb.y = gp[H]; gb.w = bp[H]; }
             }
             {
-                const bool ok = mbar_wait_or_abort(&full[s], ns & 1, abort_flag);
+                const bool ok = mbar_wait_or_abort(&full[s], ns & 1, abort_flag, a.wait_ns);
                 if (group_any(kBarPrep, kPrepThreads, !ok)) {
                     if (ptid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;
@@ -455,7 +457,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
             }
             {
-                const bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag);
+                const bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag, a.wait_ns);
                 if (group_any(kBarPrep, kPrepThreads, !ok)) {
                     if (ptid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;
@@ -654,10 +656,10 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 mma_commit(pa_bar);
             }
             {
-                bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag);
+                bool ok = mbar_wait_or_abort(pa_bar, pa_phase, abort_flag, a.wait_ns);
                 // -W^T is about to be overwritten: the state group's MMA1 of the
                 // previous chunk must be done reading it.
-                if (ok && i > 0) ok = mbar_wait_or_abort(wt_free, (i - 1) & 1, abort_flag);
+                if (ok && i > 0) ok = mbar_wait_or_abort(wt_free, (i - 1) & 1, abort_flag, a.wait_ns);
                 if (group_any(kBarPrep, kPrepThreads, !ok)) {
                     if (ptid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;
@@ -740,7 +742,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 // and e^{gamma_L} S^T in R_S -- R_S always holds the state pre-decayed
                 // by the coming chunk, ready for the accumulation of K~^T U.
                 {
-                    const bool ok = mbar_wait_or_abort(&gready[s], ns & 1, abort_flag);
+                    const bool ok = mbar_wait_or_abort(&gready[s], ns & 1, abort_flag, a.wait_ns);
                     if (group_any(kBarState, kStateThreads, !ok)) {
                         if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                         break;
@@ -770,7 +772,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 group_sync(kBarState, kStateThreads);
             }
             {
-                const bool ok = mbar_wait_or_abort(&pdone[s], ns & 1, abort_flag);
+                const bool ok = mbar_wait_or_abort(&pdone[s], ns & 1, abort_flag, a.wait_ns);
                 if (group_any(kBarState, kStateThreads, !ok)) {
                     if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;
@@ -803,7 +805,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 }
             }
             {
-                const bool ok = mbar_wait_or_abort(u_bar, ph, abort_flag);
+                const bool ok = mbar_wait_or_abort(u_bar, ph, abort_flag, a.wait_ns);
                 if (group_any(kBarState, kStateThreads, !ok)) {
                     if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;
@@ -845,9 +847,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 bulk_wait_group_read0();  // the previous O store has read the staging tile
             }
             {
-                bool ok = mbar_wait_or_abort(s_bar, ph, abort_flag);
+                bool ok = mbar_wait_or_abort(s_bar, ph, abort_flag, a.wait_ns);
                 // gamma of the next chunk (other stage), for the pre-decay below
-                if (ok && !it.last) ok = mbar_wait_or_abort(&gready[s ^ 1], ((i + 1) >> 1) & 1, abort_flag);
+                if (ok && !it.last) ok = mbar_wait_or_abort(&gready[s ^ 1], ((i + 1) >> 1) & 1, abort_flag, a.wait_ns);
                 if (group_any(kBarState, kStateThreads, !ok)) {
                     if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;
@@ -890,7 +892,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 tmem_wait_st();
             }
             {
-                const bool ok = mbar_wait_or_abort(o_bar, ph, abort_flag);
+                const bool ok = mbar_wait_or_abort(o_bar, ph, abort_flag, a.wait_ns);
                 if (group_any(kBarState, kStateThreads, !ok)) {
                     if (stid == 0 && !*abort_flag) abort_now(kStatusTimeout);
                     break;

@@ -50,9 +50,12 @@
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
  *     contiguous, 16-byte aligned. The library never allocates or frees.
- *   - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
- *     asynchronous on it. Argument errors are detected on the host and
- *     returned synchronously; nothing is launched in that case.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream) of the
+ *     CURRENT device (cudaSetDevice), and every tensor lives on that device:
+ *     the library looks up its per-device status word (and the fixed scratch
+ *     array of gdn_prefill_noalloc) on the current device. All work is
+ *     asynchronous on the stream. Argument errors are detected on the host
+ *     and returned synchronously; nothing is launched in that case.
  *   - A launch failure returns GDN_ERR_CUDA (the CUDA error is left for the
  *     caller to query with cudaGetLastError()).
  *   - Problems that only the device can see (a cu_seqlens array that is not
@@ -193,9 +196,10 @@ GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gd
  * The scratch gdn_prefill keeps in the workspace lives instead in one fixed
  * array in device global memory, gdn_prefill_noalloc_max_scratch() bytes
  * (64 KiB: schedules of up to 16320 sequences), which every GPU that loads the
- * library holds until the process exits. Problems that need more scratch than
- * that return GDN_ERR_WORKSPACE before anything is launched. The call itself
- * allocates nothing.
+ * library holds until the process exits. Arguments are checked exactly as
+ * gdn_prefill checks them; a valid problem that needs more scratch than the
+ * array holds then returns GDN_ERR_WORKSPACE before anything is launched. The
+ * call itself allocates nothing.
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
@@ -327,6 +331,19 @@ GDN_API gdn_status_t gdn_gated_rmsnorm(const void* y, const void* z, const float
 GDN_API const char* gdn_status_string(gdn_status_t status);
 
 /*
+ * Diagnostic setting, process-wide: the limit in nanoseconds of each bounded
+ * wait between the warp groups of the tensor-core prefill kernel (the default
+ * is 2 s; a negative value restores it). A wait that runs out records
+ * GDN_ERR_TIMEOUT in the device status word; the kernel then stops its work,
+ * waits (again bounded) for the copies and tensor-core operations it has in
+ * flight, frees its tensor memory and returns, leaving the context usable.
+ * 0 makes every such wait whose phase is not already complete at its first
+ * probe give up at once, which exercises that path on purpose (tests). The
+ * setting applies to launches made after the call.
+ */
+GDN_API void gdn_set_wait_limit_ns(int64_t ns);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word that
  * kernels set when they skip work they cannot do safely. Returns GDN_OK,
  * GDN_ERR_INVALID_ARG (a device-side cu_seqlens check failed),
@@ -335,8 +352,9 @@ GDN_API const char* gdn_status_string(gdn_status_t status);
 GDN_API gdn_status_t gdn_check_device_status(void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH (0.2.0: q/k head count Hk,
- * the `undecayed` order, gdn_backward). Argument lists change between minor
- * versions; a binding checks the version before calling anything else. */
+ * the `undecayed` order, gdn_backward; 0.2.1: gdn_set_wait_limit_ns). Argument
+ * lists change between minor versions; a binding checks the version before
+ * calling anything else. */
 GDN_API int gdn_version(void);
 
 #ifdef __cplusplus

@@ -69,3 +69,22 @@ def oracle_unit(P, n: int, h: int):
                               dtype=P.dtype, h0=h0, scale=P.scale, qk_l2norm=P.qk_l2norm,
                               eps=P.eps, threads=1)
     return o[:, 0], hT[0, 0]
+
+
+def oracle_seq(P, n: int):
+    """Oracle on every head of one sequence of a packed problem:
+    (o [T_n, H, dv], hT [H, dk, dv]); threads over heads."""
+    a, b = int(P.cu_seqlens[n]), int(P.cu_seqlens[n + 1])
+    sl = lambda x: np.ascontiguousarray(x[a:b])
+    h0 = None if P.h0 is None else P.h0[n:n + 1]
+    o, hT = oracle.recurrence(sl(P.q), sl(P.k), sl(P.v), sl(P.g), sl(P.beta), [0, b - a],
+                              dtype=P.dtype, h0=h0, scale=P.scale, qk_l2norm=P.qk_l2norm,
+                              eps=P.eps)
+    return o, hT[0]
+
+
+def longest_first(cu_seqlens) -> np.ndarray:
+    """Sequence indices in the order the persistent prefill kernels take them:
+    longest first, ties by index."""
+    lens = np.diff(np.asarray(cu_seqlens, np.int64))
+    return np.lexsort((np.arange(lens.size), -lens))

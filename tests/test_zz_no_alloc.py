@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 import gated_deltanet_linear_silu_b200 as gdn
 import gdn_inputs as gi
-from gpu_util import DEV, TOL_BF16, dev_tensor, err, host
+from gpu_util import DEV, TOL_BF16, dev_tensor, err, host, prefill_oracle
 
 
 @pytest.fixture(autouse=True, scope="module")
@@ -62,15 +62,53 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         gdn.check_device_status(DEV)
         assert err(host(o), host(o_ref)) <= TOL_BF16
         assert err(host(hT), host(hT_ref)) <= TOL_BF16
+        # and against the fp64 oracle, so a fault shared by both entry points shows
+        o_or, h_or = prefill_oracle(P)
+        assert err(host(o), o_or) <= TOL_BF16
+        assert err(host(hT), h_or) <= TOL_BF16
 
 
-def test_noalloc_rejects_problems_larger_than_its_scratch():
+def _call_empty(L, N, hT):
+    """N empty sequences (T_tot = 0, zero initial state): only the schedule and
+    the final-state copies run, through the shared array."""
+    cu = torch.zeros(N + 1, dtype=torch.int32, device=DEV)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
+    return L.gdn_prefill_noalloc(None, None, None, gdn.GDN_F32, None, None, _p(cu), None, N, 0, 1,
+                                 0, 16, 16, 0, 0, 0, 1.0, 1, 1e-6, 0, 64, None, _p(hT), None, 0,
+                                 stream)
+
+
+def test_noalloc_size_limit_boundary():
+    """The array holds a 256-byte header plus 4 bytes per sequence: 16320
+    sequences fit (the identity-order schedule used above 8192 sequences runs
+    through the shared array), 16321 are refused with GDN_ERR_WORKSPACE."""
     L = gdn.lib()
     cap = L.gdn_prefill_noalloc_max_scratch()
     assert cap == 64 * 1024
-    too_many = cap // 4  # the schedule needs 4 bytes per sequence plus a header
+    n_max = (cap - 256) // 4
+    assert n_max == 16320
+    hT = torch.full((n_max, 1, 16, 16), 7.0, dtype=torch.float32, device=DEV)
+    assert _call_empty(L, n_max, hT) == 0
+    gdn.check_device_status(DEV)
+    assert torch.count_nonzero(hT).item() == 0  # empty sequences: hT = h0 = 0
+    hT2 = torch.empty((n_max + 1, 1, 16, 16), dtype=torch.float32, device=DEV)
+    assert _call_empty(L, n_max + 1, hT2) == 3  # GDN_ERR_WORKSPACE, nothing launched
+    gdn.check_device_status(DEV)
+
+
+def test_noalloc_checks_arguments_before_the_size_limit():
+    """An invalid problem reports the same error as gdn_prefill would, even when
+    it is also too large for the array."""
+    L = gdn.lib()
     fake = ctypes.c_void_p(1 << 20)
+    too_many = 20000
+    # H = 3 value heads on Hk = 2 q/k heads: INVALID_ARG from the argument checks
     st = L.gdn_prefill_noalloc(fake, fake, fake, gdn.GDN_BF16, fake, fake, fake, None, too_many,
-                               too_many, 1, 0, 128, 128, 0, 0, 0, 1.0, 1, 1e-6, 0, 64, None, None, fake, 0,
-                               None)
-    assert st == 3  # GDN_ERR_WORKSPACE, before anything is launched
+                               too_many, 3, 2, 128, 128, 0, 0, 0, 1.0, 1, 1e-6, 0, 64, None, None,
+                               fake, 0, None)
+    assert st == 1
+    # a valid problem of that size: WORKSPACE, before anything is launched
+    st = L.gdn_prefill_noalloc(fake, fake, fake, gdn.GDN_BF16, fake, fake, fake, None, too_many,
+                               too_many, 1, 0, 128, 128, 0, 0, 0, 1.0, 1, 1e-6, 0, 64, None, None,
+                               fake, 0, None)
+    assert st == 3
