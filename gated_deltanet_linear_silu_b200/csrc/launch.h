@@ -121,7 +121,8 @@ struct PrefillArgs {
     void* o;
     // Workspace carve-up (see prefill_workspace_layout).
     int32_t* order;    // [N] sequences, longest first
-    int32_t* counter;  // [1] work counter of the persistent kernels
+    int32_t* counter;  // [2]: work counter of the persistent kernels; number of
+                       // work sequences (tokens, sane bounds: order's first entries)
     int* status;
     // Limit of each bounded hand-off wait inside the tensor-core kernel (ns);
     // 0: a wait whose phase is not complete at its first probe gives up.

@@ -73,11 +73,12 @@ def test_prefill_degenerate_gates(algo):
     assert err(hT, P.h0) <= TOL_BF16
 
 
-@pytest.mark.parametrize("g_scale", [1.6, 4.0])
+@pytest.mark.parametrize("g_scale", [1.0, 4.0])
 def test_prefill_bf16_decay_ranges(g_scale):
-    """Chunks whose decay range (gamma_0 - gamma_63, about 51 * g_scale here) stays
-    below or exceeds the range the tensor-core path factors into row and column
-    terms (80): both ways of forming e^{gamma_r - gamma_j} against the oracle."""
+    """Chunks whose cumulative decay |gamma| (about 51 * g_scale at a chunk's end
+    here) stays below or exceeds the bound under which the tensor-core path
+    factors e^{gamma_r - gamma_j} into e^{gamma_r} e^{-gamma_j} (60): both ways of
+    forming the decay, against the oracle."""
     P = gi.random_prefill(13, [130, 64, 200], H=2, dk=128, dv=128, g_scale=g_scale, with_h0=True)
     o, hT = prefill_gpu(P, algo="tensor")
     o_ref, h_ref = prefill_oracle(P)
