@@ -339,6 +339,59 @@ def bench_prefill(args, dist, pk):
     return res
 
 
+def bench_prefill_gated(args, dist, pk):
+    """The headline prefill with the layer's gated RMSNorm output
+    (gdn_prefill_gated: the recurrence, then the gate over o in place), against
+    the same call without the gate, alternated on the same inputs."""
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    P = gi.long_prefill(SEQS, SEQ_LEN, H, D)
+    T = P.T_tot
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k, v = bf(P.q), bf(P.k), bf(P.v)
+    g, beta = torch.from_numpy(P.g).to(dev), torch.from_numpy(P.beta).to(dev)
+    cu = torch.from_numpy(P.cu_seqlens).to(dev)
+    r = np.random.default_rng(7)
+    z = torch.from_numpy(r.standard_normal((T, H, D), dtype=np.float32)).to(dev).to(torch.bfloat16)
+    w = torch.from_numpy((1.0 + 0.1 * r.standard_normal(D)).astype(np.float32)).to(dev)
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((SEQS, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(SEQS, T, H, D, D, CHUNK), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def plain():
+        gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, algo=args.algo)
+
+    def gated():
+        gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, algo=args.algo, z=z,
+                    norm_w=w)
+
+    for fn in (plain, gated, plain, gated):
+        fn()
+    torch.cuda.synchronize()
+    reps = max(3, min(args.steps, 10))
+    p_ms, g_ms = [], []
+    for _ in range(2):
+        p_ms.append(timed(plain, reps, stream)[0] / reps)
+        g_ms.append(timed(gated, reps, stream)[0] / reps)
+    gdn.check_device_status(dev)
+    pm, gm = dist.max(min(p_ms)), dist.max(min(g_ms))
+    th = T * H
+    bytes_g = th * (BYTES_PER_TOKEN_HEAD + 3 * D * 2) + SEQS * H * STATE_BYTES  # + z, o in and out
+    res = {"ms": gm, "ms_ungated": pm, "ratio": gm / pm,
+           "workload": f"long_prefill_{SEQS}x{SEQ_LEN}_h16_d128_bf16_gated_rmsnorm",
+           "roofline": {"bound": "hbm", "achieved": bytes_g / (gm * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": bytes_g / (gm * 1e-3) / 1e9 / pk["hbm_gbs"],
+                        "algorithmic_bytes": bytes_g},
+           "gpu_launches": 2 * reps}
+    del q, k, v, z, o, hT
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_decode(args, dist, pk):
     """256 sequences x 16 heads, d=128, 100 in-place steps (one call each)."""
     import torch
@@ -831,6 +884,7 @@ def run_ours(args, dist: Dist):
         extras["varlen"] = bench_varlen(args, dist, pk)
         extras["decode_layer"] = bench_decode_layer(args, dist, pk)
         extras["gated_rmsnorm"] = bench_gated_norm(args, dist, pk)
+        extras["prefill_gated"] = bench_prefill_gated(args, dist, pk)
         extras["grouped"] = bench_grouped(args, dist, pk)
         extras["undecayed"] = bench_undecayed(args, dist, pk)
         extras["backward"] = bench_backward(args, dist, pk)
@@ -892,6 +946,8 @@ def summarize(line, extras):
             o["hbm"] = r(d["roofline"]["frac"], 3)
         if "tc_roofline" in d:
             o["tc"] = r(d["tc_roofline"]["frac"], 3)
+        if "ratio" in d:
+            o["ratio"] = r(d["ratio"], 3)
         if "conv" in d:
             o["conv_ms"] = r(d["conv"]["ms"])
             o["conv_hbm"] = r(d["conv"]["roofline"]["frac"], 3)
@@ -899,7 +955,7 @@ def summarize(line, extras):
 
     s = {"prefill": {"ms": r(line["ms_per_step"]), "hbm": r(line["roofline"]["frac"], 3),
                      "tc": r(line["tc_roofline"]["frac"], 3)}}
-    for name in ("decode", "decode_layer", "layer", "varlen", "gated_rmsnorm", "backward"):
+    for name in ("decode", "decode_layer", "layer", "varlen", "gated_rmsnorm", "prefill_gated", "backward"):
         if name in extras:
             s[name] = obj(extras[name])
     if "decode" in extras and isinstance(extras["decode"].get("ms_per_step_graph"), float):
@@ -949,7 +1005,8 @@ def main():
 
 ONLY = {"decode": bench_decode, "layer": bench_layer, "varlen": bench_varlen,
         "decode_layer": bench_decode_layer, "gated_rmsnorm": bench_gated_norm,
-        "grouped": bench_grouped, "undecayed": bench_undecayed, "backward": bench_backward}
+        "grouped": bench_grouped, "undecayed": bench_undecayed, "backward": bench_backward,
+        "prefill_gated": bench_prefill_gated}
 
 if __name__ == "__main__":
     main()

@@ -26,7 +26,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
-ABI_VERSION = 201  # gdn_version() of the C ABI these argument lists describe
+ABI_VERSION = 202  # gdn_version() of the C ABI these argument lists describe
 
 GDN_F32, GDN_BF16 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tensor": 2}
@@ -61,6 +61,10 @@ def lib() -> ctypes.CDLL:
                                   i64, i64, i64, f32, i32, f32, i32, i32, vp, vp, vp, vp, sz, i32,
                                   vp]
         L.gdn_prefill.restype = i32
+        L.gdn_prefill_gated.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                        i32, i64, i64, i64, f32, i32, f32, i32, i32, vp, vp, vp, vp,
+                                        vp, f32, vp, sz, i32, vp]
+        L.gdn_prefill_gated.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
                                       f32, i32, vp, vp]
         L.gdn_decode_layer_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, f32, i32, i32,
@@ -190,13 +194,17 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
             scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6, chunk: int = 64,
             cu_seqlens_host: Optional[torch.Tensor] = None, algo: str = "auto",
             workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-            undecayed: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+            undecayed: bool = False, z: Optional[torch.Tensor] = None,
+            norm_w: Optional[torch.Tensor] = None, norm_eps: float = 1e-6
+            ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked gated delta rule. q,k [T,Hk,dk], v [T,H,dv] (bf16 or fp32; each
     may be a token-strided view, e.g. a slice of the fused conv output; Hk < H
     groups H / Hk value heads on each q, k head), g,beta [T,H] fp32, cu_seqlens
     int32 [N+1] (device). Returns (o, hT); final_state may be initial_state
     itself for an in-place update. undecayed=True reads each token's memory
-    from the state before its decay (the 7.6.2 order)."""
+    from the state before its decay (the 7.6.2 order). With z [T,H,dv] (and
+    norm_w [dv] fp32) the output is the gated RMSNorm RMSNorm(y) * norm_w *
+    SiLU(z) of the recurrence's output y, applied before the output is stored."""
     _check_heads(q, k, v, g, beta)
     T, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
@@ -213,14 +221,26 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     host_cu = None
     if cu_seqlens_host is not None:
         host_cu = cu_seqlens_host.to(torch.int32).contiguous()
-    with _on(q.device):
-        st = lib().gdn_prefill(
-            _ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
-            None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
-            ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(undecayed), int(chunk),
-            _ptr(initial_state), _ptr(hT),
-            _ptr(o), _ptr(workspace), workspace.numel(), ALGOS[algo], _stream(q.device))
-    _check(st, "gdn_prefill")
+    common = (_ptr(q), _ptr(k), _ptr(v), _dtype_code(q), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+              None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()), N, T, H, Hk, dk, dv,
+              ld[0], ld[1], ld[2], float(scale), int(qk_l2norm), float(eps), int(undecayed),
+              int(chunk), _ptr(initial_state), _ptr(hT), _ptr(o))
+    if z is None:
+        with _on(q.device):
+            st = lib().gdn_prefill(*common, _ptr(workspace), workspace.numel(), ALGOS[algo],
+                                   _stream(q.device))
+        _check(st, "gdn_prefill")
+    else:
+        if norm_w is None:
+            raise ValueError("a gated prefill needs norm_w")
+        _cuda(z, norm_w)
+        if tuple(z.shape) != (T, H, dv) or z.dtype != q.dtype:
+            raise ValueError("z must be [T, H, dv] in the dtype of q")
+        with _on(q.device):
+            st = lib().gdn_prefill_gated(*common, _ptr(z), _ptr(norm_w), float(norm_eps),
+                                         _ptr(workspace), workspace.numel(), ALGOS[algo],
+                                         _stream(q.device))
+        _check(st, "gdn_prefill_gated")
     return o, hT
 
 

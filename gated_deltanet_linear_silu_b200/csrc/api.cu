@@ -63,8 +63,8 @@ uint64_t wait_limit_ns() {
 
 extern "C" {
 
-// 0.2.1: gdn_set_wait_limit_ns; 0.2.0: Hk, undecayed, gdn_backward
-int gdn_version(void) { return 201; }
+// 0.2.2: gdn_prefill_gated; 0.2.1: gdn_set_wait_limit_ns; 0.2.0: Hk, undecayed, gdn_backward
+int gdn_version(void) { return 202; }
 
 void gdn_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns < 0 ? -1 : ns, std::memory_order_relaxed); }
 
@@ -128,13 +128,18 @@ size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, i
     return gdn::prefill_workspace_layout(N < 0 ? 0 : N).total;
 }
 
-gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
-                         const float* g, const float* beta, const int32_t* cu_seqlens,
-                         const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
-                         int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale,
-                         int qk_l2norm, float eps, int undecayed, int chunk, const float* h0,
-                         float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
-                         void* stream) {
+}  // extern "C"
+
+namespace {
+
+// gdn_prefill and gdn_prefill_gated (z == nullptr: no gate).
+gdn_status_t prefill_impl(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                          const float* g, const float* beta, const int32_t* cu_seqlens,
+                          const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
+                          int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale,
+                          int qk_l2norm, float eps, int undecayed, int chunk, const float* h0,
+                          float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
+                          const void* z, const float* norm_w, float norm_eps, void* stream) {
     if (Hk == 0) Hk = H;
     if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0 || Hk < 0 || H % Hk != 0)
         return GDN_ERR_INVALID_ARG;
@@ -179,7 +184,45 @@ gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_
     cudaError_t e = gdn::launch_prefill_schedule(a, s);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
     e = use_tc ? gdn::launch_prefill_tc(a, s) : gdn::launch_prefill_simt(a, s);
-    return from_cuda(e);
+    if (e != cudaSuccess || !z || T_tot == 0) return from_cuda(e);
+    // The gate as a second pass over o, in place: one warp per row reduces the
+    // row's d_v values in registers. (Inside the tensor-core kernel's output
+    // epilogue, where a thread holds one d_v column of 64 tokens, the per-token
+    // reduction and gate loads cost more than this pass.)
+    gdn::GatedNormArgs gn{o, z, norm_w, dtype == GDN_BF16, T_tot * H, dv, norm_eps, o};
+    return from_cuda(gdn::launch_gated_rmsnorm(gn, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                         const float* g, const float* beta, const int32_t* cu_seqlens,
+                         const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
+                         int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale,
+                         int qk_l2norm, float eps, int undecayed, int chunk, const float* h0,
+                         float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
+                         void* stream) {
+    return prefill_impl(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv,
+                        ld_q, ld_k, ld_v, scale, qk_l2norm, eps, undecayed, chunk, h0, hT, o, workspace,
+                        ws_bytes, algo, nullptr, nullptr, 0.f, stream);
+}
+
+gdn_status_t gdn_prefill_gated(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                               const float* g, const float* beta, const int32_t* cu_seqlens,
+                               const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
+                               int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale,
+                               int qk_l2norm, float eps, int undecayed, int chunk, const float* h0,
+                               float* hT, void* o, const void* z, const float* norm_w, float norm_eps,
+                               void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream) {
+    if (T_tot > 0 && (!z || !norm_w)) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(z) || !aligned16(norm_w) || !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if (z && z == o) return GDN_ERR_INVALID_ARG;
+    if (dv > 256 || dv % 4 != 0) return GDN_ERR_UNSUPPORTED;  // the CUDA-core path's gate kernel
+    return prefill_impl(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv,
+                        ld_q, ld_k, ld_v, scale, qk_l2norm, eps, undecayed, chunk, h0, hT, o, workspace,
+                        ws_bytes, algo, T_tot > 0 ? z : nullptr, norm_w, norm_eps, stream);
 }
 
 int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_algo_t algo) {

@@ -14,6 +14,8 @@
 // the first use, so a CTA keeps (TT + 3) x 16 bytes per thread in flight; tiles
 // that touch a sequence start take a token-by-token path that reads the conv
 // state (or zeros) for positions before the start.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -87,6 +89,27 @@ template <> struct Raw8<float> {
 // SiLU(x) = x * sigmoid(x) = x / (1 + e^-x), with the fast exponential and
 // divide (both within a few ulp of fp32; the result is 0 when e^-x overflows).
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+
+// SiLU for bf16 outputs, one XU operation: x sigmoid(x) = h + h tanh(h), h = x/2,
+// with the hardware tanh (PTX tanh.approx.f32: absolute error about 2^-11 on
+// tanh, so |error| <= |x| 2^-12 on SiLU -- below the bf16 rounding of the result
+// where SiLU is not vanishingly small).
+__device__ __forceinline__ float silu_tanh(float x) {
+    const float h = 0.5f * x;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+}
+
+// One token's 8 channels as four fp32 pairs (bf16: exact widening).
+template <typename T> struct Pairs;
+template <> struct Pairs<uint16_t> {
+    __device__ __forceinline__ static void get(const uint4& u, float2 (&x)[4]) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    }
+};
 
 // conv (4-wide window, taps right-aligned) + SiLU for one token; returns the
 // squared norm of the 8 outputs.
@@ -181,6 +204,58 @@ __global__ void __launch_bounds__(kThreads) conv_silu_kernel(ConvArgs a) {
 #pragma unroll
         for (int u = 0; u < kTT + 3; ++u)
             if (active && t0 - 3 + u < t1) r[u].load(xp + (int64_t)u * a.C);
+        if constexpr (std::is_same<T, uint16_t>::value) {
+            // bf16: packed fp32 pairs (two channels per FFMA2), one-XU SiLU, pair
+            // packing to bf16 -- about 10 instructions per element
+            float2 w2[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int p = 0; p < 4; ++p) w2[j][p] = make_float2(wp[j][2 * p], wp[j][2 * p + 1]);
+            float2 xm3[4], xm2[4], xm1[4];
+            Pairs<T>::get(r[0].u, xm3);
+            Pairs<T>::get(r[1].u, xm2);
+            Pairs<T>::get(r[2].u, xm1);
+#pragma unroll
+            for (int u = 0; u < kTT; ++u) {
+                const int64_t t = t0 + u;
+                if (t >= t1) break;  // uniform over the CTA
+                float2 xt[4], y[4];
+                Pairs<T>::get(r[u + 3].u, xt);
+                float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    float2 acc = __fmul2_rn(w2[0][p], xm3[p]);
+                    acc = __ffma2_rn(w2[1][p], xm2[p], acc);
+                    acc = __ffma2_rn(w2[2][p], xm1[p], acc);
+                    acc = __ffma2_rn(w2[3][p], xt[p], acc);
+                    acc = make_float2(silu_tanh(acc.x), silu_tanh(acc.y));
+                    y[p] = acc;
+                    ss2 = __ffma2_rn(acc, acc, ss2);
+                }
+                if (a.qk_l2norm) {
+                    const float ss = group_sum(ss2.x + ss2.y, lanes_per_head);
+                    if (norm_me) {
+                        const float inv = rsqrtf(ss + a.eps);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) y[p] = __fmul2_rn(y[p], make_float2(inv, inv));
+                    }
+                }
+                if (active) {
+                    __nv_bfloat162 o[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) o[p] = __floats2bfloat162_rn(y[p].x, y[p].y);
+                    *reinterpret_cast<uint4*>(static_cast<T*>(a.y) + t * a.C + c0) = *reinterpret_cast<uint4*>(o);
+                }
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    xm3[p] = xm2[p];
+                    xm2[p] = xm1[p];
+                    xm1[p] = xt[p];
+                }
+            }
+            return;
+        }
         float xm3[8], xm2[8], xm1[8];
         r[0].get(xm3);
         r[1].get(xm2);

@@ -186,6 +186,31 @@ GDN_API gdn_status_t gdn_prefill(const void* q, const void* k, const void* v, gd
                          void* workspace, size_t ws_bytes, gdn_algo_t algo, void* stream);
 
 /*
+ * gdn_prefill followed by the layer's gated RMSNorm output, in one call. [G]
+ * For every (token, value head) row of d_v features, with y the recurrence's
+ * output as gdn_prefill computes it:
+ *   o = y / sqrt(mean(y^2) + norm_eps) * norm_w * SiLU(z),   SiLU(x) = x / (1 + e^-x)
+ * in fp32, rounded once to dtype: a second kernel over o, in place, after the
+ * recurrence (the pass of gdn_gated_rmsnorm).
+ *
+ *   z        [T_tot, H, dv]   dtype, the gate (may not alias o)
+ *   norm_w   [dv]             fp32, applied as given (a caller with zero-centred
+ *                             weights passes 1 + w)
+ *   norm_eps                  >= 0
+ * Every other argument, result and error as gdn_prefill; in addition
+ * GDN_ERR_UNSUPPORTED for dv > 256 or dv not a multiple of 4.
+ */
+GDN_API gdn_status_t gdn_prefill_gated(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
+                                       const float* g, const float* beta, const int32_t* cu_seqlens,
+                                       const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H,
+                                       int Hk, int dk, int dv, int64_t ld_q, int64_t ld_k,
+                                       int64_t ld_v, float scale, int qk_l2norm, float eps,
+                                       int undecayed, int chunk, const float* h0, float* hT, void* o,
+                                       const void* z, const float* norm_w, float norm_eps,
+                                       void* workspace, size_t ws_bytes, gdn_algo_t algo,
+                                       void* stream);
+
+/*
  * gdn_prefill without a caller-supplied workspace. The sources describe no
  * counterpart of this call: it exists for callers that cannot allocate device
  * memory where they run the mixer -- a runtime whose memory planner reserved
@@ -352,7 +377,8 @@ GDN_API void gdn_set_wait_limit_ns(int64_t ns);
 GDN_API gdn_status_t gdn_check_device_status(void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH (0.2.0: q/k head count Hk,
- * the `undecayed` order, gdn_backward; 0.2.1: gdn_set_wait_limit_ns). Argument
+ * the `undecayed` order, gdn_backward; 0.2.1: gdn_set_wait_limit_ns; 0.2.2:
+ * gdn_prefill_gated). Argument
  * lists change between minor versions; a binding checks the version before
  * calling anything else. */
 GDN_API int gdn_version(void);

@@ -253,6 +253,32 @@ def test_prefill_more_units_than_sms(algo):
     assert np.array_equal(hT[5], P.h0[5]) and np.array_equal(hT[17], P.h0[17])
 
 
+@pytest.mark.parametrize("algo", ["tensor", "simt"])
+@pytest.mark.parametrize("undecayed", [False, True])
+def test_prefill_gated_output(algo, undecayed):
+    """The gated RMSNorm output fused into the prefill (7.6.2: RMSNorm(y) * w *
+    SiLU(z)) against the oracle's gate applied to the oracle's recurrence: ragged
+    lengths with partial chunks, an empty sequence and initial states."""
+    P = gi.random_prefill(24, [1, 63, 64, 65, 0, 200, 130], H=3, dk=128, dv=128, with_h0=True)
+    r = np.random.default_rng(25)
+    z = gi.to_bf16_bits((r.normal(size=(P.T_tot, P.H, 128)) * 2).astype(np.float32))
+    w = (1.0 + 0.1 * r.normal(size=128)).astype(np.float32)
+    q, k, v = (dev_tensor(a, "bf16") for a in (P.q, P.k, P.v))
+    o, hT = gdn.prefill(q, k, v, dev_tensor(P.g, "f32"), dev_tensor(P.beta, "f32"),
+                        torch.from_numpy(P.cu_seqlens).to(DEV), initial_state=dev_tensor(P.h0, "f32"),
+                        algo=algo, undecayed=undecayed, z=dev_tensor(z, "bf16"),
+                        norm_w=torch.from_numpy(w).to(DEV), norm_eps=1e-6)
+    gdn.check_device_status(DEV)
+    y_ref, h_ref = prefill_oracle(P, undecayed=undecayed)
+    ref = oracle.gated_rmsnorm(y_ref, gi.bf16_bits_to_f32(z).astype(np.float64), w, dtype="f64",
+                               eps=1e-6)
+    assert err(host(o), ref) <= TOL_BF16
+    assert err(host(hT), h_ref) <= TOL_BF16
+    # the gate does not change the state
+    o2, hT2 = prefill_gpu(P, algo=algo, undecayed=undecayed)
+    assert np.array_equal(host(hT), hT2)
+
+
 def test_varlen_packing_equals_separate_calls():
     P = gi.random_prefill(6, [33, 0, 97, 64], H=2, dk=64, dv=64, dtype="f32", with_h0=True)
     o, hT = prefill_gpu(P)
