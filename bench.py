@@ -556,7 +556,7 @@ def bench_decode_layer(args, dist, pk):
             "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                         "traffic": profiled_traffic("decode_layer_kernel", ["decode.cu"], N * H),
+                         "traffic": profiled_traffic("decode_layer_stream_kernel", ["decode_stream.cu"], N * H),
                          "algorithmic_bytes": bytes_step},
             "gpu_launches": steps}
 

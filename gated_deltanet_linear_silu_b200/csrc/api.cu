@@ -256,7 +256,7 @@ gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v, gdn_dt
     if (qk_l2norm && !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
     gdn::DecodeArgs a{q, k, v, dtype == GDN_BF16, g, beta, state, N, H, Hk, dk, dv, scale, qk_l2norm, eps, undecayed, o,
-                      nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0.f};
+                      nullptr, nullptr, nullptr, 0, nullptr, nullptr, 0.f, status_ptr(), gdn::wait_limit_ns()};
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -282,7 +282,8 @@ gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv
     if (z && !(norm_eps >= 0.f)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)N * H >= (int64_t)1 << 31) return GDN_ERR_UNSUPPORTED;
     gdn::DecodeArgs a{nullptr, nullptr, nullptr, dtype == GDN_BF16, g, beta, state, N, H, Hk, dk, dv,
-                      scale, qk_l2norm, eps, undecayed, o, x, conv_w, conv_state, K, z, norm_w, norm_eps};
+                      scale, qk_l2norm, eps, undecayed, o, x, conv_w, conv_state, K, z, norm_w, norm_eps,
+                      status_ptr(), gdn::wait_limit_ns()};
     return from_cuda(gdn::launch_decode_step(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -318,6 +318,7 @@ cudaError_t launch_t(const DecodeArgs& a, cudaStream_t s) {
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s) {
     if ((int64_t)a.N * a.H == 0) return cudaSuccess;
+    if (decode_stream_supported(a)) return launch_decode_stream(a, s);
     return a.is_bf16 ? launch_t<uint16_t>(a, s) : launch_t<float>(a, s);
 }
 

@@ -48,8 +48,15 @@ struct DecodeArgs {
     const void* z;        // [N, H, dv]
     const float* norm_w;  // [dv]
     float norm_eps;
+    int* status;      // device status word (GDN_ERR_TIMEOUT when a wait runs out)
+    uint64_t wait_ns;  // bound on each wait of the streaming kernel
 };
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
+// Persistent streaming form of the whole-mixer step (ungrouped heads): two
+// CTAs per SM, each prefetching its next unit's state and conv inputs into a
+// shared-memory slot by bulk copies.
+bool decode_stream_supported(const DecodeArgs& a);
+cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s);
 // Largest value-head group (H / Hk) of the whole-mixer decode step: one
 // thread-block cluster per group, 8 being the portable cluster size.
 constexpr int kMaxDecodeGroup = 8;

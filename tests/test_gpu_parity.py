@@ -563,6 +563,71 @@ def test_decode_layer_step_undecayed_read(kind):
     assert worst <= tol_ and err(host(st_d), st_o) <= tol_
 
 
+@pytest.mark.parametrize("kind,K,gate", [("bf16", 4, True), ("f32", 4, True), ("bf16", 1, False),
+                                         ("f32", 3, False)])
+def test_decode_layer_step_many_units_per_sm(kind, K, gate):
+    """640 (sequence, head) units, several per SM: the streaming kernel's ring
+    of state slots wraps around (three slots in bf16, two in fp32, whose conv
+    inputs are twice as large); K = 1 runs without a conv state."""
+    r = np.random.default_rng(46 + K)
+    N, H, dk, dv = 40, 16, 128, 128
+    C = 2 * H * dk + H * dv
+    to = (lambda a: gi.to_bf16_bits(a.astype(np.float32))) if kind == "bf16" else (
+        lambda a: a.astype(np.float32))
+    cw = to(r.normal(size=(C, K)) * 0.5)
+    cs = to(r.normal(size=(N, C, K - 1))) if K > 1 else None
+    st = (r.normal(size=(N, H, dk, dv)) * 0.1).astype(np.float32)
+    nw = (1.0 + 0.1 * r.normal(size=dv)).astype(np.float32)
+    cs_d = dev_tensor(cs, kind) if K > 1 else None
+    st_d = torch.from_numpy(st).to(DEV)
+    cs_o, st_o = cs, st.astype(np.float64)
+    worst = 0.0
+    for t in range(2):
+        x = to(r.normal(size=(N, C)))
+        z = to(r.normal(size=(N, H, dv))) if gate else None
+        g = (-np.log1p(np.exp(r.normal(size=(N, H))))).astype(np.float32)
+        b = (1.0 / (1.0 + np.exp(-r.normal(size=(N, H))))).astype(np.float32)
+        o = gdn.decode_layer_step(dev_tensor(x, kind), dev_tensor(cw, kind), cs_d,
+                                  torch.from_numpy(g).to(DEV), torch.from_numpy(b).to(DEV), st_d,
+                                  H=H, dk=dk, dv=dv, z=None if z is None else dev_tensor(z, kind),
+                                  norm_w=torch.from_numpy(nw).to(DEV) if gate else None)
+        o_ref, cs_n, st_o = oracle.decode_layer_step(x, cw, cs_o, g, b, st_o, dtype=kind, H=H,
+                                                     dk=dk, dv=dv, z=z, norm_w=nw if gate else None)
+        if K > 1:
+            cs_o = to(cs_n) if kind == "bf16" else cs_n
+        worst = max(worst, err(host(o), o_ref))
+    gdn.check_device_status(DEV)
+    tol_ = TOL_BF16 if kind == "bf16" else TOL_F32
+    assert worst <= tol_
+    assert err(host(st_d), st_o) <= tol_
+    if K > 1:
+        assert np.array_equal(host(cs_d), (gi.bf16_bits_to_f32(cs_o) if kind == "bf16" else cs_o)
+                              .astype(np.float32))
+
+
+@pytest.mark.parametrize("kind,dk,dv", [("f32", 128, 128), ("bf16", 48, 80), ("bf16", 16, 32)])
+def test_decode_step_many_units_per_sm(kind, dk, dv):
+    """More (sequence, head) units than SMs, shapes with 1, 4 and 16 state rows
+    per thread."""
+    r = np.random.default_rng(47)
+    N, H = 70, 9
+    q, k = r.normal(size=(N, H, dk)).astype(np.float32), r.normal(size=(N, H, dk)).astype(np.float32)
+    v = r.normal(size=(N, H, dv)).astype(np.float32)
+    if kind == "bf16":
+        q, k, v = gi.to_bf16_bits(q), gi.to_bf16_bits(k), gi.to_bf16_bits(v)
+    g = -np.abs(r.normal(size=(N, H))).astype(np.float32)
+    beta = r.uniform(size=(N, H)).astype(np.float32)
+    s0 = r.normal(0, 0.1, size=(N, H, dk, dv)).astype(np.float32)
+    state = dev_tensor(s0, "f32")
+    o = gdn.decode_step(dev_tensor(q, kind), dev_tensor(k, kind), dev_tensor(v, kind),
+                        dev_tensor(g, "f32"), dev_tensor(beta, "f32"), state, scale=0.7)
+    gdn.check_device_status(DEV)
+    o_ref, s_ref = oracle.recurrence(q, k, v, g, beta, np.arange(N + 1), dtype=kind, h0=s0,
+                                     scale=0.7)
+    assert err(host(o), o_ref) <= tol(kind)
+    assert err(host(state), s_ref) <= TOL_F32
+
+
 def test_decode_layer_step_equals_separate_kernels():
     """The fused step equals conv_silu, then decode_step, then gated_rmsnorm run as
     three library calls (fp32, same arithmetic order up to rounding)."""
