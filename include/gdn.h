@@ -292,7 +292,10 @@ GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v
  *   o           [N, H, dv]        dtype   output
  * Supported: dk, dv in {16, 32, ..., 128}; H / Hk <= 8 (the CTAs of one
  * value-head group run as one thread-block cluster; larger groups return
- * GDN_ERR_UNSUPPORTED). No buffer may overlap another.
+ * GDN_ERR_UNSUPPORTED). No buffer may overlap another. With H == Hk the step
+ * runs as a persistent kernel whose wait for each state copy is bounded (see
+ * gdn_set_wait_limit_ns): a wait that runs out leaves some (sequence, head)
+ * units unprocessed and records GDN_ERR_TIMEOUT for gdn_check_device_status.
  */
 GDN_API gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv_state, int K,
                                            gdn_dtype_t dtype, const float* g, const float* beta,
@@ -357,7 +360,8 @@ GDN_API const char* gdn_status_string(gdn_status_t status);
 
 /*
  * Diagnostic setting, process-wide: the limit in nanoseconds of each bounded
- * wait between the warp groups of the tensor-core prefill kernel (the default
+ * wait between the warp groups of the tensor-core prefill kernel and of the
+ * wait for a state copy in the streaming whole-mixer decode step (the default
  * is 2 s; a negative value restores it). A wait that runs out records
  * GDN_ERR_TIMEOUT in the device status word; the kernel then stops its work,
  * waits (again bounded) for the copies and tensor-core operations it has in
