@@ -23,16 +23,20 @@ _F32, _BF16, _F64 = 0, 1, 2
 _lib = None
 
 
+def _rec_argtypes():
+    vp, i32, f64, i64p = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
+    return [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32, i32, i32, f64, i32, f64, i32, vp,
+            i32, vp, vp, i32]
+
+
 def lib():
     global _lib
     if _lib is None:
         path = _build.build()
         L = ctypes.CDLL(path)
         vp, i32, f64, i64p = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
-        L.gdn_oracle_recurrence_mut.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32,
-                                                i32, i32, f64, i32, f64, i32, vp, i32, vp, vp, i32,
-                                                i32]
-        L.gdn_oracle_recurrence_mut.restype = i32
+        L.gdn_oracle_recurrence.argtypes = _rec_argtypes()
+        L.gdn_oracle_recurrence.restype = i32
         L.gdn_oracle_chunked.argtypes = [vp, vp, vp, i32, vp, vp, i32, i64p, i32, i32, i32, i32,
                                          i32, f64, i32, f64, i32, vp, i32, vp, vp, i32, i32]
         L.gdn_oracle_chunked.restype = i32
@@ -41,6 +45,16 @@ def lib():
         L.gdn_oracle_conv_silu.restype = i32
         _lib = L
     return _lib
+
+
+def _pincheck_entry():
+    """The recurrence with a planted mistake, from the pin-check build of the
+    same source (used only by the pin-sensitivity test)."""
+    L = ctypes.CDLL(_build.build_pincheck())
+    fn = L.gdn_oracle_recurrence_planted
+    fn.argtypes = _rec_argtypes() + [ctypes.c_int]
+    fn.restype = ctypes.c_int
+    return fn
 
 
 def default_threads() -> int:
@@ -63,7 +77,7 @@ def _ptr(a: Optional[np.ndarray]):
 
 def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: float = 1.0,
                qk_l2norm: bool = True, eps: float = 1e-6, threads: Optional[int] = None,
-               want_o: bool = True, mutation: int = 0, undecayed: bool = False):
+               want_o: bool = True, undecayed: bool = False, _planted: int = 0):
     """Token-by-token gated delta rule in fp64.
 
     Default order (Qwen3.5-MoE source walkthrough, 4.3): decay the state, then
@@ -76,6 +90,8 @@ def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: floa
     Value head h reads q, k head h // (H // Hk) (grouped value heads; Hk == H
     is the plain layer).
     Returns (o [T,H,dv] float64 or None, hT [N,H,dk,dv] float64).
+    `_planted` (1..4) is for the pin-sensitivity test only: it runs the
+    pin-check build with that deliberate mistake.
     """
     T, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
@@ -89,10 +105,13 @@ def recurrence(q, k, v, g, beta, cu_seqlens, *, dtype: str, h0=None, scale: floa
     h0a, h0dt = (None, _F64) if h0 is None else _arr(np.asarray(h0), "f")
     hT = np.empty((N, H, dk, dv), np.float64)
     o = np.empty((T, H, dv), np.float64) if want_o else None
-    rc = lib().gdn_oracle_recurrence_mut(
-        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, Hk, dk, dv,
-        float(scale), int(qk_l2norm), float(eps), int(undecayed), _ptr(h0a), h0dt, _ptr(hT),
-        _ptr(o), threads or default_threads(), int(mutation))
+    args = [_ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), _ptr(beta), gdt, _ptr(cu), N, H, Hk, dk, dv,
+            float(scale), int(qk_l2norm), float(eps), int(undecayed), _ptr(h0a), h0dt, _ptr(hT),
+            _ptr(o), threads or default_threads()]
+    if _planted:
+        rc = _pincheck_entry()(*args, int(_planted))
+    else:
+        rc = lib().gdn_oracle_recurrence(*args)
     if rc != 0:
         raise ValueError("oracle recurrence: bad arguments")
     return o, hT

@@ -23,7 +23,7 @@
  *       page writes it: S_t = alpha_t S_{t-1} + k_t [beta_t (v_t - S_{t-1}^T k_t)]^T,
  *       i.e. the memory is read from the state before the decay. Selected by
  *       `undecayed`; [R]'s decay-first order is the default.
- * Readings where the pages are silent (all listed in the design notes):
+ * Readings where the pages are silent:
  *   SiLU follows the conv; L2(x) = x / sqrt(sum x^2 + eps); `scale` multiplies
  *   the normalised q; the conv state exposes the K-1 most recent inputs
  *   (the K-th is never read again); sequences never mix across cu_seqlens.
@@ -33,6 +33,12 @@
  * inputs, a library conv1d, linearity, a contraction bound and the fp64
  * chunkwise evaluator below.  Absolute parity against the pages is unpinned:
  * they print no worked numeric example of the mixer.
+ *
+ * Built with -DGDN_ORACLE_PIN_CHECK (a separate library that only the
+ * pin-sensitivity test loads), gdn_oracle_recurrence_planted can plant one of
+ * four deliberate mistakes in the recurrence, to show that the pins catch
+ * each. The oracle library proper is built without that flag and has no such
+ * code.
  */
 #include <math.h>
 #include <pthread.h>
@@ -113,8 +119,16 @@ typedef struct {
     const void *h0;
     int h0_dtype;
     double *hT, *o;
-    int mutation; /* 0 for the oracle; >0 only from the pin-sensitivity test */
+#ifdef GDN_ORACLE_PIN_CHECK
+    int planted; /* the deliberate mistake to plant (1..4), 0 for none */
+#endif
 } rec_ctx;
+
+#ifdef GDN_ORACLE_PIN_CHECK
+#define PLANTED(n) (c->planted == (n))
+#else
+#define PLANTED(n) 0
+#endif
 
 /* Normalise x (length d) in place: x / sqrt(sum x^2 + eps). */
 static void l2_normalise(double *x, int d, double eps) {
@@ -156,8 +170,8 @@ static void rec_item(void *vctx, int64_t item) {
         const double alpha = exp(g);
 
         /* [U]: kv_mem_j = sum_i S_{t-1}[i][j] k_i, before the decay.
-         * (mutation 1, pin check only: the same read planted in the default rule) */
-        if (c->undecayed || c->mutation == 1)
+         * (planted mistake 1: the same read in the default rule) */
+        if (c->undecayed || PLANTED(1))
             for (int j = 0; j < dv; ++j) {
                 double acc = 0.0;
                 for (int i = 0; i < dk; ++i) acc += S[i * dv + j] * k[i];
@@ -165,16 +179,16 @@ static void rec_item(void *vctx, int64_t item) {
             }
 
         /* S <- S * exp(g_t) */
-        if (c->mutation != 3)
+        if (!PLANTED(3)) /* planted mistake 3: no decay */
             for (int64_t e = 0; e < (int64_t)dk * dv; ++e) S[e] *= alpha;
 
         /* [R]: kv_mem_j = sum_i S[i][j] k_i  (reduction over the key axis) */
-        if (!c->undecayed && c->mutation != 1)
+        if (!c->undecayed && !PLANTED(1))
             for (int j = 0; j < dv; ++j) {
                 double acc = 0.0;
                 for (int i = 0; i < dk; ++i) {
-                    /* mutation 2 (pin check only): transposed state read */
-                    const double s = (c->mutation == 2 && dk == dv) ? S[j * dv + i] : S[i * dv + j];
+                    /* planted mistake 2: transposed state read */
+                    const double s = (PLANTED(2) && dk == dv) ? S[j * dv + i] : S[i * dv + j];
                     acc += s * k[i];
                 }
                 m[j] = acc;
@@ -183,7 +197,8 @@ static void rec_item(void *vctx, int64_t item) {
         /* delta_j = (v_j - kv_mem_j) * beta_t */
         for (int j = 0; j < dv; ++j) {
             const double vj = load_elem(c->v, c->dtype, v_base + j);
-            delta[j] = (c->mutation == 4) ? (vj + m[j]) * beta : (vj - m[j]) * beta;
+            /* planted mistake 4: wrong sign of the memory */
+            delta[j] = PLANTED(4) ? (vj + m[j]) * beta : (vj - m[j]) * beta;
         }
 
         /* S[i][j] += k_i * delta_j  (outer product k^T delta) */
@@ -216,15 +231,20 @@ static void rec_item(void *vctx, int64_t item) {
  * the plain layer). undecayed = 1 selects the [U] order (read, then decay).
  * Returns 0, or -1 on a bad argument.
  */
-int gdn_oracle_recurrence_mut(const void *q, const void *k, const void *v, int dtype,
-                              const void *g, const void *beta, int gate_dtype,
-                              const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
-                              double scale, int qk_l2norm, double eps, int undecayed,
-                              const void *h0, int h0_dtype, double *hT, double *o,
-                              int n_threads, int mutation) {
+static int recurrence_impl(const void *q, const void *k, const void *v, int dtype,
+                           const void *g, const void *beta, int gate_dtype,
+                           const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
+                           double scale, int qk_l2norm, double eps, int undecayed,
+                           const void *h0, int h0_dtype, double *hT, double *o, int n_threads,
+                           int planted) {
     if (N < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
     rec_ctx c = {q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, Hk, dk, dv, scale,
-                 qk_l2norm, eps, undecayed, h0, h0_dtype, hT, o, mutation};
+                 qk_l2norm, eps, undecayed, h0, h0_dtype, hT, o
+#ifdef GDN_ORACLE_PIN_CHECK
+                 , planted
+#endif
+    };
+    (void)planted;
     run_items(rec_item, &c, (int64_t)N * H, n_threads);
     return 0;
 }
@@ -234,10 +254,23 @@ int gdn_oracle_recurrence(const void *q, const void *k, const void *v, int dtype
                           const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
                           double scale, int qk_l2norm, double eps, int undecayed,
                           const void *h0, int h0_dtype, double *hT, double *o, int n_threads) {
-    return gdn_oracle_recurrence_mut(q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, N, H, Hk,
-                                     dk, dv, scale, qk_l2norm, eps, undecayed, h0, h0_dtype, hT, o,
-                                     n_threads, 0);
+    return recurrence_impl(q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, N, H, Hk, dk, dv, scale,
+                           qk_l2norm, eps, undecayed, h0, h0_dtype, hT, o, n_threads, 0);
 }
+
+#ifdef GDN_ORACLE_PIN_CHECK
+/* gdn_oracle_recurrence with planted mistake `planted` (1..4; pin check only). */
+int gdn_oracle_recurrence_planted(const void *q, const void *k, const void *v, int dtype,
+                                  const void *g, const void *beta, int gate_dtype,
+                                  const int64_t *cu_seqlens, int N, int H, int Hk, int dk, int dv,
+                                  double scale, int qk_l2norm, double eps, int undecayed,
+                                  const void *h0, int h0_dtype, double *hT, double *o,
+                                  int n_threads, int planted) {
+    if (planted < 1 || planted > 4) return -1;
+    return recurrence_impl(q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, N, H, Hk, dk, dv, scale,
+                           qk_l2norm, eps, undecayed, h0, h0_dtype, hT, o, n_threads, planted);
+}
+#endif
 
 /* ------------------------------------------------------------------------ */
 /* Conv stage [C]: causal depthwise conv, SiLU, per-head L2 norm of q and k.  */
@@ -445,7 +478,11 @@ int gdn_oracle_chunked(const void *q, const void *k, const void *v, int dtype,
     if (N < 0 || H <= 0 || Hk <= 0 || H % Hk != 0 || dk <= 0 || dv <= 0 || chunk <= 0 || !cu_seqlens)
         return -1;
     chunk_ctx c = {{q, k, v, dtype, g, beta, gate_dtype, cu_seqlens, H, Hk, dk, dv, scale, qk_l2norm,
-                    eps, undecayed, h0, h0_dtype, hT, o, 0},
+                    eps, undecayed, h0, h0_dtype, hT, o
+#ifdef GDN_ORACLE_PIN_CHECK
+                    , 0
+#endif
+                   },
                    chunk};
     run_items(chunk_item, &c, (int64_t)N * H, n_threads);
     return 0;

@@ -33,12 +33,12 @@ def _unit(x):
     return x / np.linalg.norm(x, axis=-1, keepdims=True)
 
 
-def _rec(mutation=0):
+def _rec(planted=0):
     def f(q, k, v, g, beta, cu, **kw):
         kw.setdefault("dtype", "f64")
         return oracle.recurrence(np.asarray(q, np.float64), np.asarray(k, np.float64),
                                  np.asarray(v, np.float64), np.asarray(g, np.float64),
-                                 np.asarray(beta, np.float64), cu, mutation=mutation,
+                                 np.asarray(beta, np.float64), cu, _planted=planted,
                                  threads=2, **kw)
     return f
 
@@ -605,9 +605,9 @@ def test_undecayed_decode_layer_steps_equal_packed_layer():
 # Pin sensitivity: each planted mistake must fail at least one pin.
 # --------------------------------------------------------------------------
 
-@pytest.mark.parametrize("mutation", [1, 2, 3, 4],
+@pytest.mark.parametrize("planted", [1, 2, 3, 4],
                          ids=["retrieve_before_decay", "transposed_state", "dropped_decay",
                               "wrong_sign_delta"])
-def test_pins_catch_planted_mistakes(mutation):
-    errs = {p.__name__: p(_rec(mutation)) for p in ALL_PINS}
+def test_pins_catch_planted_mistakes(planted):
+    errs = {p.__name__: p(_rec(planted)) for p in ALL_PINS}
     assert max(errs.values()) > 1e-6, errs
