@@ -213,7 +213,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     hT = final_state
     if hT is None and output_final_state:
         hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
-    ws_bytes = prefill_workspace_size(N, T, H, dk, dv, chunk)
+    with _on(q.device):  # the workspace can depend on the device's SM count
+        ws_bytes = prefill_workspace_size(N, T, H, dk, dv, chunk)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     ld = [_token_stride(t) for t in (q, k, v)]

@@ -124,8 +124,12 @@ gdn_status_t gdn_conv_silu(const void* x, gdn_dtype_t dtype, const void* w,
 }
 
 size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, int chunk) {
-    (void)T_tot; (void)H; (void)dk; (void)dv; (void)chunk;
-    return gdn::prefill_workspace_layout(N < 0 ? 0 : N).total;
+    const size_t base = gdn::prefill_workspace_layout(N < 0 ? 0 : N).total;
+    if (H <= 0 || T_tot < 0) return base;
+    const int S = gdn::prefill_split_segments(N, T_tot, H, dk, dv, chunk);
+    if (S <= 1) return base;
+    const size_t split = gdn::prefill_split_workspace_bytes(N, T_tot, H, S);
+    return split > base ? split : base;
 }
 
 }  // extern "C"
@@ -181,9 +185,17 @@ gdn_status_t prefill_impl(const void* q, const void* k, const void* v, gdn_dtype
     const bool use_tc = tc_ok && algo != GDN_ALGO_SIMT;
     if (!use_tc && gdn::prefill_simt_smem_bytes(chunk, dk, dv) > 227 * 1024) return GDN_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = gdn::launch_prefill_schedule(a, s);
-    if (e != cudaSuccess) return GDN_ERR_CUDA;
-    e = use_tc ? gdn::launch_prefill_tc(a, s) : gdn::launch_prefill_simt(a, s);
+    // Few (sequence, head) units: cut the sequences into segments so the
+    // tensor-core passes fill the GPU (when the workspace has room for it).
+    const int S = use_tc ? gdn::prefill_split_segments(N, T_tot, H, dk, dv, chunk) : 1;
+    cudaError_t e;
+    if (S > 1 && ws_bytes >= gdn::prefill_split_workspace_bytes(N, T_tot, H, S)) {
+        e = gdn::launch_prefill_split(a, S, workspace, s);
+    } else {
+        e = gdn::launch_prefill_schedule(a, s);
+        if (e != cudaSuccess) return GDN_ERR_CUDA;
+        e = use_tc ? gdn::launch_prefill_tc(a, s) : gdn::launch_prefill_simt(a, s);
+    }
     if (e != cudaSuccess || !z || T_tot == 0) return from_cuda(e);
     // The gate as a second pass over o, in place: one warp per row reduces the
     // row's d_v values in registers. (Inside the tensor-core kernel's output

@@ -145,6 +145,15 @@ struct WorkspaceLayout {
 };
 WorkspaceLayout prefill_workspace_layout(int N);
 
+// Sequence split for launches with few (sequence, head) units on the
+// tensor-core path: the number of segments per sequence (1: no split, which
+// also holds when dk, dv or the chunk rule it out), the workspace it needs,
+// and the split launch itself (three prefill passes and the fp32 hand-off of
+// the segments' start states).
+int prefill_split_segments(int N, int64_t T_tot, int H, int dk, int dv, int chunk);
+size_t prefill_split_workspace_bytes(int N, int64_t T_tot, int H, int S);
+cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, cudaStream_t s);
+
 // Builds the longest-first schedule and zeroes the work counter.
 cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);

@@ -1,0 +1,273 @@
+// Sequence-split prefill for launches with few (sequence, head) units.
+//
+// The recurrence is linear in the state: over a segment of a sequence,
+//   S_end = Phi S_start + L,
+// where Phi [dk, dk] is the product of the tokens' alpha_t (I - beta_t k^_t k^_t^T)
+// ("Qwen3.5-MoE source walkthrough", 4.3: decay, then the delta-rule
+// correction) and L is the segment's final state from a zero start. With
+// dk == dv the tensor-core prefill gives both from two runs over the segment:
+// a zero initial state yields L, and the identity as initial state with all
+// values v = 0 yields Phi. So when N * H units leave most SMs idle, each
+// sequence is cut into S chunk-aligned segments and
+//   pass 1a: every segment from a zero state (segment 0 from the caller's h0),
+//            final states -> L (segment 0's is the true state at segment 1);
+//   pass 1b: every segment from the identity with v = 0, final states -> Phi;
+//   combine: S_start(k+1) = Phi_k S_start(k) + L_k, k = 1 .. S-2, in fp32;
+//   pass 2:  every segment from its true start state, writing o; the last
+//            segment's final state is the sequence's hT.
+// The three passes are the ordinary prefill kernel over the segments as
+// sequences, each with S times the units of the plain launch; passes 1a and
+// 1b write o too, and pass 2 overwrites it. Outputs of pass 2 differ from the
+// plain launch only by rounding.
+#include "common.cuh"
+#include "launch.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kMaxSegments = 16;
+constexpr int kMinSegmentChunks = 4;  // average 64-token chunks per segment
+// Fewest segments worth the three passes: each pass has a fixed cost of about
+// four chunks' time (pipeline fill, state load and store), so 4 segments of
+// 16 chunks measured no faster than the plain launch, 9 segments 1.2x faster
+// and 16 segments about 1.9x faster.
+constexpr int kMinSegments = 6;
+constexpr int kSplitD = 128;          // dk = dv of the tensor-core prefill
+constexpr int64_t kStateFloats = (int64_t)kSplitD * kSplitD;
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+struct SplitLayout {
+    WorkspaceLayout base;  // schedule of the N * S segment sequences
+    size_t cu_off, a_off, b_off, l_off, r_off, zv_off, total;
+};
+
+SplitLayout split_layout(int N, int64_t T_tot, int H, int S) {
+    SplitLayout l;
+    const int64_t NS = (int64_t)N * S;
+    l.base = prefill_workspace_layout((int)NS);
+    l.cu_off = round256(l.base.total);
+    const size_t states = (size_t)NS * H * kStateFloats * sizeof(float);
+    l.a_off = round256(l.cu_off + sizeof(int32_t) * (size_t)(NS + 1));
+    l.b_off = l.a_off + states;
+    l.l_off = l.b_off + states;
+    l.r_off = l.l_off + states;
+    l.zv_off = l.r_off + states;  // bf16 zeros standing in for v in pass 1b
+    l.total = l.zv_off + round256((size_t)T_tot * H * kSplitD * 2);
+    return l;
+}
+
+// Segment boundaries: sequence n = [st, en) of c = ceil(len / 64) chunks gives
+// segment k = [st + 64 floor(k c / S), st + 64 floor((k+1) c / S)) clipped to
+// en (empty segments when c < S). A sequence with bad bounds gets empty
+// segments and keeps its bad end, so the prefill flags it.
+__global__ void split_bounds_kernel(const int32_t* cu, int N, int S, int32_t* cu_seg) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t NS = (int64_t)N * S;
+    if (idx > NS) return;
+    if (idx == NS) {
+        cu_seg[idx] = cu[N];
+        return;
+    }
+    const int n = (int)(idx / S), k = (int)(idx % S);
+    const int64_t st = cu[n], en = cu[n + 1];
+    const int64_t len = en > st ? en - st : 0;
+    const int64_t c = (len + 63) / 64;
+    const int64_t off = 64 * ((k * c) / S);
+    cu_seg[idx] = (int32_t)(st + (off < len ? off : len));
+}
+
+// A (pass 1a and pass 2 initial states): segment 0 <- h0 (zeros if none),
+// the rest zeros; B (pass 1b initial states): the identity.
+__global__ void split_fill_kernel(const float* h0, int N, int H, int S, float* A, float* B) {
+    const int64_t n4 = (int64_t)N * S * H * kStateFloats / 4;
+    for (int64_t e4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e4 < n4;
+         e4 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e = 4 * e4;
+        const int64_t blk = e / kStateFloats, within = e % kStateFloats;
+        const int h = (int)(blk % H);
+        const int k = (int)((blk / H) % S);
+        const int64_t n = blk / ((int64_t)H * S);
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k == 0 && h0) x = *reinterpret_cast<const float4*>(h0 + (n * H + h) * kStateFloats + within);
+        reinterpret_cast<float4*>(A)[e4] = x;
+        const int row = (int)(within / kSplitD), col = (int)(within % kSplitD);  // col % 4 == 0
+        const float4 id = make_float4(row == col ? 1.f : 0.f, row == col + 1 ? 1.f : 0.f,
+                                      row == col + 2 ? 1.f : 0.f, row == col + 3 ? 1.f : 0.f);
+        reinterpret_cast<float4*>(B)[e4] = id;
+    }
+}
+
+// The chain of segment start states, per (sequence, head) and block of 16
+// state columns (columns evolve independently: Phi acts on the rows), one CTA
+// each (N * H * 8 CTAs: one wave when the split applies). Thread (row i, half
+// hf) owns columns [8 hf, 8 hf + 8) of row i, in packed fp32 pairs. Phi_k is
+// staged in shared memory (rows padded to 132 floats: a quarter-warp's float4
+// reads of 8 rows hit 32 distinct banks), the next one prefetched with
+// cp.async while step k runs; the current start state's block is read as
+// broadcast float4s.
+constexpr int kCombCols = 16;
+constexpr int kCombThreads = 256;
+constexpr int kPhiLd = 132;
+constexpr size_t kCombSmem = sizeof(float) * (2 * kSplitD * kPhiLd + kSplitD * kCombCols);
+
+__device__ __forceinline__ void stage_phi(float* dst, const float* src) {
+    for (int p = threadIdx.x; p < kSplitD * kSplitD / 4; p += kCombThreads) {
+        const int r = p / (kSplitD / 4), c4 = p % (kSplitD / 4);
+        cp_async_16(dst + r * kPhiLd + 4 * c4, src + (int64_t)r * kSplitD + 4 * c4);
+    }
+    cp_async_commit_group();
+}
+
+__global__ void __launch_bounds__(kCombThreads) split_combine_kernel(int N, int H, int S, const float* Lst,
+                                                                    const float* Phi, float* A) {
+    extern __shared__ float4 comb_smem4[];
+    float* phi_s = reinterpret_cast<float*>(comb_smem4);  // [2][128][kPhiLd]
+    float* cur = phi_s + 2 * kSplitD * kPhiLd;             // [128][16]
+    const int nh = blockIdx.x;                             // n * H + h
+    const int n = nh / H, h = nh % H;
+    const int i = threadIdx.x >> 1, hf = threadIdx.x & 1;
+    const int cl = 8 * hf;                                 // first column within the block
+    const int c0 = blockIdx.y * kCombCols + cl;            // first state column
+    const int64_t off0 = ((int64_t)n * S * H + h) * kStateFloats;  // segment 0 of (n, h)
+    const int64_t seg = (int64_t)H * kStateFloats;                  // between segments
+    if (S > 2) stage_phi(phi_s, Phi + off0 + seg);
+    // S_start(1) = L_0 (segment 0 ran from the true initial state)
+    {
+        const float* l0 = Lst + off0 + (int64_t)i * kSplitD + c0;
+        float* a1 = A + off0 + seg + (int64_t)i * kSplitD + c0;
+        const float4 x0 = *reinterpret_cast<const float4*>(l0);
+        const float4 x1 = *reinterpret_cast<const float4*>(l0 + 4);
+        *reinterpret_cast<float4*>(cur + i * kCombCols + cl) = x0;
+        *reinterpret_cast<float4*>(cur + i * kCombCols + cl + 4) = x1;
+        *reinterpret_cast<float4*>(a1) = x0;
+        *reinterpret_cast<float4*>(a1 + 4) = x1;
+    }
+    for (int k = 1; k + 1 < S; ++k) {
+        const float* lr = Lst + off0 + k * seg + (int64_t)i * kSplitD + c0;
+        const float4 l0 = *reinterpret_cast<const float4*>(lr);
+        const float4 l1 = *reinterpret_cast<const float4*>(lr + 4);
+        if (k + 2 < S) {
+            // buffer (k & 1) was last read in step k - 1, which ended with a barrier
+            stage_phi(phi_s + (k & 1) * kSplitD * kPhiLd, Phi + off0 + (k + 1) * seg);
+            cp_async_wait_group1();  // Phi_k is in; Phi_{k+1} may still be in flight
+        } else {
+            cp_async_wait_all_groups();
+        }
+        __syncthreads();  // Phi_k and cur visible to every thread
+        const float* pr = phi_s + ((k - 1) & 1) * kSplitD * kPhiLd + i * kPhiLd;  // row i of Phi_k
+        float2 acc[4] = {make_float2(l0.x, l0.y), make_float2(l0.z, l0.w), make_float2(l1.x, l1.y),
+                         make_float2(l1.z, l1.w)};
+#pragma unroll 4
+        for (int m = 0; m < kSplitD; m += 4) {
+            const float4 p4 = *reinterpret_cast<const float4*>(pr + m);
+            const float phi[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+            for (int mm = 0; mm < 4; ++mm) {
+                const float2 f = make_float2(phi[mm], phi[mm]);
+                const float4 s0 = *reinterpret_cast<const float4*>(cur + (m + mm) * kCombCols + cl);
+                const float4 s1 = *reinterpret_cast<const float4*>(cur + (m + mm) * kCombCols + cl + 4);
+                acc[0] = __ffma2_rn(f, make_float2(s0.x, s0.y), acc[0]);
+                acc[1] = __ffma2_rn(f, make_float2(s0.z, s0.w), acc[1]);
+                acc[2] = __ffma2_rn(f, make_float2(s1.x, s1.y), acc[2]);
+                acc[3] = __ffma2_rn(f, make_float2(s1.z, s1.w), acc[3]);
+            }
+        }
+        __syncthreads();  // every thread has read cur and Phi_k
+        const float4 a0 = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
+        const float4 a1 = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
+        *reinterpret_cast<float4*>(cur + i * kCombCols + cl) = a0;
+        *reinterpret_cast<float4*>(cur + i * kCombCols + cl + 4) = a1;
+        float* an = A + off0 + (k + 1) * seg + (int64_t)i * kSplitD + c0;
+        *reinterpret_cast<float4*>(an) = a0;
+        *reinterpret_cast<float4*>(an + 4) = a1;
+    }
+}
+
+// hT[n] <- the final state of sequence n's last segment (pass 2's output).
+__global__ void split_final_kernel(const float* B, int N, int H, int S, float* hT) {
+    const int64_t n4 = (int64_t)N * H * kStateFloats / 4;
+    for (int64_t e4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e4 < n4;
+         e4 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e = 4 * e4;
+        const int64_t nh = e / kStateFloats, within = e % kStateFloats;
+        const int64_t n = nh / H, h = nh % H;
+        reinterpret_cast<float4*>(hT)[e4] =
+            *reinterpret_cast<const float4*>(B + ((n * S + S - 1) * H + h) * kStateFloats + within);
+    }
+}
+
+int sm_count() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+}  // namespace
+
+int prefill_split_segments(int N, int64_t T_tot, int H, int dk, int dv, int chunk) {
+    if (N <= 0 || T_tot <= 0 || dk != kSplitD || dv != kSplitD || chunk != 64) return 1;
+    const int64_t units = (int64_t)N * H;
+    int64_t S = sm_count() / units;  // segments per sequence that still fit one wave
+    const int64_t by_len = T_tot / N / 64 / kMinSegmentChunks;
+    if (by_len < S) S = by_len;
+    if (S > kMaxSegments) S = kMaxSegments;
+    return S >= kMinSegments ? (int)S : 1;
+}
+
+size_t prefill_split_workspace_bytes(int N, int64_t T_tot, int H, int S) {
+    return split_layout(N, T_tot, H, S).total;
+}
+
+cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, cudaStream_t s) {
+    const SplitLayout l = split_layout(a.N, a.T_tot, a.H, S);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* cu_seg = reinterpret_cast<int32_t*>(ws + l.cu_off);
+    float* A = reinterpret_cast<float*>(ws + l.a_off);
+    float* B = reinterpret_cast<float*>(ws + l.b_off);
+    float* Lst = reinterpret_cast<float*>(ws + l.l_off);
+    float* Phi = reinterpret_cast<float*>(ws + l.r_off);
+    void* zeros_v = ws + l.zv_off;
+    const int NS = a.N * S;
+    const int fill_blocks = 4 * sm_count();
+
+    split_bounds_kernel<<<(NS + 1 + 255) / 256, 256, 0, s>>>(a.cu, a.N, S, cu_seg);
+    split_fill_kernel<<<fill_blocks, 256, 0, s>>>(a.h0, a.N, a.H, S, A, B);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(zeros_v, 0, (size_t)a.T_tot * a.H * kSplitD * 2, s)) != cudaSuccess) return e;
+
+    PrefillArgs p = a;
+    p.cu = cu_seg;
+    p.N = NS;
+    p.order = reinterpret_cast<int32_t*>(ws + l.base.order_off);
+    p.counter = reinterpret_cast<int32_t*>(ws + l.base.counter_off);
+    auto pass = [&](const float* h0, float* hT) {
+        p.h0 = h0;
+        p.hT = hT;
+        cudaError_t err = launch_prefill_schedule(p, s);
+        return err != cudaSuccess ? err : launch_prefill_tc(p, s);
+    };
+    if ((e = pass(a.h0 ? A : nullptr, Lst)) != cudaSuccess) return e;  // 1a
+    p.v = zeros_v;
+    p.ld_v = (int64_t)a.H * kSplitD;
+    e = pass(B, Phi);  // 1b
+    p.v = a.v;
+    p.ld_v = a.ld_v;
+    if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(split_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kCombSmem)) != cudaSuccess)
+        return e;
+    split_combine_kernel<<<dim3((unsigned)(a.N * a.H), kSplitD / kCombCols), kCombThreads, kCombSmem, s>>>(
+        a.N, a.H, S, Lst, Phi, A);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = pass(A, a.hT ? B : nullptr)) != cudaSuccess) return e;  // 2
+    if (a.hT) {
+        split_final_kernel<<<fill_blocks, 256, 0, s>>>(B, a.N, a.H, S, a.hT);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace gdn

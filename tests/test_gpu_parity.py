@@ -738,6 +738,38 @@ def test_layer_0p8b_conv_then_prefill():
     assert err(host(hT), h_ref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("lengths,H,Hk,undecayed,with_h0,in_place", [
+    ([3000, 0, 1400, 4200], 2, 1, False, True, True),
+    ([4096], 8, 8, True, False, False),
+    ([640, 9000], 2, 2, False, True, False),
+])
+def test_prefill_sequence_split(lengths, H, Hk, undecayed, with_h0, in_place):
+    """Few (sequence, head) units: the sequences are cut into segments (zero-
+    and identity-start passes, the fp32 chain of segment start states, then
+    the output pass). Every element against the oracle, and against the plain
+    launch, which a workspace of only the schedule's size selects. Covers an
+    empty sequence, sequences with fewer chunks than segments, grouped heads,
+    the read-before-decay order and hT == h0 in place."""
+    P = gi.random_prefill(61 + H, lengths, H=H, dk=128, dv=128, with_h0=with_h0, Hk=Hk)
+    assert gdn.prefill_workspace_size(P.N, P.T_tot, H, 128, 128) > 256 + 4 * P.N + 255  # splits
+    q, k, v = (dev_tensor(a, "bf16") for a in (P.q, P.k, P.v))
+    g, beta = dev_tensor(P.g, "f32"), dev_tensor(P.beta, "f32")
+    cu = torch.from_numpy(P.cu_seqlens.astype(np.int32)).to(DEV)
+    h0 = dev_tensor(P.h0, "f32") if with_h0 else None
+    h0_copy = None if h0 is None else h0.clone()
+    o, hT = gdn.prefill(q, k, v, g, beta, cu, initial_state=h0, undecayed=undecayed,
+                        final_state=h0 if in_place else None)
+    gdn.check_device_status(DEV)
+    base_ws = torch.empty(256 + (4 * P.N + 255) // 256 * 256, dtype=torch.uint8, device=DEV)
+    o1, h1 = gdn.prefill(q, k, v, g, beta, cu, initial_state=h0_copy, undecayed=undecayed,
+                         workspace=base_ws)
+    gdn.check_device_status(DEV)
+    o_ref, h_ref = prefill_oracle(P, undecayed=undecayed)
+    assert err(host(o), o_ref) <= TOL_BF16 and err(host(hT), h_ref) <= TOL_BF16
+    assert err(host(o1), o_ref) <= TOL_BF16 and err(host(h1), h_ref) <= TOL_BF16
+    assert err(host(o), host(o1)) <= TOL_BF16
+
+
 def _check_sequences(P, seqs, o, hT):
     worst = 0.0
     for n in seqs:
