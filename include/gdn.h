@@ -133,9 +133,17 @@ GDN_API gdn_status_t gdn_conv_silu(const void* x, gdn_dtype_t dtype, const void*
                            void* y, void* stream);
 
 /*
- * Bytes of device workspace gdn_prefill needs for this problem (a multiple of
- * 256; never 0). The workspace holds the work schedule (sequences ordered
- * longest first) and a work counter; it is rewritten by every call.
+ * Bytes of device workspace gdn_prefill needs for this problem on the current
+ * device (a multiple of 256; never 0). The workspace holds the work schedule
+ * (sequences ordered longest first) and a work counter; it is rewritten by
+ * every call. When the (sequence, head) units are too few to fill the device
+ * (bf16, dk = dv = 128, chunk 64, N * H at most a sixth of the SM count and
+ * long enough sequences), the size also covers the sequence split: each
+ * sequence is cut into S segments run as three tensor-core passes (zero and
+ * identity initial states, then the true ones) with an fp32 hand-off of the
+ * segment start states between them, about 4 * N * S * H * dk * dv * 4 bytes
+ * plus a zero value buffer of T_tot * H * dv bf16. A workspace of only
+ * 256 + 4 * N bytes (rounded up to 256) runs the plain single pass instead.
  */
 GDN_API size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, int chunk);
 
