@@ -19,7 +19,9 @@
 //
 // Layout: thread (rg, cg) holds rows [rg*RPT, rg*RPT+RPT) x columns [4cg, 4cg+4)
 // of S_{t-1} and of dS in registers; sums over rows go through `red`
-// [RG][dv], sums over columns through `redr` [dk][dv/4].
+// [RG][dv], sums over columns through `redr` [dk][dv/4 + 1] (the extra column
+// keeps the threads that add up one row each on distinct banks), and the
+// per-thread terms of dg through `gps` [threads].
 #include "common.cuh"
 #include "launch.h"
 
@@ -50,9 +52,11 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
     float* dmm = dl + dv;        // [dv] dm
     float* dbt = dmm + dv;       // [dv] ddelta (v - m)
     float* red = dbt + dv;       // [RG][dv]
-    float* redr = red + RG * dv; // [dk][cols4]
-    float* scal = redr + dk * cols4;  // [16]: a, beta, |q|, |k|, delta.do, k^.dk^, q~.dq~, <dS', Sp>,
-                                      //       g, beta as loaded
+    const int ldr = cols4 + 1;
+    float* redr = red + RG * dv; // [dk][ldr]
+    float* scal = redr + dk * ldr;  // [16]: a, beta, |q|, |k|, delta.do, k^.dk^, q~.dq~, -,
+                                    //       g, beta as loaded
+    float* gps = scal + 16;         // [threads]
 
     const int64_t start = a.cu[n], end = a.cu[n + 1];
     const int64_t ck_base = 2 * (int64_t)n + (start + kCk - 1) / kCk;  // first checkpoint slot
@@ -74,21 +78,50 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
 #pragma unroll
         for (int r = 0; r < RPT; ++r) *reinterpret_cast<float4*>(base + (int64_t)(i0 + r) * dv + j0) = x[r];
     };
-    // Token t's k^ (and q~, do when `full`), v, a, beta into shared memory.
-    auto load_token = [&](int64_t t, bool full) {
+    // Token t's k^ (and q~, do when `full`), v, a, beta into shared memory. A
+    // thread holds at most one element of each vector (the CTA has at least
+    // max(dk, dv) threads), and the next token's elements are requested into
+    // registers while the current token is worked on: the guess is t + 1 in the
+    // forward passes and t - 1 in the reverse sweep; a wrong guess (once per
+    // block of kCk tokens) just loads again.
+    struct Pref {
+        float k, q, v, d, g, b;
+        int64_t t;
+        bool full;
+    } pf{0.f, 0.f, 0.f, 0.f, 0.f, 0.f, -1, false};
+    auto issue = [&](int64_t t, bool full) {
+        pf.t = t;
+        pf.full = full;
+        if (t < start || t >= end) return;
+        if (tid < dk) {
+            pf.k = Elem<T>::load(k, (t * Hk + hk) * dk + tid);
+            if (full) pf.q = Elem<T>::load(q, (t * Hk + hk) * dk + tid);
+        }
+        if (tid < dv) {
+            pf.v = Elem<T>::load(v, (t * H + h) * dv + tid);
+            if (full) pf.d = a.dO[(t * H + h) * dv + tid];
+        }
+        if (tid == 0) {
+            pf.g = a.g[t * H + h];
+            pf.b = a.beta[t * H + h];
+        }
+    };
+    auto load_token = [&](int64_t t, bool full, int64_t t_next, bool full_next) {
+        if (pf.t != t || pf.full != full) issue(t, full);
         __syncthreads();  // the previous token's values are no longer read
-        if (tid == 0) {  // the gates travel with the vectors (one round trip per token)
-            scal[8] = a.g[t * H + h];
-            scal[9] = a.beta[t * H + h];
+        if (tid == 0) {
+            scal[8] = pf.g;
+            scal[9] = pf.b;
         }
-        for (int i = tid; i < dk; i += blockDim.x) {
-            kh[i] = Elem<T>::load(k, (t * Hk + hk) * dk + i);
-            if (full) qn[i] = Elem<T>::load(q, (t * Hk + hk) * dk + i);
+        if (tid < dk) {
+            kh[tid] = pf.k;
+            if (full) qn[tid] = pf.q;
         }
-        for (int j = tid; j < dv; j += blockDim.x) {
-            vv[j] = Elem<T>::load(v, (t * H + h) * dv + j);
-            if (full) dov[j] = a.dO[(t * H + h) * dv + j];
+        if (tid < dv) {
+            vv[tid] = pf.v;
+            if (full) dov[tid] = pf.d;
         }
+        issue(t_next, full_next);
         __syncthreads();
         if (warp == 0) {
             float sk = 0.f, sq = 0.f;
@@ -129,7 +162,7 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
         const float4 w4 = *reinterpret_cast<const float4*>(w + j0);
 #pragma unroll
         for (int r = 0; r < RPT; ++r)
-            redr[(i0 + r) * cols4 + cg] = x[r].x * w4.x + x[r].y * w4.y + x[r].z * w4.z + x[r].w * w4.w;
+            redr[(i0 + r) * ldr + cg] = x[r].x * w4.x + x[r].y * w4.y + x[r].z * w4.z + x[r].w * w4.w;
     };
     auto col_total = [&](int j) {
         float s = 0.f;
@@ -138,12 +171,12 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
     };
     auto row_total = [&](int i) {
         float s = 0.f;
-        for (int c = 0; c < cols4; ++c) s += redr[i * cols4 + c];
+        for (int c = 0; c < cols4; ++c) s += redr[i * ldr + c];
         return s;
     };
     // One forward token on the register tile S (the state before token t).
     auto forward_step = [&](int64_t t, float4 (&S)[RPT]) {
-        load_token(t, false);
+        load_token(t, false, t + 1, false);
         col_partial(S);
         __syncthreads();
         const float al = scal[0], be = scal[1];
@@ -186,7 +219,7 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
             __syncthreads();  // buf writes (and the previous token's reads) are done
             float4 Sp[RPT];
             load_tile(buf + (t - c0) * DD, Sp);
-            load_token(t, true);
+            load_token(t, true, t - 1, true);
             const float al = scal[0], be = scal[1];
             // A: m = a Sp^T k^, delta; r = Sp do
             col_partial(Sp);
@@ -198,7 +231,6 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
                 dl[j] = be * (vv[j] - m);
             }
             for (int i = tid; i < dk; i += blockDim.x) rr[i] = row_total(i);
-            if (tid == 0) scal[7] = 0.f;
             __syncthreads();
             // B: dS += q^ do^T; ddelta = dS^T k^; dk^ = dS delta
             const float sc = a.scale;
@@ -238,21 +270,23 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
                 }
             }
             // (the CTA may end in a partial warp, so no shuffles outside warp 0)
-            atomicAdd(scal + 7, gp);
+            gps[tid] = gp;
             __syncthreads();
             for (int i = tid; i < dk; i += blockDim.x) dkh[i] += al * row_total(i);
             if (warp == 0) {
-                float dd = 0.f, db = 0.f;
+                float dd = 0.f, db = 0.f, gsum = 0.f;
                 for (int j = lane; j < dv; j += 32) {
                     dd += dl[j] * dov[j];
                     db += dbt[j];
                 }
+                for (int x = lane; x < (int)blockDim.x; x += 32) gsum += gps[x];
                 dd = warp_sum(dd);
                 db = warp_sum(db);
+                gsum = warp_sum(gsum);
                 if (lane == 0) {
                     scal[4] = dd;
                     a.dbeta[t * H + h] = db;
-                    a.dg[t * H + h] = al * scal[7];
+                    a.dg[t * H + h] = al * gsum;
                 }
             }
             __syncthreads();
@@ -295,7 +329,7 @@ template <typename T, int RPT>
 cudaError_t launch_rpt(const BackwardArgs& a, cudaStream_t s) {
     const int cols4 = a.dv / 4, RG = a.dk / RPT;
     const int threads = cols4 * RG;
-    const size_t smem = sizeof(float) * (5 * a.dk + 6 * a.dv + RG * a.dv + a.dk * cols4 + 16);
+    const size_t smem = sizeof(float) * (5 * a.dk + 6 * a.dv + RG * a.dv + a.dk * (cols4 + 1) + 16 + threads);
     backward_kernel<T, RPT><<<(unsigned)((int64_t)a.N * a.H), threads, smem, s>>>(a);
     return cudaGetLastError();
 }
