@@ -491,13 +491,18 @@ def bench_varlen(args, dist, pk):
     flops = T * H * FLOP_PER_TOKEN_HEAD
     byts = T * H * BYTES_PER_TOKEN_HEAD + 2 * N * H * STATE_BYTES
     # per-CTA work of the tensor-core kernel: (sequence, head) units in longest-first
-    # order, unit u on CTA u mod grid
+    # order; CTA c starts with unit c and each later unit goes to the CTA that runs
+    # out of work first (the kernel's work counter), emulated in tokens
+    import heapq
     lens = np.diff(host_cu.numpy().astype(np.int64))
     order = sorted(range(N), key=lambda n: (-int(lens[n]), n))
     grid = min(torch.cuda.get_device_properties(dev).multi_processor_count, N * H)
     work = np.zeros(grid)
+    heap = []
     for u in range(N * H):
-        work[u % grid] += lens[order[u // H]]
+        c = u if u < grid else heapq.heappop(heap)[1]
+        work[c] += lens[order[u // H]]
+        heapq.heappush(heap, (work[c], c))
     return {"value": T / (ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": ms,
             "workload": f"varlen_64seqs_{T}tok_h16_d128_bf16_h0",
             "tc_roofline": {"achieved": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",

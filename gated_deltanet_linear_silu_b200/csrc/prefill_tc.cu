@@ -100,7 +100,9 @@ constexpr uint32_t kVecBytes = 2176;
 constexpr uint32_t kOffOf = kOffVec + kStages * kVecBytes;  // output row factors, 2 x 64 fp32
 constexpr uint32_t kOffBar = kOffOf + 2 * 64 * 4;
 constexpr uint32_t kOffMisc = kOffBar + 512;
-constexpr uint32_t kSmemBytes = kOffMisc + 64;
+constexpr int kRing = 16;                            // unit ring: [kRing] x (unit, ordinal tag)
+constexpr uint32_t kOffRing = kOffMisc + 64;
+constexpr uint32_t kSmemBytes = kOffRing + kRing * 8;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(kOffP % 1024 == 0 && kOffT1 % 1024 == 0 && kOffWT % 1024 == 0, "swizzle alignment");
@@ -249,16 +251,63 @@ __device__ __forceinline__ bool load_unit_checked(const PrefillArgs& a, int u, U
     return U.start >= 0 && U.start <= U.end && U.end <= a.T_tot;
 }
 
-// The CTA's work list: the 64-token chunks of its units u = blockIdx.x +
-// k * gridDim.x < n_work * H, in order (the schedule puts the sequences that
-// have tokens first). Every role walks the same list.
+// The CTA's work list: the 64-token chunks of its units, in order. The first
+// unit is u = blockIdx.x; each later one is taken from the work counter when
+// the producer reaches it (units in longest-first order, the sequences with
+// tokens first), so a CTA whose units are short takes more of them. The
+// producer publishes the k-th unit of the CTA in slot k % kRing of a ring in
+// shared memory (the unit, then the ordinal k as its tag); every other role
+// reads the slot once the tag shows k. No role trails the producer by kRing
+// units: the stage ring keeps them within a few chunks. Every role walks the
+// same list.
 struct Item {
     int u;
+    int k;  // ordinal of the unit within this CTA
     Unit U;
     int64_t c0;
     int L;
     bool first, last;
 };
+
+struct UnitRing {
+    volatile int* slot;  // [kRing][2]
+    int* counter;        // work counter (the schedule zeroes it)
+    int* status;
+    volatile int* abort_flag;
+    uint64_t wlim;
+    bool producer;
+};
+
+// The k-th (k >= 1) unit of this CTA, or -1 past the last. A reader whose wait
+// runs out (or sees another role's abort) records the timeout and gets -1.
+// Scalar arguments: the one copy of the wait loop serves every call site.
+__device__ __noinline__ int ring_unit(volatile int* slot, int* counter, int* status, volatile int* abort_flag,
+                                      uint64_t wlim, bool producer, int k, int units) {
+    volatile int* e = slot + 2 * (k % kRing);
+    if (producer) {
+        const int u = (int)gridDim.x + atomicAdd(counter, 1);
+        const int v = u < units ? u : -1;
+        e[0] = v;
+        __threadfence_block();
+        e[1] = k;
+        return v;
+    }
+    if (e[1] != k) {
+        const uint64_t t0 = globaltimer_ns();
+        while (e[1] != k) {
+            if (*abort_flag || globaltimer_ns() - t0 >= wlim) {
+                if (!*abort_flag) {
+                    *abort_flag = 1;
+                    set_status(status, kStatusTimeout);
+                }
+                return -1;
+            }
+            __nanosleep(64);
+        }
+    }
+    __threadfence_block();
+    return e[0];
+}
 
 __device__ __forceinline__ void item_unit(const PrefillArgs& a, Item& it) {
     it.U.h = it.u % a.H;
@@ -274,17 +323,20 @@ __device__ __forceinline__ void item_len(Item& it) {
 }
 __device__ __forceinline__ bool item_first(const PrefillArgs& a, int units, Item& it) {
     it.u = blockIdx.x;
+    it.k = 0;
     if (it.u >= units) return false;
     item_unit(a, it);
     item_len(it);
     return true;
 }
-__device__ __forceinline__ bool item_next(const PrefillArgs& a, int units, Item& it) {
+__device__ __forceinline__ bool item_next(const PrefillArgs& a, int units, Item& it, const UnitRing& ring) {
     it.c0 += kC;
     it.first = false;
     if (it.c0 >= it.U.end) {
-        it.u += gridDim.x;
-        if (it.u >= units) return false;
+        it.k += 1;
+        it.u = ring_unit(ring.slot, ring.counter, ring.status, ring.abort_flag, ring.wlim, ring.producer, it.k,
+                         units);
+        if (it.u < 0) return false;
         item_unit(a, it);
     }
     item_len(it);
@@ -384,6 +436,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     Bars& B = *reinterpret_cast<Bars*>(sm + kOffBar);
     uint32_t* tmem_base_p = reinterpret_cast<uint32_t*>(sm + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+    // the unit ring; only the producer (warp 0, lane 0) takes units from the counter
+    const UnitRing ring{reinterpret_cast<volatile int*>(sm + kOffRing), a.counter, a.status, abort_flag, wlim,
+                        warp == kWarpTma && lane == 0};
     float* sA = reinterpret_cast<float*>(sm + kOffA);
     uint8_t* sT1 = sm + kOffT1;
     uint8_t* sT2 = sm + kOffT2;
@@ -418,6 +473,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         mbar_init(&B.drain_state, 1);
         fence_mbar_init();
         *abort_flag = 0;
+        for (int e = 0; e < kRing; ++e) ring.slot[2 * e + 1] = -1;
     }
     if (warp == 0) tmem_alloc(tmem_base_p, kTmemCols);
     tc_fence_before();
@@ -444,7 +500,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             uint32_t issued = 0, issued_par = 0;  // last load per stage, for the drain
             Item it;
             bool have = item_first(a, units, it);
-            for (int i = 0; have; ++i, have = item_next(a, units, it)) {
+            for (int i = 0; have; ++i, have = item_next(a, units, it, ring)) {
                 const int s = i % kStages, k = i / kStages;
                 if (!mbar_wait_or_abort(&B.empty[s], (k & 1) ^ 1, abort_flag, wlim)) {
                     fail();
@@ -489,14 +545,14 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             };
             if (have_g) {
                 ok = gram();
-                have_g = item_next(a, units, git);
+                have_g = item_next(a, units, git, ring);
             }
             // The next chunk's Gram goes out before this chunk's W, so the Gram
             // epilogue of chunk i + 1 can follow the solve of chunk i at once.
-            for (int i = 0; ok && have_w; ++i, have_w = item_next(a, units, wit)) {
+            for (int i = 0; ok && have_w; ++i, have_w = item_next(a, units, wit, ring)) {
                 if (have_g) {
                     if (!(ok = gram())) break;
-                    have_g = item_next(a, units, git);
+                    have_g = item_next(a, units, git, ring);
                 }
                 // W^T = K^T T1 -> R_W ; U~^T = V^T T2 -> R_U[i & 1]
                 const int s = i % kStages, b = i & 1;
@@ -529,7 +585,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             bool ok = true;
             Item it;
             bool have = item_first(a, units, it);
-            for (int i = 0; have; ++i, have = item_next(a, units, it)) {
+            for (int i = 0; have; ++i, have = item_next(a, units, it, ring)) {
                 const int s = i % kStages, b = i & 1;
                 const uint8_t* st = stage(s);
                 if (!mbar_wait_or_abort(&B.wt_ready, i & 1, abort_flag, wlim) ||
@@ -590,7 +646,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         // ============================================================== gates
         Item it;
         bool have = item_first(a, units, it);
-        for (int i = 0; have; ++i, have = item_next(a, units, it)) {
+        for (int i = 0; have; ++i, have = item_next(a, units, it, ring)) {
             const int s = i % kStages, k = i / kStages;
             const int L = it.L;
             // gates of rows 2*lane, 2*lane+1 (g = beta = 0 past the chunk's end)
@@ -649,7 +705,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         const int gtid = tid - 32 * kWg1;  // 0..127
         Item it;
         bool have = item_first(a, units, it);
-        for (int i = 0; have; ++i, have = item_next(a, units, it)) {
+        for (int i = 0; have; ++i, have = item_next(a, units, it, ring)) {
             const int s = i % kStages, k = i / kStages;
             const int L = it.L;
             float* vec = vecp(s);
@@ -958,7 +1014,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             have_prev = have;
             if (have) {
                 prev = it;
-                have = item_next(a, units, it);
+                have = item_next(a, units, it, ring);
             }
         }
     } else {
@@ -981,7 +1037,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         float E = 1.f;
         Item it;
         bool have = item_first(a, units, it);
-        for (int i = 0; have; ++i, have = item_next(a, units, it)) {
+        for (int i = 0; have; ++i, have = item_next(a, units, it, ring)) {
             const int s = i % kStages, k = i / kStages, b = i & 1;
             const int64_t sbase = ((int64_t)it.U.n * H + it.U.h) * kD * kD;
             if (it.first) {
