@@ -569,7 +569,8 @@ def bench_decode_layer(args, dist, pk):
 def bench_grouped(args, dist, pk):
     """Grouped value heads: 32 value heads on 16 q, k heads, d=128. The prefill
     of 8 sequences x 8192 tokens (fp32 final state), and the whole-mixer decode
-    step for 256 sequences (one two-CTA cluster per q, k head), 100 steps."""
+    step for 256 sequences (a CTA runs the two value heads of a q, k head back
+    to back), 100 steps."""
     import numpy as np
     import torch
     import gated_deltanet_linear_silu_b200 as gdn
@@ -648,7 +649,7 @@ def bench_grouped(args, dist, pk):
            "roofline": {"bound": "hbm", "achieved": bytes_step / (step_ms * 1e-3) / 1e9,
                         "peak": pk["hbm_gbs"], "unit": "GB/s",
                         "frac": bytes_step / (step_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                        "traffic": profiled_traffic("decode_layer_grouped_kernel", ["decode.cu"],
+                        "traffic": profiled_traffic("decode_layer_grouped_kernel", ["decode_stream.cu"],
                                                     Nd * Hv),
                         "algorithmic_bytes": bytes_step},
            "gpu_launches": steps}

@@ -281,7 +281,7 @@ gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv
     if (!dtype_ok(dtype) || N < 0 || H <= 0 || K < 1 || Hk < 0 || H % Hk != 0)
         return GDN_ERR_INVALID_ARG;
     if (undecayed != 0 && undecayed != 1) return GDN_ERR_INVALID_ARG;
-    if (K > 4 || H / Hk > gdn::kMaxDecodeGroup) return GDN_ERR_UNSUPPORTED;
+    if (K > 4) return GDN_ERR_UNSUPPORTED;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (N == 0) return GDN_OK;
     if (!x || !conv_w || !g || !beta || !state || !o || (K > 1 && !conv_state))

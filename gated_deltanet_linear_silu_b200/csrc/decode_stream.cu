@@ -15,8 +15,11 @@
 // first applies the causal conv update of its head's q, k, v channels ("7.6
 // Qwen3.5: linear-attention hybrid", 7.6.2; conv state = the K-1 latest
 // inputs) and SiLU; with a gate z the output goes through the gated RMSNorm.
-// Value heads that share q, k heads (grouped) keep the per-(sequence, head)
-// kernel, whose clusters share the q, k conv channels.
+// With grouped value heads (H = G Hk, value head h reading q, k head h / G)
+// a CTA takes whole groups: the G units of (sequence, q/k head) run back to
+// back, the first one computes the shared q, k channels' conv (and shifts
+// their conv state: this CTA is the only reader), the others reuse q, k and
+// their norms from shared memory and bring in only their own v channels.
 //
 // Thread (rg, cg) owns columns [4cg, 4cg+4) of rows [rg*RPT, rg*RPT+RPT). The
 // squared norms of q and k and their dot product are summed in the phase that
@@ -75,16 +78,20 @@ Geometry geometry(const DecodeArgs& a, int rpt) {
     return g;
 }
 
-// Issue the bulk copies of unit u into the slot (one thread).
+// Issue the bulk copies of unit u (value head h of sequence n) into the slot
+// (one thread): the state, the v channels' conv inputs, z, and with `qk` also
+// the conv inputs of the q, k channels of the head's q/k group.
 template <typename T>
-__device__ __forceinline__ void load_unit(const DecodeArgs& a, const Geometry& geo, uint8_t* sl, int64_t u,
+__device__ __forceinline__ void load_unit(const DecodeArgs& a, const Geometry& geo, uint8_t* sl, int u, bool qk,
                                           uint64_t* full) {
-    const int dk = a.dk, dv = a.dv, H = a.H, K = a.K;
+    const int dk = a.dk, dv = a.dv, H = a.H, Hk = a.Hk, K = a.K;
     const int nconv = 2 * dk + dv;
-    mbar_arrive_expect_tx(full, geo.state_bytes + geo.in_bytes);
-    bulk_load(sl, a.state + u * dk * dv, geo.state_bytes, full);
-    const int n = (int)(u / H), h = (int)(u % H);
-    const int64_t C = 2 * (int64_t)H * dk + (int64_t)H * dv;
+    const int esz = (int)sizeof(T);
+    const uint32_t v_bytes = (uint32_t)(dv * 2 * K * esz), qk_bytes = (uint32_t)(2 * dk * 2 * K * esz);
+    mbar_arrive_expect_tx(full, geo.state_bytes + v_bytes + (qk ? qk_bytes : 0u) + (a.z ? dv * esz : 0));
+    bulk_load(sl, a.state + (int64_t)u * dk * dv, geo.state_bytes, full);
+    const int n = u / H, h = u % H, hk = h / (H / Hk);
+    const int64_t C = 2 * (int64_t)Hk * dk + (int64_t)H * dv;
     const T* x = static_cast<const T*>(a.x) + n * C;
     const T* w = static_cast<const T*>(a.conv_w);
     const T* cs = static_cast<const T*>(a.conv_state) + n * C * (K - 1);
@@ -92,15 +99,15 @@ __device__ __forceinline__ void load_unit(const DecodeArgs& a, const Geometry& g
     T* cw = cx + nconv;
     T* ccs = cw + nconv * K;
 #pragma unroll
-    for (int b = 0; b < 3; ++b) {  // q, k, v channel blocks of the head
+    for (int b = qk ? 0 : 2; b < 3; ++b) {  // q, k, v channel blocks
         const int nb = b < 2 ? dk : dv;
-        const int64_t ch0 = b == 0 ? (int64_t)h * dk : (b == 1 ? (int64_t)H * dk + h * dk : 2 * (int64_t)H * dk + h * dv);
+        const int64_t ch0 = b == 0 ? (int64_t)hk * dk : (b == 1 ? (int64_t)Hk * dk + hk * dk : 2 * (int64_t)Hk * dk + h * dv);
         const int c0 = b == 0 ? 0 : (b == 1 ? dk : 2 * dk);
-        bulk_load(cx + c0, x + ch0, nb * sizeof(T), full);
-        bulk_load(cw + c0 * K, w + ch0 * K, nb * K * sizeof(T), full);
-        if (K > 1) bulk_load(ccs + c0 * (K - 1), cs + ch0 * (K - 1), nb * (K - 1) * sizeof(T), full);
+        bulk_load(cx + c0, x + ch0, nb * esz, full);
+        bulk_load(cw + c0 * K, w + ch0 * K, nb * K * esz, full);
+        if (K > 1) bulk_load(ccs + c0 * (K - 1), cs + ch0 * (K - 1), nb * (K - 1) * esz, full);
     }
-    if (a.z) bulk_load(sl + geo.z_off, static_cast<const T*>(a.z) + u * dv, dv * sizeof(T), full);
+    if (a.z) bulk_load(sl + geo.z_off, static_cast<const T*>(a.z) + (int64_t)u * dv, dv * esz, full);
 }
 
 // Causal conv of one channel (local index c of the slot's nconv) against its
@@ -135,8 +142,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
     const int nthr = cols4 * RG;  // threads with state rows (<= kThreads)
     const int cg = tid % cols4, rg = tid / cols4;
     const int nconv = 2 * dk + dv;
-    const int64_t total = (int64_t)a.N * a.H;
-    const int H = a.H, K = a.K;
+    const int H = a.H, Hk = a.Hk, G = H / Hk, K = a.K;
+    // units u = n H + h (N H < 2^31) in group order: the CTA takes groups
+    // blockIdx.x, blockIdx.x + gridDim.x, ... (a group is (sequence, q/k head),
+    // its G value heads are units group G + g, g = 0 .. G-1); -1 past the last
+    const int total = a.N * H;
+    const int skip = (int)(gridDim.x - 1) * G;  // from a group's last unit to the next group's first
 
     const float* Ss = reinterpret_cast<const float*>(sl);
     const T* cx = reinterpret_cast<const T*>(sl + geo.state_bytes);  // [nconv]
@@ -149,14 +160,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
     float4* part = reinterpret_cast<float4*>(red + 2 * RG * dv);  // [kWarps]: |q|^2, |k|^2, q.k
     uint64_t* full = reinterpret_cast<uint64_t*>(part + kWarps);
 
-    int64_t u = blockIdx.x;
+    int u = (int)blockIdx.x * G < total ? (int)blockIdx.x * G : -1;
+    int gpos = 0;  // u's position in its group
     if (tid == 0) {
         mbar_init(full, 1);
         fence_mbar_init();
-        if (u < total) load_unit<T>(a, geo, sl, u, full);
+        if (u >= 0) load_unit<T>(a, geo, sl, u, true, full);
     }
     float g_next = 0.f, b_next = 0.f;  // gate and beta one unit ahead
-    if (u < total) {
+    if (u >= 0) {
         g_next = a.g[u];
         b_next = a.beta[u];
     }
@@ -164,12 +176,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
     if (a.z && tid < cols4) nw4 = *reinterpret_cast<const float4*>(a.norm_w + 4 * cg);
     __syncthreads();
 
-    bool in_flight = u < total;
-    for (int i = 0; u < total; u += gridDim.x, ++i) {
+    bool in_flight = u >= 0;
+    int i = 0;
+    for (; u >= 0; ++i) {
         const float alpha = expf(g_next);
         const float beta = b_next;
-        const int64_t un = u + gridDim.x;
-        if (un < total) {
+        const bool first = gpos == 0;  // the group's first unit: q, k conv
+        const int gpos_n = gpos + 1 == G ? 0 : gpos + 1;
+        const int64_t un64 = (int64_t)u + 1 + (gpos_n == 0 ? skip : 0);
+        const int un = un64 < total ? (int)un64 : -1;
+        if (un >= 0) {
             g_next = a.g[un];
             b_next = a.beta[un];
         }
@@ -180,17 +196,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
                 break;
             }
         }
-        // conv update + SiLU of q, k, v into fp32 shared memory; item j < dk
-        // makes q_j and k_j and sums their squares and product
-        float sq = 0.f, sk = 0.f, kq = 0.f;
+        // conv update + SiLU into fp32 shared memory: the v channels, and in the
+        // group's first unit the q, k channels too (item j < dk makes q_j and k_j
+        // and sums their squares and product); later units of the group keep
+        // q, k and the norm partials
         {
-            const int n = (int)(u / H), h = (int)(u % H);
-            const int64_t C = 2 * (int64_t)H * dk + (int64_t)H * dv;
+            const int n = u / H, h = u % H, hk = h / G;
+            const int64_t C = 2 * (int64_t)Hk * dk + (int64_t)H * dv;
             T* cs = static_cast<T*>(a.conv_state) + n * C * (K - 1);
-            for (int j = tid; j < dk + dv; j += kThreads) {
+            const int j0 = first ? 0 : dk;
+            float sq = 0.f, sk = 0.f, kq = 0.f;
+            for (int j = j0 + tid; j < dk + dv; j += kThreads) {
                 if (j < dk) {
-                    const float qv = conv_channel(cx, cw, ccs, cs, j, (int64_t)h * dk + j, K);
-                    const float kv = conv_channel(cx, cw, ccs, cs, dk + j, (int64_t)H * dk + h * dk + j, K);
+                    const float qv = conv_channel(cx, cw, ccs, cs, j, (int64_t)hk * dk + j, K);
+                    const float kv = conv_channel(cx, cw, ccs, cs, dk + j, (int64_t)Hk * dk + hk * dk + j, K);
                     qs[j] = qv;
                     ks[j] = kv;
                     sq = fmaf(qv, qv, sq);
@@ -198,14 +217,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
                     kq = fmaf(qv, kv, kq);
                 } else {
                     const int c = j - dk;
-                    vs[c] = conv_channel(cx, cw, ccs, cs, 2 * dk + c, 2 * (int64_t)H * dk + h * dv + c, K);
+                    vs[c] = conv_channel(cx, cw, ccs, cs, 2 * dk + c, 2 * (int64_t)Hk * dk + h * dv + c, K);
                 }
             }
+            if (first) {
+                sq = warp_sum(sq);
+                sk = warp_sum(sk);
+                kq = warp_sum(kq);
+                if (lane == 0) part[warp] = make_float4(sq, sk, kq, 0.f);
+            }
         }
-        sq = warp_sum(sq);
-        sk = warp_sum(sk);
-        kq = warp_sum(kq);
-        if (lane == 0) part[warp] = make_float4(sq, sk, kq, 0.f);
         // this thread's state rows and gate
         float4 st[RPT];
         if (tid < nthr) {
@@ -217,10 +238,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
         if (a.z && tid < cols4) z4 = load4(reinterpret_cast<const T*>(sl + geo.z_off) + 4 * cg);
         __syncthreads();  // the slot is read; q, k, v and the norm partials are in
         if (tid == 0) {
-            in_flight = un < total;
+            in_flight = un >= 0;
             if (in_flight) {
                 fence_proxy_async();  // the slot's reads come before the copy's writes
-                load_unit<T>(a, geo, sl, un, full);
+                load_unit<T>(a, geo, sl, un, gpos_n == 0, full);
             }
         }
         float4 nrm = part[0];
@@ -285,9 +306,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
                     o.z = o.z * inv * nw4.z * silu_s(z4.z);
                     o.w = o.w * inv * nw4.w * silu_s(z4.w);
                 }
-                if (rg == 0) store4(static_cast<T*>(a.o) + u * dv + 4 * cg, o);
+                if (rg == 0) store4(static_cast<T*>(a.o) + (int64_t)u * dv + 4 * cg, o);
             }
-            float* Sg = a.state + u * dk * dv;
+            float* Sg = a.state + (int64_t)u * dk * dv;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const float kn = ks[rg * RPT + r] * inv_k;
@@ -299,12 +320,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
                 __stcs(reinterpret_cast<float4*>(Sg + (int64_t)(rg * RPT + r) * dv + 4 * cg), x);
             }
         }
+        u = un;
+        gpos = gpos_n;
     }
-    // after a timeout the copy being waited on may still land: let it
-    if (tid == 0 && in_flight) {
-        const int64_t done = (u - blockIdx.x) / gridDim.x;  // units this CTA finished
-        mbar_wait(full, (uint32_t)(done & 1), kDrainNs);
-    }
+    // after a timeout the copy being waited on (the i-th) may still land: let it
+    if (tid == 0 && in_flight) mbar_wait(full, (uint32_t)(i & 1), kDrainNs);
 }
 
 template <typename T, int RPT>
@@ -316,9 +336,9 @@ cudaError_t launch_rpt(const DecodeArgs& a, cudaStream_t s) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t units = (int64_t)a.N * a.H;
+    const int64_t groups = (int64_t)a.N * a.Hk;  // a CTA takes whole q/k groups
     const int64_t slots = (int64_t)kCtasPerSm * sms;
-    kernel<<<(unsigned)(units < slots ? units : slots), kThreads, geo.smem, s>>>(a, geo);
+    kernel<<<(unsigned)(groups < slots ? groups : slots), kThreads, geo.smem, s>>>(a, geo);
     return cudaGetLastError();
 }
 
@@ -336,10 +356,10 @@ bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 }  // namespace
 
 bool decode_stream_supported(const DecodeArgs& a) {
-    // the whole-mixer step with ungrouped heads; the state rows of a thread
+    // the whole-mixer step (any q/k grouping); the state rows of a thread
     // fit its registers; every bulk copy starts on a 16-byte boundary and
     // moves a multiple of 16 bytes; two CTAs fit in an SM's shared memory
-    if (!a.x || a.H != a.Hk || a.dv % 4 != 0 || a.dv > 128 || a.dk % 16 != 0 || a.dk > 128) return false;
+    if (!a.x || a.Hk <= 0 || a.H % a.Hk != 0 || a.dv % 4 != 0 || a.dv > 128 || a.dk % 16 != 0 || a.dk > 128) return false;
     const int esz = a.is_bf16 ? 2 : 4;
     if ((a.dk * esz) % 16 != 0 || (a.dv * esz) % 16 != 0) return false;
     const int rpt = stream_rpt(a);

@@ -52,14 +52,11 @@ struct DecodeArgs {
     uint64_t wait_ns;  // bound on each wait of the streaming kernel
 };
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
-// Persistent streaming form of the whole-mixer step (ungrouped heads): two
-// CTAs per SM, each prefetching its next unit's state and conv inputs into a
-// shared-memory slot by bulk copies.
+// Persistent streaming form of the whole-mixer step: two CTAs per SM, each
+// taking whole q/k groups of value heads and prefetching its next unit's state
+// and conv inputs into a shared-memory slot by bulk copies.
 bool decode_stream_supported(const DecodeArgs& a);
 cudaError_t launch_decode_stream(const DecodeArgs& a, cudaStream_t s);
-// Largest value-head group (H / Hk) of the whole-mixer decode step: one
-// thread-block cluster per group, 8 being the portable cluster size.
-constexpr int kMaxDecodeGroup = 8;
 
 // Backward of the recurrence (fp32, one CTA per (sequence, value head)).
 constexpr int kCk = 16;  // tokens between state checkpoints

@@ -298,10 +298,10 @@ GDN_API gdn_status_t gdn_decode_step(const void* q, const void* k, const void* v
  *   z           [N, H, dv]        dtype   nullable: no gate
  *   norm_w      [dv]              fp32    required when z is given
  *   o           [N, H, dv]        dtype   output
- * Supported: dk, dv in {16, 32, ..., 128}; H / Hk <= 8 (the CTAs of one
- * value-head group run as one thread-block cluster; larger groups return
- * GDN_ERR_UNSUPPORTED). No buffer may overlap another. With H == Hk the step
- * runs as a persistent kernel whose wait for each state copy is bounded (see
+ * Supported: dk, dv in {16, 32, ..., 128}; any H / Hk (a CTA runs the value
+ * heads of one q/k head back to back, so the shared q, k conv state is
+ * shifted once). No buffer may overlap another. The step runs as a persistent
+ * kernel whose wait for each state copy is bounded (see
  * gdn_set_wait_limit_ns): a wait that runs out leaves some (sequence, head)
  * units unprocessed and records GDN_ERR_TIMEOUT for gdn_check_device_status.
  */

@@ -171,7 +171,6 @@ def _layer_step(L, **kw):
     (dict(z=FAKE, nw=FAKE, neps=-1.0), 1), (dict(o=ctypes.c_void_p((1 << 20) + 8)), 1),
     (dict(cs=ctypes.c_void_p((1 << 20) + 2)), 1), (dict(eps=float("nan")), 1),
     (dict(Hk=3), 1), (dict(Hk=-1), 1),
-    (dict(Hk=1), 2),                         # 16 value heads per q, k head: above the cluster limit
     (dict(und=7), 1),
 ])
 def test_decode_layer_step_rejects_bad_arguments(L, kw, expect):

@@ -493,11 +493,11 @@ def test_decode_layer_step_matches_oracle(kind, gate, K):
 
 
 @pytest.mark.parametrize("kind", ["bf16", "f32"])
-@pytest.mark.parametrize("G", [2, 4, 8])
+@pytest.mark.parametrize("G", [2, 4, 8, 16])
 def test_decode_layer_step_grouped_value_heads(kind, G):
-    """G value heads per q, k head: the G CTAs of a group run as one cluster and
-    share the q, k conv channels; three tokens in a row check that the shared
-    conv state is shifted exactly once per token."""
+    """G value heads per q, k head share the q, k conv channels (one CTA runs a
+    group's value heads back to back); three tokens in a row check that the
+    shared conv state is shifted exactly once per token."""
     r = np.random.default_rng(34 + G)
     N, Hk, dk, dv, K = 5, 2, 128, 128, 4
     H = G * Hk
@@ -563,15 +563,18 @@ def test_decode_layer_step_undecayed_read(kind):
     assert worst <= tol_ and err(host(st_d), st_o) <= tol_
 
 
-@pytest.mark.parametrize("kind,K,gate", [("bf16", 4, True), ("f32", 4, True), ("bf16", 1, False),
-                                         ("f32", 3, False)])
-def test_decode_layer_step_many_units_per_sm(kind, K, gate):
-    """640 (sequence, head) units, several per SM: the streaming kernel's ring
-    of state slots wraps around (three slots in bf16, two in fp32, whose conv
-    inputs are twice as large); K = 1 runs without a conv state."""
-    r = np.random.default_rng(46 + K)
-    N, H, dk, dv = 40, 16, 128, 128
-    C = 2 * H * dk + H * dv
+@pytest.mark.parametrize("kind,K,gate,G", [("bf16", 4, True, 1), ("f32", 4, True, 1), ("bf16", 1, False, 1),
+                                           ("f32", 3, False, 1), ("bf16", 4, True, 2), ("f32", 4, True, 4)])
+def test_decode_layer_step_many_units_per_sm(kind, K, gate, G):
+    """More q/k groups than the streaming kernel's CTAs (two per SM), so CTAs
+    take several groups and each CTA's prefetch slot is refilled many times;
+    with G > 1 a CTA runs a group's G value heads back to back on shared q, k;
+    K = 1 runs without a conv state."""
+    r = np.random.default_rng(46 + K + 10 * G)
+    H, dk, dv = 16, 128, 128
+    Hk = H // G
+    N = 640 // Hk
+    C = 2 * Hk * dk + H * dv
     to = (lambda a: gi.to_bf16_bits(a.astype(np.float32))) if kind == "bf16" else (
         lambda a: a.astype(np.float32))
     cw = to(r.normal(size=(C, K)) * 0.5)
@@ -589,9 +592,9 @@ def test_decode_layer_step_many_units_per_sm(kind, K, gate):
         b = (1.0 / (1.0 + np.exp(-r.normal(size=(N, H))))).astype(np.float32)
         o = gdn.decode_layer_step(dev_tensor(x, kind), dev_tensor(cw, kind), cs_d,
                                   torch.from_numpy(g).to(DEV), torch.from_numpy(b).to(DEV), st_d,
-                                  H=H, dk=dk, dv=dv, z=None if z is None else dev_tensor(z, kind),
+                                  H=H, Hk=Hk, dk=dk, dv=dv, z=None if z is None else dev_tensor(z, kind),
                                   norm_w=torch.from_numpy(nw).to(DEV) if gate else None)
-        o_ref, cs_n, st_o = oracle.decode_layer_step(x, cw, cs_o, g, b, st_o, dtype=kind, H=H,
+        o_ref, cs_n, st_o = oracle.decode_layer_step(x, cw, cs_o, g, b, st_o, dtype=kind, H=H, Hk=Hk,
                                                      dk=dk, dv=dv, z=z, norm_w=nw if gate else None)
         if K > 1:
             cs_o = to(cs_n) if kind == "bf16" else cs_n
