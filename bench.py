@@ -255,16 +255,23 @@ def resident_bytes():
 # our arm
 # ----------------------------------------------------------------------------
 
-def timed(fn, steps, stream):
-    """Run fn `steps` times between two events; returns (total ms, per-call ms)."""
+def timed(fn, steps, stream, per_call=True):
+    """Run fn `steps` times between two events; returns (total ms, per-call ms).
+    per_call=False records no event between the calls (back-to-back calls may
+    then overlap a launch with the previous kernel's tail, as in a user's loop);
+    the per-call list is then empty."""
     import torch
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    n_ev = steps + 1 if per_call else 2
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     evs[0].record(stream)
     for i in range(steps):
         fn()
-        evs[i + 1].record(stream)
+        if per_call:
+            evs[i + 1].record(stream)
+    if not per_call:
+        evs[1].record(stream)
     torch.cuda.synchronize()
-    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)] if per_call else []
     return evs[0].elapsed_time(evs[-1]), per
 
 
@@ -417,7 +424,7 @@ def bench_decode(args, dist, pk):
     for _ in range(5):
         step()
     torch.cuda.synchronize()
-    total_ms, per = timed(step, steps, stream)
+    total_ms, _ = timed(step, steps, stream, per_call=False)
     total_ms = dist.max(total_ms)
     step_ms = total_ms / steps
     # the same 100 steps captured once in a CUDA graph and replayed (launch cost
@@ -551,7 +558,7 @@ def bench_decode_layer(args, dist, pk):
     for _ in range(5):
         step()
     torch.cuda.synchronize()
-    total_ms, _ = timed(step, steps, stream)
+    total_ms, _ = timed(step, steps, stream, per_call=False)
     step_ms = dist.max(total_ms) / steps
     # state in and out, x, conv state in and out, z, o, gates; taps once
     bytes_step = (2 * N * H * STATE_BYTES + N * C * 2 + 2 * N * C * (K - 1) * 2
@@ -640,7 +647,7 @@ def bench_grouped(args, dist, pk):
         dstep()
     gdn.check_device_status(dev)
     torch.cuda.synchronize()
-    total_ms, _ = timed(dstep, steps, stream)
+    total_ms, _ = timed(dstep, steps, stream, per_call=False)
     step_ms = dist.max(total_ms) / steps
     bytes_step = (2 * Nd * Hv * STATE_BYTES + Nd * C * 2 + 2 * Nd * C * (K - 1) * 2
                   + 2 * Nd * Hv * D * 2 + Nd * Hv * 8 + C * K * 2)
@@ -720,7 +727,7 @@ def bench_undecayed(args, dist, pk):
     for _ in range(5):
         dstep()
     torch.cuda.synchronize()
-    total_ms, _ = timed(dstep, steps, stream)
+    total_ms, _ = timed(dstep, steps, stream, per_call=False)
     step_ms = dist.max(total_ms) / steps
     bytes_step = N * H * (2 * STATE_BYTES + 4 * D * 2 + 8)
     dec = {"value": N / (step_ms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": step_ms,

@@ -72,6 +72,14 @@ __device__ __forceinline__ void cp_async_wait_all_groups() { asm volatile("cp.as
 __device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // Index of the sequence that contains token t: largest n with cu[n] <= t.
+// Programmatic dependent launch (launches made with launch_pdl): a kernel lets
+// the next kernel on the stream begin launching (its CTAs take SM slots as
+// this one's free up), and waits for the previous kernel's completion and
+// memory before it touches anything that kernel wrote. Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_previous() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ int find_sequence(const int32_t* cu, int N, int64_t t) {
     int lo = 0, hi = N - 1;
     while (lo < hi) {

@@ -36,6 +36,11 @@ __global__ void __launch_bounds__(256, 2) decode_step_kernel(DecodeArgs a) {
     float* red = ks + dk;             // [2][RG][dv]
     float* scal = red + 2 * RG * dv;  // [4]: inv_k, q_scale, kq
 
+    // 0. The next step may start launching; this one reads the state the
+    // previous step wrote only after that step has finished.
+    pdl_launch_dependents();
+    pdl_wait_previous();
+
     // 1. Issue the state loads: they are the bulk of the traffic.
     float* Sg = a.state + nh * dk * dv;
     float4 s[RPT];
@@ -137,8 +142,7 @@ cudaError_t launch_rpt(const DecodeArgs& a, cudaStream_t s) {
     const int RG = a.dk / RPT;
     const int threads = cols4 * RG;
     const size_t smem = sizeof(float) * (2 * a.dk + 2 * RG * a.dv + 4);
-    decode_step_kernel<T, RPT><<<(unsigned)((int64_t)a.N * a.H), threads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(decode_step_kernel<T, RPT>, dim3((unsigned)((int64_t)a.N * a.H)), dim3(threads), smem, s, a);
 }
 
 template <typename T>

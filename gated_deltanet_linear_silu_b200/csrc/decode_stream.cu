@@ -162,11 +162,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_layer_stream_kern
 
     int u = (int)blockIdx.x * G < total ? (int)blockIdx.x * G : -1;
     int gpos = 0;  // u's position in its group
+    pdl_launch_dependents();  // the next step may start launching
     if (tid == 0) {
         mbar_init(full, 1);
         fence_mbar_init();
-        if (u >= 0) load_unit<T>(a, geo, sl, u, true, full);
     }
+    pdl_wait_previous();  // the previous step's states and conv states are written
+    if (tid == 0 && u >= 0) load_unit<T>(a, geo, sl, u, true, full);
     float g_next = 0.f, b_next = 0.f;  // gate and beta one unit ahead
     if (u >= 0) {
         g_next = a.g[u];
@@ -338,8 +340,8 @@ cudaError_t launch_rpt(const DecodeArgs& a, cudaStream_t s) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t groups = (int64_t)a.N * a.Hk;  // a CTA takes whole q/k groups
     const int64_t slots = (int64_t)kCtasPerSm * sms;
-    kernel<<<(unsigned)(groups < slots ? groups : slots), kThreads, geo.smem, s>>>(a, geo);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3((unsigned)(groups < slots ? groups : slots)), dim3(kThreads), geo.smem, s, a,
+                      geo);
 }
 
 int stream_rpt(const DecodeArgs& a) {
