@@ -40,10 +40,12 @@
 // over A: 16 x 16 diagonal blocks by substitution in registers, merged on
 // tf32 mma.sync tiles.
 //
-// Warp roles (one persistent CTA of 16 warps per SM; units (sequence, head)
-// round-robin over the CTAs in longest-first order; every role walks the same
-// list of 64-token chunks):
-//   warp 0        TMA producer: q, k, v tiles of a chunk into a 3-stage ring
+// Warp roles (one persistent CTA of 16 warps per SM; units (sequence, head) in
+// longest-first order, CTA c starting with unit c and taking the next from a
+// work counter as it runs out; every role walks the same list of 64-token
+// chunks):
+//   warp 0        TMA producer: q, k, v tiles of a chunk into a 3-stage ring;
+//                 takes the CTA's next unit from the work counter
 //   warp 1        issues the state-independent MMAs (Gram, W^T, U~^T)
 //   warp 2        issues the state MMAs (U, O, S); the last MMA of a chunk
 //                 frees its stage for the producer
