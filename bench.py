@@ -317,31 +317,60 @@ def bench_prefill(args, dist, pk):
     kernel_ms = dist.max(statistics.mean(per))
     gdn.check_device_status(dev)
 
-    # end to end: pinned host inputs -> device -> library -> host outputs
+    # end to end: pinned host inputs -> device -> library -> host outputs, as a
+    # serving loop would run it: two device buffer sets, the host-to-device copy
+    # of step i+1 on one copy stream while step i computes, the device-to-host
+    # copy of step i on another (PCIe carries both directions at once). Every
+    # step's copies are inside the timed region.
     ho = torch.empty((T, H, D), dtype=torch.bfloat16).pin_memory()
     hhT = torch.empty((SEQS, H, D, D), dtype=torch.float32).pin_memory()
-    cu_e = torch.empty_like(cu)
+    bufs = [dict(q=q, k=k, v=v, g=g, beta=beta, cu=torch.empty_like(cu), o=o, hT=hT)]
+    bufs.append({n: torch.empty_like(t) for n, t in bufs[0].items()})
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    done_in = [ev(), ev()]      # inputs of buffer set b are on the device
+    done_comp = [ev(), ev()]    # the prefill on buffer set b finished
+    done_out = [ev(), ev()]     # the results of buffer set b are on the host
+    e2e_i = [0]
 
     def e2e_step():
-        for dst, src in ((q, hq), (k, hk), (v, hv), (g, hg), (beta, hb), (cu_e, hcu)):
-            dst.copy_(src, non_blocking=True)
-        gdn.prefill(q, k, v, g, beta, cu_e, final_state=hT, out=o, workspace=ws, chunk=CHUNK,
-                    algo=args.algo)
-        ho.copy_(o, non_blocking=True)
-        hhT.copy_(hT, non_blocking=True)
+        b = e2e_i[0] % 2
+        e2e_i[0] += 1
+        B = bufs[b]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(done_comp[b])  # the previous prefill on this set has read its inputs
+            for n, src in (("q", hq), ("k", hk), ("v", hv), ("g", hg), ("beta", hb), ("cu", hcu)):
+                B[n].copy_(src, non_blocking=True)
+            done_in[b].record(s_in)
+        stream.wait_event(done_in[b])
+        stream.wait_event(done_out[b])  # the previous results of this set have left
+        gdn.prefill(B["q"], B["k"], B["v"], B["g"], B["beta"], B["cu"], final_state=B["hT"], out=B["o"],
+                    workspace=ws, chunk=CHUNK, algo=args.algo)
+        done_comp[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done_comp[b])
+            ho.copy_(B["o"], non_blocking=True)
+            hhT.copy_(B["hT"], non_blocking=True)
+            done_out[b].record(s_out)
 
-    e2e_step()
+    def e2e_run(n):
+        for _ in range(n):
+            e2e_step()
+        for b in range(2):  # the timed region ends when the last results are on the host
+            stream.wait_event(done_out[b])
+
+    e2e_run(2)
     dist.barrier()
     torch.cuda.synchronize()
-    e2e_ms, _ = timed(e2e_step, max(1, min(args.steps, 5)), stream)
     e2e_steps = max(1, min(args.steps, 5))
+    e2e_ms, _ = timed(lambda: e2e_run(e2e_steps), 1, stream)
     dist.barrier()
     e2e_ms = dist.max(e2e_ms)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hcu))
     d2h = ho.numel() * ho.element_size() + hhT.numel() * hhT.element_size()
     res = {"P": P, "tokens": T, "total_ms": total_ms, "kernel_ms": kernel_ms,
            "e2e_ms_per_step": e2e_ms / e2e_steps, "h2d": h2d, "d2h": d2h}
-    del q, k, v, g, beta, o, hT, hq, hk, hv, ho, hhT
+    del q, k, v, g, beta, o, hT, hq, hk, hv, ho, hhT, bufs
     torch.cuda.empty_cache()
     return res
 
@@ -932,7 +961,9 @@ def run_ours(args, dist: Dist):
                         if pk.get("bf16_tflops_sustained") else None,
                         "algorithmic_flops": flops},
         "e2e": {"value": tokens_all / (pre["e2e_ms_per_step"] * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"]},
+                "h2d_bytes_per_step": pre["h2d"], "d2h_bytes_per_step": pre["d2h"],
+                "how": "gdn.prefill on two device buffer sets; each step's H2D (pinned) and D2H on "
+                       "their own streams, overlapping the neighbouring steps"},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
         "algo": algo,
