@@ -253,6 +253,24 @@ def test_prefill_more_units_than_sms(algo):
     assert np.array_equal(hT[5], P.h0[5]) and np.array_equal(hT[17], P.h0[17])
 
 
+def test_prefill_many_short_units_work_counter():
+    """750 sequences of 0..150 tokens x 4 heads = 3000 units on the tensor-core
+    kernel: each CTA takes about twenty units from the work counter, so the
+    shared-memory ring that hands a unit to every role wraps around (16 slots)
+    and the roles meet units of one to three chunks back to back; every element
+    and every final state against the oracle."""
+    lens = np.random.default_rng(29).integers(0, 151, size=750)
+    lens[[3, 400, 749]] = 0
+    P = gi.random_prefill(29, lens.tolist(), H=4, dk=128, dv=128, with_h0=True)
+    sms = torch.cuda.get_device_properties(DEV).multi_processor_count
+    assert P.N * P.H > 16 * sms
+    o, hT = prefill_gpu(P, algo="tensor")
+    o_ref, h_ref = prefill_oracle(P)
+    assert err(o, o_ref) <= TOL_BF16
+    assert err(hT, h_ref) <= TOL_BF16
+    assert np.array_equal(hT[400], P.h0[400])
+
+
 @pytest.mark.parametrize("algo", ["tensor", "simt"])
 @pytest.mark.parametrize("undecayed", [False, True])
 def test_prefill_gated_output(algo, undecayed):
