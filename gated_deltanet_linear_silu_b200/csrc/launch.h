@@ -170,8 +170,10 @@ int prefill_split_segments(int N, int64_t T_tot, int H, int dk, int dv, int chun
 size_t prefill_split_workspace_bytes(int N, int64_t T_tot, int H, int S);
 cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, cudaStream_t s);
 
-// Builds the longest-first schedule and zeroes the work counter.
-cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s);
+// Builds the longest-first schedule and zeroes the work counter; `copies`
+// counter pairs, 2 ints apart in the 256-byte counter line (launches that share
+// one schedule each take their own pair).
+cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s, int copies = 1);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 bool prefill_tc_supported(const PrefillArgs& a);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);

@@ -16,14 +16,16 @@ __device__ __forceinline__ bool is_work(const int32_t* cu, int i, int64_t T_tot)
     return cu[i] >= 0 && cu[i + 1] > cu[i] && cu[i + 1] <= T_tot;
 }
 
+// `copies` counter pairs (work counter, number of work sequences), 2 ints
+// apart, for launches that share one schedule.
 __global__ void __launch_bounds__(1024) prefill_schedule_kernel(const int32_t* cu, int N,
                                                                 int64_t T_tot, int32_t* order,
-                                                                int32_t* counter, int* status) {
+                                                                int32_t* counter, int copies, int* status) {
     extern __shared__ int32_t len[];
     __shared__ int32_t s_work, s_warp[32];
     const bool sort = N <= kMaxSortN;
     if (threadIdx.x == 0) {
-        counter[0] = 0;
+        for (int c = 0; c < copies; ++c) counter[2 * c] = 0;
         s_work = 0;
         if (cu[0] != 0 || cu[N] != T_tot) set_status(status, kStatusBadSeqlens);
     }
@@ -39,7 +41,8 @@ __global__ void __launch_bounds__(1024) prefill_schedule_kernel(const int32_t* c
     atomicAdd(&s_work, mine);
     __syncthreads();
     const int n_work = s_work;
-    if (threadIdx.x == 0) counter[1] = n_work;
+    if (threadIdx.x == 0)
+        for (int c = 0; c < copies; ++c) counter[2 * c + 1] = n_work;
     if (sort) {
         // Rank sort: position = number of sequences that go before this one
         // (longer, or equally long with a smaller index); non-work (-1) last.
@@ -91,9 +94,9 @@ WorkspaceLayout prefill_workspace_layout(int N) {
     return l;
 }
 
-cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s) {
+cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s, int copies) {
     const size_t smem = a.N <= kMaxSortN ? sizeof(int32_t) * (size_t)a.N : 0;
-    prefill_schedule_kernel<<<1, 1024, smem, s>>>(a.cu, a.N, a.T_tot, a.order, a.counter, a.status);
+    prefill_schedule_kernel<<<1, 1024, smem, s>>>(a.cu, a.N, a.T_tot, a.order, a.counter, copies, a.status);
     return cudaGetLastError();
 }
 

@@ -57,32 +57,33 @@ SplitLayout split_layout(int N, int64_t T_tot, int H, int S) {
     return l;
 }
 
-// Segment boundaries: sequence n = [st, en) of c = ceil(len / 64) chunks gives
-// segment k = [st + 64 floor(k c / S), st + 64 floor((k+1) c / S)) clipped to
-// en (empty segments when c < S). A sequence with bad bounds gets empty
-// segments and keeps its bad end, so the prefill flags it.
-__global__ void split_bounds_kernel(const int32_t* cu, int N, int S, int32_t* cu_seg) {
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// One launch prepares the three passes (grid-stride over all of it):
+//  - segment bounds: sequence n = [st, en) of c = ceil(len / 64) chunks gives
+//    segment k = [st + 64 floor(k c / S), st + 64 floor((k+1) c / S)) clipped
+//    to en (empty segments when c < S); a sequence with bad bounds gets empty
+//    segments and keeps its bad end, so the prefill flags it;
+//  - A (pass 1a and pass 2 initial states): segment 0 <- h0 (zeros if none),
+//    the rest zeros; B (pass 1b initial states): the identity;
+//  - the bf16 zero values of pass 1b.
+__global__ void split_init_kernel(const int32_t* cu, const float* h0, int N, int H, int S, int32_t* cu_seg,
+                                  float* A, float* B, uint4* zeros_v, int64_t n_zero16) {
     const int64_t NS = (int64_t)N * S;
-    if (idx > NS) return;
-    if (idx == NS) {
-        cu_seg[idx] = cu[N];
-        return;
+    const int64_t n4 = NS * H * kStateFloats / 4;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t idx = i0; idx <= NS; idx += stride) {
+        if (idx == NS) {
+            cu_seg[idx] = cu[N];
+            continue;
+        }
+        const int n = (int)(idx / S), k = (int)(idx % S);
+        const int64_t st = cu[n], en = cu[n + 1];
+        const int64_t len = en > st ? en - st : 0;
+        const int64_t c = (len + 63) / 64;
+        const int64_t off = 64 * ((k * c) / S);
+        cu_seg[idx] = (int32_t)(st + (off < len ? off : len));
     }
-    const int n = (int)(idx / S), k = (int)(idx % S);
-    const int64_t st = cu[n], en = cu[n + 1];
-    const int64_t len = en > st ? en - st : 0;
-    const int64_t c = (len + 63) / 64;
-    const int64_t off = 64 * ((k * c) / S);
-    cu_seg[idx] = (int32_t)(st + (off < len ? off : len));
-}
-
-// A (pass 1a and pass 2 initial states): segment 0 <- h0 (zeros if none),
-// the rest zeros; B (pass 1b initial states): the identity.
-__global__ void split_fill_kernel(const float* h0, int N, int H, int S, float* A, float* B) {
-    const int64_t n4 = (int64_t)N * S * H * kStateFloats / 4;
-    for (int64_t e4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e4 < n4;
-         e4 += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t e4 = i0; e4 < n4; e4 += stride) {
         const int64_t e = 4 * e4;
         const int64_t blk = e / kStateFloats, within = e % kStateFloats;
         const int h = (int)(blk % H);
@@ -96,6 +97,7 @@ __global__ void split_fill_kernel(const float* h0, int N, int H, int S, float* A
                                       row == col + 2 ? 1.f : 0.f, row == col + 3 ? 1.f : 0.f);
         reinterpret_cast<float4*>(B)[e4] = id;
     }
+    for (int64_t z = i0; z < n_zero16; z += stride) zeros_v[z] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 // The chain of segment start states, per (sequence, head) and block of 16
@@ -232,27 +234,31 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
     const int NS = a.N * S;
     const int fill_blocks = 4 * sm_count();
 
-    split_bounds_kernel<<<(NS + 1 + 255) / 256, 256, 0, s>>>(a.cu, a.N, S, cu_seg);
-    split_fill_kernel<<<fill_blocks, 256, 0, s>>>(a.h0, a.N, a.H, S, A, B);
+    split_init_kernel<<<fill_blocks, 256, 0, s>>>(a.cu, a.h0, a.N, a.H, S, cu_seg, A, B,
+                                                  static_cast<uint4*>(zeros_v),
+                                                  (int64_t)a.T_tot * a.H * kSplitD * 2 / 16);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(zeros_v, 0, (size_t)a.T_tot * a.H * kSplitD * 2, s)) != cudaSuccess) return e;
 
+    // One schedule of the N S segments serves the three passes, each with its
+    // own work counter.
     PrefillArgs p = a;
     p.cu = cu_seg;
     p.N = NS;
     p.order = reinterpret_cast<int32_t*>(ws + l.base.order_off);
-    p.counter = reinterpret_cast<int32_t*>(ws + l.base.counter_off);
-    auto pass = [&](const float* h0, float* hT) {
+    int32_t* counters = reinterpret_cast<int32_t*>(ws + l.base.counter_off);
+    p.counter = counters;
+    if ((e = launch_prefill_schedule(p, s, 3)) != cudaSuccess) return e;
+    auto pass = [&](int which, const float* h0, float* hT) {
         p.h0 = h0;
         p.hT = hT;
-        cudaError_t err = launch_prefill_schedule(p, s);
-        return err != cudaSuccess ? err : launch_prefill_tc(p, s);
+        p.counter = counters + 2 * which;
+        return launch_prefill_tc(p, s);
     };
-    if ((e = pass(a.h0 ? A : nullptr, Lst)) != cudaSuccess) return e;  // 1a
+    if ((e = pass(0, a.h0 ? A : nullptr, Lst)) != cudaSuccess) return e;  // 1a
     p.v = zeros_v;
     p.ld_v = (int64_t)a.H * kSplitD;
-    e = pass(B, Phi);  // 1b
+    e = pass(1, B, Phi);  // 1b
     p.v = a.v;
     p.ld_v = a.ld_v;
     if (e != cudaSuccess) return e;
@@ -262,7 +268,7 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
     split_combine_kernel<<<dim3((unsigned)(a.N * a.H), kSplitD / kCombCols), kCombThreads, kCombSmem, s>>>(
         a.N, a.H, S, Lst, Phi, A);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = pass(A, a.hT ? B : nullptr)) != cudaSuccess) return e;  // 2
+    if ((e = pass(2, A, a.hT ? B : nullptr)) != cudaSuccess) return e;  // 2
     if (a.hT) {
         split_final_kernel<<<fill_blocks, 256, 0, s>>>(B, a.N, a.H, S, a.hT);
         e = cudaGetLastError();
