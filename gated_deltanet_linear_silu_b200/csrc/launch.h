@@ -173,9 +173,11 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
 // Builds the longest-first schedule and zeroes the work counter; `copies`
 // counter pairs, 2 ints apart in the 256-byte counter line (launches that share
 // one schedule each take their own pair).
-cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s, int copies = 1);
+// pdl: launch with programmatic dependent launch (the sequence split's chain;
+// measured slower for the single-pass prefill, which launches ordinarily).
+cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s, int copies = 1, bool pdl = false);
 cudaError_t launch_prefill_simt(const PrefillArgs& a, cudaStream_t s);
 bool prefill_tc_supported(const PrefillArgs& a);
-cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s, bool pdl = false);
 
 }  // namespace gdn

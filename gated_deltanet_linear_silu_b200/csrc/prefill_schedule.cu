@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(1024) prefill_schedule_kernel(const int32_t* c
                                                                 int32_t* counter, int copies, int* status) {
     extern __shared__ int32_t len[];
     __shared__ int32_t s_work, s_warp[32];
+    pdl_launch_dependents();  // dependent launch (the sequence split): the chunk kernel may
+    pdl_wait_previous();      // start launching; no-ops for an ordinary launch
     const bool sort = N <= kMaxSortN;
     if (threadIdx.x == 0) {
         for (int c = 0; c < copies; ++c) counter[2 * c] = 0;
@@ -94,8 +96,11 @@ WorkspaceLayout prefill_workspace_layout(int N) {
     return l;
 }
 
-cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s, int copies) {
+cudaError_t launch_prefill_schedule(const PrefillArgs& a, cudaStream_t s, int copies, bool pdl) {
     const size_t smem = a.N <= kMaxSortN ? sizeof(int32_t) * (size_t)a.N : 0;
+    if (pdl)
+        return launch_pdl(prefill_schedule_kernel, dim3(1), dim3(1024), smem, s, a.cu, a.N, a.T_tot, a.order,
+                          a.counter, copies, a.status);
     prefill_schedule_kernel<<<1, 1024, smem, s>>>(a.cu, a.N, a.T_tot, a.order, a.counter, copies, a.status);
     return cudaGetLastError();
 }

@@ -67,6 +67,8 @@ SplitLayout split_layout(int N, int64_t T_tot, int H, int S) {
 //  - the bf16 zero values of pass 1b.
 __global__ void split_init_kernel(const int32_t* cu, const float* h0, int N, int H, int S, int32_t* cu_seg,
                                   float* A, float* B, uint4* zeros_v, int64_t n_zero16) {
+    pdl_launch_dependents();
+    pdl_wait_previous();
     const int64_t NS = (int64_t)N * S;
     const int64_t n4 = NS * H * kStateFloats / 4;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -124,6 +126,8 @@ __device__ __forceinline__ void stage_phi(float* dst, const float* src) {
 __global__ void __launch_bounds__(kCombThreads) split_combine_kernel(int N, int H, int S, const float* Lst,
                                                                     const float* Phi, float* A) {
     extern __shared__ float4 comb_smem4[];
+    pdl_launch_dependents();
+    pdl_wait_previous();
     float* phi_s = reinterpret_cast<float*>(comb_smem4);  // [2][128][kPhiLd]
     float* cur = phi_s + 2 * kSplitD * kPhiLd;             // [128][16]
     const int nh = blockIdx.x;                             // n * H + h
@@ -188,6 +192,7 @@ __global__ void __launch_bounds__(kCombThreads) split_combine_kernel(int N, int 
 
 // hT[n] <- the final state of sequence n's last segment (pass 2's output).
 __global__ void split_final_kernel(const float* B, int N, int H, int S, float* hT) {
+    pdl_wait_previous();
     const int64_t n4 = (int64_t)N * H * kStateFloats / 4;
     for (int64_t e4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e4 < n4;
          e4 += (int64_t)gridDim.x * blockDim.x) {
@@ -234,10 +239,9 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
     const int NS = a.N * S;
     const int fill_blocks = 4 * sm_count();
 
-    split_init_kernel<<<fill_blocks, 256, 0, s>>>(a.cu, a.h0, a.N, a.H, S, cu_seg, A, B,
-                                                  static_cast<uint4*>(zeros_v),
-                                                  (int64_t)a.T_tot * a.H * kSplitD * 2 / 16);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(split_init_kernel, dim3(fill_blocks), dim3(256), 0, s, a.cu, a.h0, a.N, a.H, S,
+                               cu_seg, A, B, static_cast<uint4*>(zeros_v),
+                               (int64_t)a.T_tot * a.H * kSplitD * 2 / 16);
     if (e != cudaSuccess) return e;
 
     // One schedule of the N S segments serves the three passes, each with its
@@ -248,12 +252,12 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
     p.order = reinterpret_cast<int32_t*>(ws + l.base.order_off);
     int32_t* counters = reinterpret_cast<int32_t*>(ws + l.base.counter_off);
     p.counter = counters;
-    if ((e = launch_prefill_schedule(p, s, 3)) != cudaSuccess) return e;
+    if ((e = launch_prefill_schedule(p, s, 3, true)) != cudaSuccess) return e;
     auto pass = [&](int which, const float* h0, float* hT) {
         p.h0 = h0;
         p.hT = hT;
         p.counter = counters + 2 * which;
-        return launch_prefill_tc(p, s);
+        return launch_prefill_tc(p, s, true);
     };
     if ((e = pass(0, a.h0 ? A : nullptr, Lst)) != cudaSuccess) return e;  // 1a
     p.v = zeros_v;
@@ -265,13 +269,13 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
     if ((e = cudaFuncSetAttribute(split_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kCombSmem)) != cudaSuccess)
         return e;
-    split_combine_kernel<<<dim3((unsigned)(a.N * a.H), kSplitD / kCombCols), kCombThreads, kCombSmem, s>>>(
-        a.N, a.H, S, Lst, Phi, A);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_pdl(split_combine_kernel, dim3((unsigned)(a.N * a.H), kSplitD / kCombCols), dim3(kCombThreads),
+                   kCombSmem, s, a.N, a.H, S, static_cast<const float*>(Lst), static_cast<const float*>(Phi), A);
+    if (e != cudaSuccess) return e;
     if ((e = pass(2, A, a.hT ? B : nullptr)) != cudaSuccess) return e;  // 2
     if (a.hT) {
-        split_final_kernel<<<fill_blocks, 256, 0, s>>>(B, a.N, a.H, S, a.hT);
-        e = cudaGetLastError();
+        e = launch_pdl(split_final_kernel, dim3(fill_blocks), dim3(256), 0, s, static_cast<const float*>(B), a.N,
+                       a.H, S, a.hT);
     }
     return e;
 }

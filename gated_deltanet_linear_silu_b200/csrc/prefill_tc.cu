@@ -425,6 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap map_q,
                   const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
     extern __shared__ uint8_t smem_raw[];
+    // Dependent launch (the sequence split's passes): the next kernel may start
+    // launching; this one reads the schedule (and every input) only after the
+    // previous kernel has finished. No-ops for an ordinary launch.
+    pdl_launch_dependents();
+    pdl_wait_previous();
     // 1024-byte alignment of the shared-window address (swizzle atoms, TMA).
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const PrefillArgs& a = P.a;
@@ -1254,7 +1259,7 @@ bool prefill_tc_supported(const PrefillArgs& a) {
            a.T_tot < ((int64_t)1 << 31) && encode_fn() != nullptr;
 }
 
-cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s, bool pdl) {
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, a.q, a.Hk, a.T_tot, a.ld_q) || !make_map(&mk, a.k, a.Hk, a.T_tot, a.ld_k) ||
         !make_map(&mv, a.v, a.H, a.T_tot, a.ld_v))
@@ -1269,6 +1274,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s) {
     const int64_t units = (int64_t)a.N * a.H;
     const int grid = (int)(units < sms ? units : sms);
     TcParams p{a};
+    if (pdl) return launch_pdl(kernel, dim3(grid), dim3(kThreads), kSmemAlloc, s, p, mq, mk, mv);
     kernel<<<grid, kThreads, kSmemAlloc, s>>>(p, mq, mk, mv);
     return cudaGetLastError();
 }
