@@ -158,6 +158,7 @@ __device__ __forceinline__ void fetch(const ConvArgs& a, int n, int64_t seq_star
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) conv_silu_kernel(ConvArgs a) {
+    pdl_launch_dependents();  // the conv-state kernel may start launching (it waits for this one)
     const int c0 = blockIdx.y * kChanPerCta + threadIdx.x * kVec;
     const bool active = c0 < a.C;
     const int64_t t0 = (int64_t)blockIdx.x * kTT;
@@ -327,6 +328,9 @@ __global__ void __launch_bounds__(kThreads) conv_silu_kernel(ConvArgs a) {
 // conv_state_out[n, c, s] = input at relative position T_n - (K-1) + s.
 template <typename T>
 __global__ void conv_state_kernel(ConvArgs a) {
+    // launched as a dependent of the conv kernel: the conv state may be updated
+    // in place, so nothing is touched before that kernel has finished
+    pdl_wait_previous();
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (int64_t)a.N * a.C) return;
     const int n = (int)(idx / a.C);
@@ -360,8 +364,7 @@ cudaError_t launch_t(const ConvArgs& a, cudaStream_t s) {
     }
     if (a.state_out && a.N > 0 && a.K > 1) {
         const int64_t total = (int64_t)a.N * a.C;
-        conv_state_kernel<T><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(a);
-        return cudaGetLastError();
+        return launch_pdl(conv_state_kernel<T>, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, s, a);
     }
     return cudaSuccess;
 }
