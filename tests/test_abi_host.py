@@ -60,6 +60,24 @@ def test_workspace_size_is_aligned_and_grows(L):
     assert a > 0 and a % 256 == 0 and b % 256 == 0 and b > a
 
 
+def test_workspace_size_covers_the_sequence_split(L):
+    """Few (sequence, head) units on the tensor-core shape: the size also holds
+    the split's segment bounds, four state arrays of N*S*H states and a bf16 zero
+    value buffer (S segments, S >= 6); many units, other head dims or chunks:
+    only the schedule (256 + 4 N, rounded up to 256)."""
+    base = lambda N: 256 + (4 * N + 255) // 256 * 256
+    assert L.gdn_prefill_workspace_size(8, 8 * 16384, 16, 128, 128, 64) == base(8)  # 128 units
+    assert L.gdn_prefill_workspace_size(1, 4096, 16, 64, 64, 64) == base(1)        # not d = 128
+    assert L.gdn_prefill_workspace_size(1, 4096, 16, 128, 128, 32) == base(1)      # not chunk 64
+    assert L.gdn_prefill_workspace_size(1, 256, 16, 128, 128, 64) == base(1)       # too short
+    split = L.gdn_prefill_workspace_size(1, 4096, 16, 128, 128, 64)
+    state = 128 * 128 * 4
+    zeros = 4096 * 16 * 128 * 2
+    assert split % 256 == 0
+    # S between 6 and 16 segments: four [S, 16] state arrays plus the zero values
+    assert base(1) + 4 * 6 * 16 * state + zeros <= split <= 2 * base(16) + 512 + 4 * 16 * 16 * state + zeros
+
+
 FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: validation fails first
 
 
