@@ -104,16 +104,19 @@ __global__ void split_init_kernel(const int32_t* cu, const float* h0, int N, int
 
 // The chain of segment start states, per (sequence, head) and block of 16
 // state columns (columns evolve independently: Phi acts on the rows), one CTA
-// each (N * H * 8 CTAs: one wave when the split applies). Thread (row i, half
-// hf) owns columns [8 hf, 8 hf + 8) of row i, in packed fp32 pairs. Phi_k is
-// staged in shared memory (rows padded to 132 floats: a quarter-warp's float4
-// reads of 8 rows hit 32 distinct banks), the next one prefetched with
-// cp.async while step k runs; the current start state's block is read as
-// broadcast float4s.
+// each (N * H * 8 CTAs: one wave when the split applies). Each step is a
+// 128 x 128 by 128 x 16 product on the tensor cores (mma.sync m16n8k8 tf32) in
+// split precision: x = hi + lo with hi = tf32(x), and hi*hi + hi*lo + lo*hi
+// keeps about fp32 accuracy. Warp w owns rows [16w, 16w + 16) of the block.
+// Phi_k is staged in shared memory (rows padded to 132 floats, so the A
+// fragments of a warp hit 32 distinct banks), the next one prefetched with
+// cp.async while step k runs; the current start state's block sits in shared
+// memory with rows padded to 24 floats (conflict-free B fragments).
 constexpr int kCombCols = 16;
 constexpr int kCombThreads = 256;
 constexpr int kPhiLd = 132;
-constexpr size_t kCombSmem = sizeof(float) * (2 * kSplitD * kPhiLd + kSplitD * kCombCols);
+constexpr int kCurLd = 24;
+constexpr size_t kCombSmem = sizeof(float) * (2 * kSplitD * kPhiLd + kSplitD * kCurLd);
 
 __device__ __forceinline__ void stage_phi(float* dst, const float* src) {
     for (int p = threadIdx.x; p < kSplitD * kSplitD / 4; p += kCombThreads) {
@@ -123,36 +126,52 @@ __device__ __forceinline__ void stage_phi(float* dst, const float* src) {
     cp_async_commit_group();
 }
 
+__device__ __forceinline__ uint32_t tf32_hi(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 __global__ void __launch_bounds__(kCombThreads) split_combine_kernel(int N, int H, int S, const float* Lst,
                                                                     const float* Phi, float* A) {
     extern __shared__ float4 comb_smem4[];
     pdl_launch_dependents();
     pdl_wait_previous();
     float* phi_s = reinterpret_cast<float*>(comb_smem4);  // [2][128][kPhiLd]
-    float* cur = phi_s + 2 * kSplitD * kPhiLd;             // [128][16]
+    float* cur = phi_s + 2 * kSplitD * kPhiLd;             // [128][kCurLd]
     const int nh = blockIdx.x;                             // n * H + h
     const int n = nh / H, h = nh % H;
-    const int i = threadIdx.x >> 1, hf = threadIdx.x & 1;
-    const int cl = 8 * hf;                                 // first column within the block
-    const int c0 = blockIdx.y * kCombCols + cl;            // first state column
+    const int cb = blockIdx.y * kCombCols;                 // first state column of the block
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * warp;
     const int64_t off0 = ((int64_t)n * S * H + h) * kStateFloats;  // segment 0 of (n, h)
     const int64_t seg = (int64_t)H * kStateFloats;                  // between segments
     if (S > 2) stage_phi(phi_s, Phi + off0 + seg);
     // S_start(1) = L_0 (segment 0 ran from the true initial state)
-    {
-        const float* l0 = Lst + off0 + (int64_t)i * kSplitD + c0;
-        float* a1 = A + off0 + seg + (int64_t)i * kSplitD + c0;
-        const float4 x0 = *reinterpret_cast<const float4*>(l0);
-        const float4 x1 = *reinterpret_cast<const float4*>(l0 + 4);
-        *reinterpret_cast<float4*>(cur + i * kCombCols + cl) = x0;
-        *reinterpret_cast<float4*>(cur + i * kCombCols + cl + 4) = x1;
-        *reinterpret_cast<float4*>(a1) = x0;
-        *reinterpret_cast<float4*>(a1 + 4) = x1;
+    for (int e = threadIdx.x; e < kSplitD * kCombCols / 4; e += kCombThreads) {
+        const int row = e / (kCombCols / 4), c4 = e % (kCombCols / 4);
+        const float4 x = *reinterpret_cast<const float4*>(Lst + off0 + (int64_t)row * kSplitD + cb + 4 * c4);
+        *reinterpret_cast<float4*>(cur + row * kCurLd + 4 * c4) = x;
+        *reinterpret_cast<float4*>(A + off0 + seg + (int64_t)row * kSplitD + cb + 4 * c4) = x;
     }
     for (int k = 1; k + 1 < S; ++k) {
-        const float* lr = Lst + off0 + k * seg + (int64_t)i * kSplitD + c0;
-        const float4 l0 = *reinterpret_cast<const float4*>(lr);
-        const float4 l1 = *reinterpret_cast<const float4*>(lr + 4);
+        // accumulators start from L_k at the fragment positions: rows r0 + g (+8),
+        // columns 8 nt + 2 t (+1) of the block
+        float acc[2][4];
+        const float* lk = Lst + off0 + k * seg + cb;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float2 x0 = *reinterpret_cast<const float2*>(lk + (int64_t)(r0 + g) * kSplitD + 8 * nt + 2 * t);
+            const float2 x1 = *reinterpret_cast<const float2*>(lk + (int64_t)(r0 + g + 8) * kSplitD + 8 * nt + 2 * t);
+            acc[nt][0] = x0.x; acc[nt][1] = x0.y; acc[nt][2] = x1.x; acc[nt][3] = x1.y;
+        }
         if (k + 2 < S) {
             // buffer (k & 1) was last read in step k - 1, which ended with a barrier
             stage_phi(phi_s + (k & 1) * kSplitD * kPhiLd, Phi + off0 + (k + 1) * seg);
@@ -161,32 +180,38 @@ __global__ void __launch_bounds__(kCombThreads) split_combine_kernel(int N, int 
             cp_async_wait_all_groups();
         }
         __syncthreads();  // Phi_k and cur visible to every thread
-        const float* pr = phi_s + ((k - 1) & 1) * kSplitD * kPhiLd + i * kPhiLd;  // row i of Phi_k
-        float2 acc[4] = {make_float2(l0.x, l0.y), make_float2(l0.z, l0.w), make_float2(l1.x, l1.y),
-                         make_float2(l1.z, l1.w)};
+        const float* pk = phi_s + ((k - 1) & 1) * kSplitD * kPhiLd;
 #pragma unroll 4
-        for (int m = 0; m < kSplitD; m += 4) {
-            const float4 p4 = *reinterpret_cast<const float4*>(pr + m);
-            const float phi[4] = {p4.x, p4.y, p4.z, p4.w};
+        for (int kk = 0; kk < kSplitD / 8; ++kk) {
+            const float af[4] = {pk[(r0 + g) * kPhiLd + 8 * kk + t], pk[(r0 + g + 8) * kPhiLd + 8 * kk + t],
+                                 pk[(r0 + g) * kPhiLd + 8 * kk + t + 4], pk[(r0 + g + 8) * kPhiLd + 8 * kk + t + 4]};
+            uint32_t ahi[4], alo[4];
 #pragma unroll
-            for (int mm = 0; mm < 4; ++mm) {
-                const float2 f = make_float2(phi[mm], phi[mm]);
-                const float4 s0 = *reinterpret_cast<const float4*>(cur + (m + mm) * kCombCols + cl);
-                const float4 s1 = *reinterpret_cast<const float4*>(cur + (m + mm) * kCombCols + cl + 4);
-                acc[0] = __ffma2_rn(f, make_float2(s0.x, s0.y), acc[0]);
-                acc[1] = __ffma2_rn(f, make_float2(s0.z, s0.w), acc[1]);
-                acc[2] = __ffma2_rn(f, make_float2(s1.x, s1.y), acc[2]);
-                acc[3] = __ffma2_rn(f, make_float2(s1.z, s1.w), acc[3]);
+            for (int q = 0; q < 4; ++q) {
+                ahi[q] = tf32_hi(af[q]);
+                alo[q] = tf32_hi(af[q] - __uint_as_float(ahi[q]));
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const float b0 = cur[(8 * kk + t) * kCurLd + 8 * nt + g];
+                const float b1 = cur[(8 * kk + t + 4) * kCurLd + 8 * nt + g];
+                const uint32_t bh0 = tf32_hi(b0), bh1 = tf32_hi(b1);
+                const uint32_t bl0 = tf32_hi(b0 - __uint_as_float(bh0)), bl1 = tf32_hi(b1 - __uint_as_float(bh1));
+                mma_16x8x8_tf32(acc[nt], alo, bh0, bh1);
+                mma_16x8x8_tf32(acc[nt], ahi, bl0, bl1);
+                mma_16x8x8_tf32(acc[nt], ahi, bh0, bh1);
             }
         }
         __syncthreads();  // every thread has read cur and Phi_k
-        const float4 a0 = make_float4(acc[0].x, acc[0].y, acc[1].x, acc[1].y);
-        const float4 a1 = make_float4(acc[2].x, acc[2].y, acc[3].x, acc[3].y);
-        *reinterpret_cast<float4*>(cur + i * kCombCols + cl) = a0;
-        *reinterpret_cast<float4*>(cur + i * kCombCols + cl + 4) = a1;
-        float* an = A + off0 + (k + 1) * seg + (int64_t)i * kSplitD + c0;
-        *reinterpret_cast<float4*>(an) = a0;
-        *reinterpret_cast<float4*>(an + 4) = a1;
+        float* an = A + off0 + (k + 1) * seg + cb;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const float2 y0 = make_float2(acc[nt][0], acc[nt][1]), y1 = make_float2(acc[nt][2], acc[nt][3]);
+            *reinterpret_cast<float2*>(cur + (r0 + g) * kCurLd + 8 * nt + 2 * t) = y0;
+            *reinterpret_cast<float2*>(cur + (r0 + g + 8) * kCurLd + 8 * nt + 2 * t) = y1;
+            *reinterpret_cast<float2*>(an + (int64_t)(r0 + g) * kSplitD + 8 * nt + 2 * t) = y0;
+            *reinterpret_cast<float2*>(an + (int64_t)(r0 + g + 8) * kSplitD + 8 * nt + 2 * t) = y1;
+        }
     }
 }
 
