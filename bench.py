@@ -789,7 +789,9 @@ def bench_backward(args, dist, pk):
     r = np.random.default_rng(9)
     do = torch.from_numpy(r.standard_normal((T, H, D), dtype=np.float32)).to(dev)
     dhT = torch.from_numpy(r.standard_normal((N, H, D, D), dtype=np.float32)).to(dev)
-    ws = torch.empty(gdn.lib().gdn_backward_workspace_size(N, T, H, D, D), dtype=torch.uint8,
+    # the workspace that keeps every token's state from the forward pass (34 GB
+    # here): one token-sequential pass fewer than recomputing 16-token blocks
+    ws = torch.empty(gdn.lib().gdn_backward_workspace_size_kept(N, T, H, D, D), dtype=torch.uint8,
                      device=dev)
     stream = torch.cuda.current_stream(dev)
 

@@ -26,7 +26,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
-ABI_VERSION = 202  # gdn_version() of the C ABI these argument lists describe
+ABI_VERSION = 203  # gdn_version() of the C ABI these argument lists describe
 
 GDN_F32, GDN_BF16 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tensor": 2}
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill_selected_algo.restype = i32
         L.gdn_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32]
         L.gdn_backward_workspace_size.restype = sz
+        L.gdn_backward_workspace_size_kept.argtypes = [i32, i64, i32, i32, i32]
+        L.gdn_backward_workspace_size_kept.restype = sz
         L.gdn_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
                                    f32, i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.gdn_backward.restype = i32
@@ -331,11 +333,13 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
              initial_state: Optional[torch.Tensor] = None, dhT: Optional[torch.Tensor] = None,
              scale: float = 1.0, qk_l2norm: bool = True, eps: float = 1e-6,
              cu_seqlens_host: Optional[torch.Tensor] = None, want_dh0: bool = True,
-             workspace: Optional[torch.Tensor] = None):
+             workspace: Optional[torch.Tensor] = None, keep_states: bool = False):
     """Gradients of the recurrence for upstream gradients do [T, H, dv] (fp32)
     and dhT [N, H, dk, dv] (fp32, optional). q, k [T, Hk, dk] and v [T, H, dv]
     dense (bf16 or fp32). Returns (dq, dk, dv, dg, dbeta, dh0), fp32; dh0 is
-    None unless want_dh0."""
+    None unless want_dh0. keep_states=True allocates the workspace with which
+    every token's state is kept from the forward pass (T * H * dk * dv * 4
+    bytes) instead of recomputed; a given workspace of that size does the same."""
     _check_heads(q, k, v, g, beta)
     T, Hk, dk = q.shape
     H, dv = v.shape[1], v.shape[2]
@@ -345,7 +349,8 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     dq, dkt = torch.empty((T, Hk, dk), **f32), torch.empty((T, Hk, dk), **f32)
     dvt, dg, db = torch.empty((T, H, dv), **f32), torch.empty((T, H), **f32), torch.empty((T, H), **f32)
     dh0 = torch.empty((N, H, dk, dv), **f32) if want_dh0 else None
-    ws_bytes = int(lib().gdn_backward_workspace_size(N, T, H, dk, dv))
+    size_fn = lib().gdn_backward_workspace_size_kept if keep_states else lib().gdn_backward_workspace_size
+    ws_bytes = int(size_fn(N, T, H, dk, dv))
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     _cuda(q, k, v, g, beta, cu_seqlens, do, initial_state, dhT, workspace)

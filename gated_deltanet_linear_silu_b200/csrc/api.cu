@@ -63,8 +63,9 @@ uint64_t wait_limit_ns() {
 
 extern "C" {
 
-// 0.2.2: gdn_prefill_gated; 0.2.1: gdn_set_wait_limit_ns; 0.2.0: Hk, undecayed, gdn_backward
-int gdn_version(void) { return 202; }
+// 0.2.3: gdn_backward_workspace_size_kept; 0.2.2: gdn_prefill_gated; 0.2.1: gdn_set_wait_limit_ns;
+// 0.2.0: Hk, undecayed, gdn_backward
+int gdn_version(void) { return 203; }
 
 void gdn_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns < 0 ? -1 : ns, std::memory_order_relaxed); }
 
@@ -301,7 +302,13 @@ gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, void* conv
 
 size_t gdn_backward_workspace_size(int N, int64_t T_tot, int H, int dk, int dv) {
     if (N < 0 || T_tot < 0 || H <= 0 || dk <= 0 || dv <= 0) return 0;
-    const size_t b = gdn::backward_workspace_floats(N, T_tot, H, dk, dv) * sizeof(float);
+    const size_t b = gdn::backward_workspace_floats(N, T_tot, H, dk, dv, gdn::kCk) * sizeof(float);
+    return (b + 255) / 256 * 256 + 256;
+}
+
+size_t gdn_backward_workspace_size_kept(int N, int64_t T_tot, int H, int dk, int dv) {
+    if (N < 0 || T_tot < 0 || H <= 0 || dk <= 0 || dv <= 0) return 0;
+    const size_t b = gdn::backward_workspace_floats(N, T_tot, H, dk, dv, 1) * sizeof(float);
     return (b + 255) / 256 * 256 + 256;
 }
 
@@ -331,11 +338,13 @@ gdn_status_t gdn_backward(const void* q, const void* k, const void* v, gdn_dtype
     const size_t need = gdn_backward_workspace_size(N, T_tot, H, dk, dv);
     if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return GDN_ERR_WORKSPACE;
-    const int64_t slots = 2 * (int64_t)N + (T_tot + gdn::kCk - 1) / gdn::kCk + 1;
+    // every state kept (no recompute) when the workspace has room for it
+    const int ck = ws_bytes >= gdn_backward_workspace_size_kept(N, T_tot, H, dk, dv) ? 1 : gdn::kCk;
+    const int64_t slots = 2 * (int64_t)N + (T_tot + ck - 1) / ck + 1;
     float* ws = static_cast<float*>(workspace);
     gdn::BackwardArgs a{q, k, v, dtype == GDN_BF16, g, beta, cu_seqlens, N, T_tot, H, Hk, dk, dv,
                         scale, qk_l2norm, eps, h0, dO, dhT, dq, dk_out, dv_out, dg, dbeta, dh0,
-                        ws, ws + slots * H * (int64_t)dk * dv, slots, status_ptr()};
+                        ws, ck > 1 ? ws + slots * H * (int64_t)dk * dv : nullptr, slots, status_ptr(), ck};
     if (!a.status) return GDN_ERR_CUDA;
     return from_cuda(gdn::launch_backward(a, static_cast<cudaStream_t>(stream)));
 }

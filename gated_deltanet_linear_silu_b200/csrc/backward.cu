@@ -13,8 +13,8 @@
 // dq = scale (dq~ - q~ (q~ . dq~)) / |q|_eps with q~ = q / |q|_eps, dq~ = dq^.
 //
 // The reverse sweep needs S_{t-1} for every token: a forward pass stores the
-// state every kCk tokens (checkpoints in the workspace), then for each block of
-// kCk tokens, last block first, the states before each token are recomputed
+// state every ck tokens (checkpoints in the workspace), then for each block of
+// ck tokens, last block first, the states before each token are recomputed
 // into a per-CTA workspace buffer and the block is swept backwards.
 //
 // Layout: thread (rg, cg) holds rows [rg*RPT, rg*RPT+RPT) x columns [4cg, 4cg+4)
@@ -59,8 +59,9 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
     float* gps = scal + 16;         // [threads]
 
     const int64_t start = a.cu[n], end = a.cu[n + 1];
-    const int64_t ck_base = 2 * (int64_t)n + (start + kCk - 1) / kCk;  // first checkpoint slot
-    const int64_t nch = (end - start + kCk - 1) / kCk;
+    const int ck = a.ck;  // tokens between checkpoints: kCk, or 1 (every state kept)
+    const int64_t ck_base = 2 * (int64_t)n + (start + ck - 1) / ck;  // first checkpoint slot
+    const int64_t nch = (end - start + ck - 1) / ck;
     if (!(start >= 0 && start <= end && end <= a.T_tot && ck_base + nch <= a.ck_slots)) {
         if (tid == 0) set_status(a.status, kStatusBadSeqlens);
         return;
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
     const T* q = static_cast<const T*>(a.q);
     const T* k = static_cast<const T*>(a.k);
     const T* v = static_cast<const T*>(a.v);
-    float* buf = a.ws_buf + unit * kCk * DD;
+    float* buf = ck > 1 ? a.ws_buf + unit * ck * DD : nullptr;
     auto ckpt = [&](int64_t c) { return a.ws_ckpt + ((ck_base + c) * H + h) * DD; };
     auto load_tile = [&](const float* base, float4 (&x)[RPT]) {
 #pragma unroll
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
     // max(dk, dv) threads), and the next token's elements are requested into
     // registers while the current token is worked on: the guess is t + 1 in the
     // forward passes and t - 1 in the reverse sweep; a wrong guess (once per
-    // block of kCk tokens) just loads again.
+    // block of ck tokens) just loads again.
     struct Pref {
         float k, q, v, d, g, b;
         int64_t t;
@@ -191,14 +192,14 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
         }
     };
 
-    // ---- forward: checkpoints every kCk tokens
+    // ---- forward: checkpoints every ck tokens
     float4 S[RPT];
     if (a.h0) load_tile(a.h0 + unit * DD, S);
     else
 #pragma unroll
         for (int r = 0; r < RPT; ++r) S[r] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int64_t t = start; t < end; ++t) {
-        if ((t - start) % kCk == 0) store_tile(ckpt((t - start) / kCk), S);
+        if ((t - start) % ck == 0) store_tile(ckpt((t - start) / ck), S);
         forward_step(t, S);
     }
 
@@ -209,16 +210,18 @@ __global__ void __launch_bounds__(256) backward_kernel(BackwardArgs a) {
 #pragma unroll
         for (int r = 0; r < RPT; ++r) dS[r] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int64_t c = nch - 1; c >= 0; --c) {
-        const int64_t c0 = start + c * kCk, c1 = (c0 + kCk < end) ? c0 + kCk : end;
-        load_tile(ckpt(c), S);
-        for (int64_t t = c0; t < c1; ++t) {
-            store_tile(buf + (t - c0) * DD, S);  // the state before token t
-            if (t + 1 < c1) forward_step(t, S);
+        const int64_t c0 = start + c * ck, c1 = (c0 + ck < end) ? c0 + ck : end;
+        if (ck > 1) {  // recompute the block's states into buf
+            load_tile(ckpt(c), S);
+            for (int64_t t = c0; t < c1; ++t) {
+                store_tile(buf + (t - c0) * DD, S);  // the state before token t
+                if (t + 1 < c1) forward_step(t, S);
+            }
         }
         for (int64_t t = c1 - 1; t >= c0; --t) {
             __syncthreads();  // buf writes (and the previous token's reads) are done
             float4 Sp[RPT];
-            load_tile(buf + (t - c0) * DD, Sp);
+            load_tile(ck > 1 ? buf + (t - c0) * DD : ckpt(c), Sp);  // the state before token t
             load_token(t, true, t - 1, true);
             const float al = scal[0], be = scal[1];
             // A: m = a Sp^T k^, delta; r = Sp do
@@ -352,9 +355,9 @@ cudaError_t launch_t(const BackwardArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-size_t backward_workspace_floats(int N, int64_t T_tot, int H, int dk, int dv) {
-    const int64_t slots = 2 * (int64_t)N + (T_tot + kCk - 1) / kCk + 1;
-    return (size_t)(slots * H + (int64_t)N * H * kCk) * dk * dv;
+size_t backward_workspace_floats(int N, int64_t T_tot, int H, int dk, int dv, int ck) {
+    const int64_t slots = 2 * (int64_t)N + (T_tot + ck - 1) / ck + 1;
+    return (size_t)(slots * H + (ck > 1 ? (int64_t)N * H * ck : 0)) * dk * dv;
 }
 
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s) {

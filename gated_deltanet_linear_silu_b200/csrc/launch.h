@@ -103,11 +103,12 @@ struct BackwardArgs {
     float* dbeta;       // [T, H]
     float* dh0;         // [N, H, dk, dv] or null
     float* ws_ckpt;     // ck_slots x H checkpoints of dk x dv
-    float* ws_buf;      // N x H x kCk states of dk x dv
+    float* ws_buf;      // N x H x ck states of dk x dv (ck > 1)
     int64_t ck_slots;
     int* status;
+    int ck;             // tokens between checkpoints: kCk, or 1 (every state kept, no recompute)
 };
-size_t backward_workspace_floats(int N, int64_t T_tot, int H, int dk, int dv);
+size_t backward_workspace_floats(int N, int64_t T_tot, int H, int dk, int dv, int ck);
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t s);
 
 struct GatedNormArgs {

@@ -320,12 +320,21 @@ GDN_API gdn_status_t gdn_decode_layer_step(const void* x, const void* conv_w, vo
 GDN_API size_t gdn_backward_workspace_size(int N, int64_t T_tot, int H, int dk, int dv);
 
 /*
+ * Bytes with which gdn_backward keeps the state before every token from its
+ * forward pass instead of recomputing blocks of 16 (one of its three
+ * token-sequential passes fewer): 4 * dk * dv * H * (2N + T_tot + 1) bytes,
+ * rounded up. gdn_backward uses this mode whenever ws_bytes is at least this.
+ */
+GDN_API size_t gdn_backward_workspace_size_kept(int N, int64_t T_tot, int H, int dk, int dv);
+
+/*
  * Gradients of the recurrence gdn_prefill computes (decay-first order, [R]),
  * for upstream gradients dO of the output and dhT of the final state. fp32
  * arithmetic on CUDA cores, one CTA per (sequence, value head), token by
  * token: a forward pass stores the state every 16 tokens in the workspace,
  * then each block of 16 tokens, last first, recomputes its states and is
- * swept in reverse. Gradients flow through the L2 norms (when qk_l2norm) and
+ * swept in reverse (with a workspace of gdn_backward_workspace_size_kept
+ * bytes every state is stored and nothing is recomputed). Gradients flow through the L2 norms (when qk_l2norm) and
  * the query scale; the q, k gradients of a q/k head shared by several value
  * heads are the sums over them.
  *
@@ -390,7 +399,7 @@ GDN_API gdn_status_t gdn_check_device_status(void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH (0.2.0: q/k head count Hk,
  * the `undecayed` order, gdn_backward; 0.2.1: gdn_set_wait_limit_ns; 0.2.2:
- * gdn_prefill_gated). Argument
+ * gdn_prefill_gated; 0.2.3: gdn_backward_workspace_size_kept). Argument
  * lists change between minor versions; a binding checks the version before
  * calling anything else. */
 GDN_API int gdn_version(void);

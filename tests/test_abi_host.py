@@ -227,6 +227,10 @@ def test_backward_workspace_size_formula(L):
     floats = ((2 * N + (T + 15) // 16 + 1) * H + N * H * 16) * dk * dv
     got = L.gdn_backward_workspace_size(N, T, H, dk, dv)
     assert got % 256 == 0 and floats * 4 <= got <= floats * 4 + 512
+    # every state kept: a checkpoint slot per token, no recompute buffer
+    kept = (2 * N + T + 1) * H * dk * dv
+    got_k = L.gdn_backward_workspace_size_kept(N, T, H, dk, dv)
+    assert got_k % 256 == 0 and kept * 4 <= got_k <= kept * 4 + 512 and got_k > got
     assert _bwd(L, N=0, T=0, q=None, k=None, v=None, dO=None, dq=None, dkk=None, dvv=None,
                 dg=None, db=None, cu=None) == 0  # empty batch: nothing to do
 

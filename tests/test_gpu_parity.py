@@ -683,7 +683,7 @@ def test_decode_layer_step_equals_separate_kernels():
 # backward
 # ----------------------------------------------------------------------------
 
-def _backward_case(P, seed, with_dhT):
+def _backward_case(P, seed, with_dhT, keep_states=False):
     from oracle import backward as ob
     r = np.random.default_rng(seed)
     T, N = P.T_tot, P.N
@@ -700,24 +700,27 @@ def _backward_case(P, seed, with_dhT):
                        initial_state=None if P.h0 is None else dev_tensor(P.h0, "f32"),
                        dhT=None if dhT is None else dev_tensor(dhT, "f32"), scale=P.scale,
                        qk_l2norm=P.qk_l2norm, eps=P.eps,
-                       cu_seqlens_host=torch.from_numpy(P.cu_seqlens.astype(np.int32)))
+                       cu_seqlens_host=torch.from_numpy(P.cu_seqlens.astype(np.int32)),
+                       keep_states=keep_states)
     gdn.check_device_status(DEV)
     return [host(x) for x in got], ref
 
 
+@pytest.mark.parametrize("keep_states", [False, True])
 @pytest.mark.parametrize("kind,H,Hk,dk,dv,with_h0,with_dhT", [
     ("bf16", 2, 2, 128, 128, True, True),
     ("f32", 4, 2, 64, 48, False, True),
     ("f32", 3, 3, 32, 128, True, False),
 ])
-def test_backward_matches_oracle(kind, H, Hk, dk, dv, with_h0, with_dhT):
+def test_backward_matches_oracle(kind, H, Hk, dk, dv, with_h0, with_dhT, keep_states):
     """Gradients of q, k, v, g, beta and h0 against autograd of the fp64 oracle:
     ragged sequences (an empty one, one shorter than a checkpoint block, one spanning
     several blocks), grouped heads, with and without initial state and final-state
-    gradient. The inputs are the same values on both sides; the kernel computes in fp32."""
+    gradient, with the states recomputed per 16-token block or all kept from the
+    forward pass. The inputs are the same values on both sides; the kernel computes in fp32."""
     P = gi.random_prefill(19, [40, 0, 7, 35], H=H, Hk=Hk, dk=dk, dv=dv, dtype=kind,
                           with_h0=with_h0, scale=0.9)
-    got, ref = _backward_case(P, 20, with_dhT)
+    got, ref = _backward_case(P, 20, with_dhT, keep_states)
     for name, a_, b_ in zip(["dq", "dk", "dv", "dg", "dbeta", "dh0"], got, ref):
         assert err(a_, b_) <= TOL_F32, name
 
