@@ -878,9 +878,15 @@ def bench_layer(args, dist, pk):
         conv()
         gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, qk_l2norm=False)
 
-    conv_ms, layer_ms = [], []
+    st2 = torch.empty_like(st)
+
+    def fused():  # the conv inside the prefill kernel (gdn_prefill_layer)
+        gdn.prefill_layer(x, w, g, beta, cu, H=H, conv_state_out=st2, final_state=hT, out=o,
+                          workspace=ws)
+
+    conv_ms, layer_ms, fused_ms = [], [], []
     for rep in range(8):
-        for fn, acc in ((conv, conv_ms), (layer, layer_ms)):
+        for fn, acc in ((conv, conv_ms), (layer, layer_ms), (fused, fused_ms)):
             flush.fill_(rep & 0xFF)  # L2 flush: the layer's inputs fit in L2
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record(stream)
@@ -889,11 +895,13 @@ def bench_layer(args, dist, pk):
             torch.cuda.synchronize()
             if rep >= 3:
                 acc.append(s.elapsed_time(e))
-    cms, lms = statistics.median(conv_ms), statistics.median(layer_ms)
+    cms, lms, fms = (statistics.median(v) for v in (conv_ms, layer_ms, fused_ms))
     conv_bytes = 2 * T * Lw.C * 2 + Lw.C * 4 * 2
     return {"value": T / (lms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": lms,
             "workload": "layer_0p8b_T4096_conv_then_prefill",
             "note": "two launches (conv, prefill); the prefill reads q, k, v as strided views of the conv output",
+            "fused": {"value": T / (fms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": fms,
+                      "note": "gdn_prefill_layer: the conv inside the tensor-core prefill (no y round trip)"},
             "conv": {"ms": cms, "roofline": {
                 "bound": "hbm", "achieved": conv_bytes / (cms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": conv_bytes / (cms * 1e-3) / 1e9 / pk["hbm_gbs"],

@@ -26,7 +26,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
-ABI_VERSION = 203  # gdn_version() of the C ABI these argument lists describe
+ABI_VERSION = 204  # gdn_version() of the C ABI these argument lists describe
 
 GDN_F32, GDN_BF16 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tensor": 2}
@@ -65,6 +65,10 @@ def lib() -> ctypes.CDLL:
                                         i32, i64, i64, i64, f32, i32, f32, i32, i32, vp, vp, vp, vp,
                                         vp, f32, vp, sz, i32, vp]
         L.gdn_prefill_gated.restype = i32
+        L.gdn_prefill_layer.argtypes = [vp, vp, i32, vp, vp, i32, vp, vp, vp, vp, i32, i64, i32, i32,
+                                        i32, i32, f32, i32, f32, i32, vp, vp, vp, vp, vp, f32, vp, sz,
+                                        vp]
+        L.gdn_prefill_layer.restype = i32
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
                                       f32, i32, vp, vp]
         L.gdn_decode_layer_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, f32, i32, i32,
@@ -244,6 +248,54 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
                                          _ptr(workspace), workspace.numel(), ALGOS[algo],
                                          _stream(q.device))
         _check(st, "gdn_prefill_gated")
+    return o, hT
+
+
+def prefill_layer(x: torch.Tensor, conv_w: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                  cu_seqlens: torch.Tensor, *, H: int, Hk: Optional[int] = None, dk: int = 128,
+                  dv: int = 128, conv_state_in: Optional[torch.Tensor] = None,
+                  conv_state_out: Optional[torch.Tensor] = None,
+                  initial_state: Optional[torch.Tensor] = None, output_final_state: bool = True,
+                  final_state: Optional[torch.Tensor] = None, scale: float = 1.0,
+                  qk_l2norm: bool = True, eps: float = 1e-6, undecayed: bool = False,
+                  z: Optional[torch.Tensor] = None, norm_w: Optional[torch.Tensor] = None,
+                  norm_eps: float = 1e-6, cu_seqlens_host: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None
+                  ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """The whole mixer for a prefill with the conv fused into the chunked
+    prefill: x [T, C] bf16 fused [q | k | v] projections before the conv
+    (C = 2 Hk dk + H dv), conv_w [C, K] bf16, conv windows [N, C, K-1] bf16 in
+    (nullable: zeros) and out (nullable; may be conv_state_in), g, beta [T, H]
+    fp32, optional gate z [T, H, dv] with norm_w [dv] fp32. Returns (o, hT)."""
+    Hk = H if Hk is None else Hk
+    T, C = x.shape
+    K = conv_w.shape[1]
+    if Hk <= 0 or C != 2 * Hk * dk + H * dv:
+        raise ValueError(f"x has {C} channels; expected 2*Hk*dk + H*dv")
+    N = cu_seqlens.shape[0] - 1
+    o = torch.empty((T, H, dv), dtype=x.dtype, device=x.device) if out is None else out
+    hT = final_state
+    if hT is None and output_final_state:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=x.device)
+    with _on(x.device):  # the workspace can depend on the device's SM count
+        ws_bytes = prefill_workspace_size(N, T, H, dk, dv, 64)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    if z is not None and norm_w is None:
+        raise ValueError("a gated prefill needs norm_w")
+    _cuda(x, conv_w, conv_state_in, conv_state_out, g, beta, cu_seqlens, initial_state, hT, o, z,
+          norm_w, workspace)
+    host_cu = None
+    if cu_seqlens_host is not None:
+        host_cu = cu_seqlens_host.to(torch.int32).contiguous()
+    with _on(x.device):
+        st = lib().gdn_prefill_layer(
+            _ptr(x), _ptr(conv_w), K, _ptr(conv_state_in), _ptr(conv_state_out), _dtype_code(x), _ptr(g),
+            _ptr(beta), _ptr(cu_seqlens), None if host_cu is None else ctypes.c_void_p(host_cu.data_ptr()),
+            N, T, H, Hk, dk, dv, float(scale), int(qk_l2norm), float(eps), int(undecayed),
+            _ptr(initial_state), _ptr(hT), _ptr(o), _ptr(z), _ptr(norm_w), float(norm_eps),
+            _ptr(workspace), workspace.numel(), _stream(x.device))
+    _check(st, "gdn_prefill_layer")
     return o, hT
 
 

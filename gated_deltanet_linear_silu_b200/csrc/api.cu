@@ -63,9 +63,9 @@ uint64_t wait_limit_ns() {
 
 extern "C" {
 
-// 0.2.3: gdn_backward_workspace_size_kept; 0.2.2: gdn_prefill_gated; 0.2.1: gdn_set_wait_limit_ns;
-// 0.2.0: Hk, undecayed, gdn_backward
-int gdn_version(void) { return 203; }
+// 0.2.4: gdn_prefill_layer; 0.2.3: gdn_backward_workspace_size_kept; 0.2.2: gdn_prefill_gated;
+// 0.2.1: gdn_set_wait_limit_ns; 0.2.0: Hk, undecayed, gdn_backward
+int gdn_version(void) { return 204; }
 
 void gdn_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns < 0 ? -1 : ns, std::memory_order_relaxed); }
 
@@ -137,14 +137,24 @@ size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, i
 
 namespace {
 
-// gdn_prefill and gdn_prefill_gated (z == nullptr: no gate).
+// The layer input's conv, fused into the tensor-core prefill (gdn_prefill_layer).
+struct ConvIn {
+    const void* w;
+    int K;
+    const void* state_in;
+    void* state_out;
+};
+
+// gdn_prefill, gdn_prefill_gated (z == nullptr: no gate) and gdn_prefill_layer
+// (conv != nullptr: q, k, v are the channels of x, ld_q = ld_k = ld_v = C).
 gdn_status_t prefill_impl(const void* q, const void* k, const void* v, gdn_dtype_t dtype,
                           const float* g, const float* beta, const int32_t* cu_seqlens,
                           const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H, int Hk,
                           int dk, int dv, int64_t ld_q, int64_t ld_k, int64_t ld_v, float scale,
                           int qk_l2norm, float eps, int undecayed, int chunk, const float* h0,
                           float* hT, void* o, void* workspace, size_t ws_bytes, gdn_algo_t algo,
-                          const void* z, const float* norm_w, float norm_eps, void* stream) {
+                          const void* z, const float* norm_w, float norm_eps, void* stream,
+                          const ConvIn* conv = nullptr) {
     if (Hk == 0) Hk = H;
     if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0 || Hk < 0 || H % Hk != 0)
         return GDN_ERR_INVALID_ARG;
@@ -183,6 +193,14 @@ gdn_status_t prefill_impl(const void* q, const void* k, const void* v, gdn_dtype
     if (!a.status) return GDN_ERR_CUDA;
     const bool tc_ok = gdn::prefill_tc_supported(a);
     if (algo == GDN_ALGO_TENSOR && !tc_ok) return GDN_ERR_UNSUPPORTED;
+    if (conv) {
+        // only the tensor-core kernel convolves; without tokens there is nothing to convolve
+        if (T_tot > 0 && !tc_ok) return GDN_ERR_UNSUPPORTED;
+        a.conv_w = conv->w;
+        a.conv_K = conv->K;
+        a.conv_state = conv->state_in;
+        a.conv_cu = cu_seqlens;
+    }
     const bool use_tc = tc_ok && algo != GDN_ALGO_SIMT;
     if (!use_tc && gdn::prefill_simt_smem_bytes(chunk, dk, dv) > 227 * 1024) return GDN_ERR_UNSUPPORTED;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -197,13 +215,23 @@ gdn_status_t prefill_impl(const void* q, const void* k, const void* v, gdn_dtype
         if (e != cudaSuccess) return GDN_ERR_CUDA;
         e = use_tc ? gdn::launch_prefill_tc(a, s) : gdn::launch_prefill_simt(a, s);
     }
-    if (e != cudaSuccess || !z || T_tot == 0) return from_cuda(e);
-    // The gate as a second pass over o, in place: one warp per row reduces the
-    // row's d_v values in registers. (Inside the tensor-core kernel's output
-    // epilogue, where a thread holds one d_v column of 64 tokens, the per-token
-    // reduction and gate loads cost more than this pass.)
-    gdn::GatedNormArgs gn{o, z, norm_w, dtype == GDN_BF16, T_tot * H, dv, norm_eps, o};
-    return from_cuda(gdn::launch_gated_rmsnorm(gn, s));
+    if (e != cudaSuccess) return from_cuda(e);
+    if (z && T_tot > 0) {
+        // The gate as a second pass over o, in place: one warp per row reduces the
+        // row's d_v values in registers. (Inside the tensor-core kernel's output
+        // epilogue, where a thread holds one d_v column of 64 tokens, the per-token
+        // reduction and gate loads cost more than this pass.)
+        gdn::GatedNormArgs gn{o, z, norm_w, dtype == GDN_BF16, T_tot * H, dv, norm_eps, o};
+        if ((e = gdn::launch_gated_rmsnorm(gn, s)) != cudaSuccess) return from_cuda(e);
+    }
+    if (conv && conv->state_out) {
+        // the conv windows the next call continues from (after every pass that read
+        // conv->state_in, so the update may be in place)
+        gdn::ConvArgs ca{q, 1, conv->w, cu_seqlens, N, T_tot, (int)ld_q, conv->K, conv->state_in,
+                         conv->state_out, 0, 0, 0, 0.f, nullptr, a.status};
+        e = gdn::launch_conv_state(ca, s);
+    }
+    return from_cuda(e);
 }
 
 }  // namespace
@@ -236,6 +264,35 @@ gdn_status_t gdn_prefill_gated(const void* q, const void* k, const void* v, gdn_
     return prefill_impl(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv,
                         ld_q, ld_k, ld_v, scale, qk_l2norm, eps, undecayed, chunk, h0, hT, o, workspace,
                         ws_bytes, algo, T_tot > 0 ? z : nullptr, norm_w, norm_eps, stream);
+}
+
+gdn_status_t gdn_prefill_layer(const void* x, const void* conv_w, int K, const void* conv_state_in,
+                               void* conv_state_out, gdn_dtype_t dtype, const float* g, const float* beta,
+                               const int32_t* cu_seqlens, const int32_t* cu_seqlens_host, int N,
+                               int64_t T_tot, int H, int Hk, int dk, int dv, float scale, int qk_l2norm,
+                               float eps, int undecayed, const float* h0, float* hT, void* o,
+                               const void* z, const float* norm_w, float norm_eps, void* workspace,
+                               size_t ws_bytes, void* stream) {
+    if (Hk == 0) Hk = H;
+    if (!dtype_ok(dtype) || N < 0 || T_tot < 0 || H <= 0 || Hk <= 0 || H % Hk != 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_BF16 || dk != 128 || dv != 128 || K < 1 || K > 4) return GDN_ERR_UNSUPPORTED;
+    if (T_tot > 0 && (!x || !conv_w)) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(conv_w) || !aligned16(conv_state_in) || !aligned16(conv_state_out))
+        return GDN_ERR_INVALID_ARG;
+    if (x && x == o) return GDN_ERR_INVALID_ARG;
+    if (z) {
+        if (!norm_w || !aligned16(z) || !aligned16(norm_w) || !(norm_eps >= 0.f) || z == o)
+            return GDN_ERR_INVALID_ARG;
+    }
+    const int64_t C = 2 * (int64_t)Hk * dk + (int64_t)H * dv;
+    const char* xb = static_cast<const char*>(x);
+    const void* q = x;
+    const void* k = xb ? xb + 2 * (int64_t)Hk * dk : nullptr;
+    const void* v = xb ? xb + 4 * (int64_t)Hk * dk : nullptr;
+    const ConvIn conv{conv_w, K, conv_state_in, conv_state_out};
+    return prefill_impl(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv, C, C,
+                        C, scale, qk_l2norm, eps, undecayed, 64, h0, hT, o, workspace, ws_bytes,
+                        GDN_ALGO_AUTO, T_tot > 0 ? z : nullptr, norm_w, norm_eps, stream, &conv);
 }
 
 int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_algo_t algo) {

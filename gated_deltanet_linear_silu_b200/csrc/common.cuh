@@ -49,6 +49,17 @@ __device__ __forceinline__ void store4(uint16_t* p, float4 v) {
     *reinterpret_cast<uint2*>(p) = u;
 }
 
+// SiLU for bf16 outputs, one XU operation: x sigmoid(x) = h + h tanh(h), h = x/2,
+// with the hardware tanh (PTX tanh.approx.f32: absolute error about 2^-11 on
+// tanh, so |error| <= |x| 2^-12 on SiLU -- below the bf16 rounding of the result
+// where SiLU is not vanishingly small).
+__device__ __forceinline__ float silu_tanh(float x) {
+    const float h = 0.5f * x;
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

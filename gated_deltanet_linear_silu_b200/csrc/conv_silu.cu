@@ -90,17 +90,6 @@ template <> struct Raw8<float> {
 // divide (both within a few ulp of fp32; the result is 0 when e^-x overflows).
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
-// SiLU for bf16 outputs, one XU operation: x sigmoid(x) = h + h tanh(h), h = x/2,
-// with the hardware tanh (PTX tanh.approx.f32: absolute error about 2^-11 on
-// tanh, so |error| <= |x| 2^-12 on SiLU -- below the bf16 rounding of the result
-// where SiLU is not vanishingly small).
-__device__ __forceinline__ float silu_tanh(float x) {
-    const float h = 0.5f * x;
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
-    return fmaf(h, t, h);
-}
-
 // One token's 8 channels as four fp32 pairs (bf16: exact widening).
 template <typename T> struct Pairs;
 template <> struct Pairs<uint16_t> {
@@ -373,6 +362,17 @@ cudaError_t launch_t(const ConvArgs& a, cudaStream_t s) {
 
 cudaError_t launch_conv_silu(const ConvArgs& a, cudaStream_t s) {
     return a.is_bf16 ? launch_t<uint16_t>(a, s) : launch_t<float>(a, s);
+}
+
+cudaError_t launch_conv_state(const ConvArgs& a, cudaStream_t s) {
+    if (!a.state_out || a.N <= 0 || a.K <= 1) return cudaSuccess;
+    const int64_t total = (int64_t)a.N * a.C;
+    const dim3 grid((unsigned)((total + 255) / 256));
+    if (a.is_bf16)
+        conv_state_kernel<uint16_t><<<grid, 256, 0, s>>>(a);
+    else
+        conv_state_kernel<float><<<grid, 256, 0, s>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace gdn

@@ -43,6 +43,8 @@ struct ConvArgs {
     int* status;
 };
 cudaError_t launch_conv_silu(const ConvArgs& a, cudaStream_t s);
+// The conv-state update alone (state_out from the last K-1 inputs of each sequence).
+cudaError_t launch_conv_state(const ConvArgs& a, cudaStream_t s);
 
 struct DecodeArgs {
     const void* q;
@@ -151,6 +153,16 @@ struct PrefillArgs {
     // Limit of each bounded hand-off wait inside the tensor-core kernel (ns);
     // 0: a wait whose phase is not complete at its first probe gives up.
     uint64_t wait_ns;
+    // Causal conv + SiLU of the layer input fused into the tensor-core kernel
+    // (conv_w != nullptr): q, k, v then point at the q, k, v channels of
+    // x [T_tot, C] (ld_q = ld_k = ld_v = C) and hold the raw rows; the kernel
+    // convolves each tile in shared memory before its first use.
+    const void* conv_w = nullptr;      // [C, K] bf16
+    int conv_K = 0;                    // taps, 1..4
+    const void* conv_state = nullptr;  // [N_seq, C, K-1] bf16 window before each sequence, or null (zeros)
+    const int32_t* conv_cu = nullptr;  // [N_seq + 1] sequence bounds of the conv windows
+    int conv_seg = 1;                  // units' sequence index / conv_seg = conv sequence (the split)
+    int conv_v = 1;                    // 0: the v tiles are used as loaded (the split's v = 0 pass)
 };
 // Default limit of the bounded hand-off waits (2 s) and the process-wide
 // setting (gdn_set_wait_limit_ns).

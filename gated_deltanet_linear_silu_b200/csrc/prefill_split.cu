@@ -274,6 +274,7 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
     PrefillArgs p = a;
     p.cu = cu_seg;
     p.N = NS;
+    p.conv_seg = S;  // fused conv: segment n of the split belongs to sequence n / S (a.cu's)
     p.order = reinterpret_cast<int32_t*>(ws + l.base.order_off);
     int32_t* counters = reinterpret_cast<int32_t*>(ws + l.base.counter_off);
     p.counter = counters;
@@ -287,9 +288,11 @@ cudaError_t launch_prefill_split(const PrefillArgs& a, int S, void* workspace, c
     if ((e = pass(0, a.h0 ? A : nullptr, Lst)) != cudaSuccess) return e;  // 1a
     p.v = zeros_v;
     p.ld_v = (int64_t)a.H * kSplitD;
+    p.conv_v = 0;  // fused conv: the zero values are used as loaded
     e = pass(1, B, Phi);  // 1b
     p.v = a.v;
     p.ld_v = a.ld_v;
+    p.conv_v = a.conv_v;
     if (e != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(split_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kCombSmem)) != cudaSuccess)

@@ -345,6 +345,100 @@ __device__ __forceinline__ bool item_next(const PrefillArgs& a, int units, Item&
     return true;
 }
 
+// ---- Fused conv ("7.6 Qwen3.5: linear-attention hybrid", 7.6.2: depthwise causal
+// Conv1d, kernel 4, padding 3, then SiLU). A producer lane owns one 16-byte column
+// (8 channels) of a 64-channel box of the stage: channel ch of x, whose row p
+// starts at xp + p * ld.
+
+// Taps of channels ch .. ch+7, right-aligned into a 4-wide window: w2[j][p] holds
+// tap j of the channel pair p (y_t = sum_j w2[j] x_{t-3+j}; zero taps for K < 4).
+__device__ __forceinline__ void conv_load_taps(const PrefillArgs& a, int ch, float2 (&w2)[4][4]) {
+    const uint16_t* w = static_cast<const uint16_t*>(a.conv_w);
+    const int K = a.conv_K;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int jj = j - (4 - K);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            float lo = 0.f, hi = 0.f;
+            if (jj >= 0) {
+                lo = bf16_to_f32(w[(int64_t)(ch + 2 * p) * K + jj]);
+                hi = bf16_to_f32(w[(int64_t)(ch + 2 * p + 1) * K + jj]);
+            }
+            w2[j][p] = make_float2(lo, hi);
+        }
+    }
+}
+
+// Raw input of the lane's 8 channels at token p of conv sequence nseq (first token
+// seq0): x from seq0 on; before it the sequence's conv state window (column
+// K-1 + p - seq0), or zeros where there is none.
+__device__ __forceinline__ void conv_fetch(const PrefillArgs& a, const uint16_t* xp, int ch, int nseq,
+                                           int64_t seq0, int64_t p, float2 (&x)[4]) {
+    if (p >= seq0) {
+        const uint4 u = *reinterpret_cast<const uint4*>(xp + p * a.ld_q);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) unpack_bf16(w[q], x[q].x, x[q].y);
+        return;
+    }
+    const int W = a.conv_K - 1;
+    const int64_t col = W + (p - seq0);
+    const uint16_t* st = static_cast<const uint16_t*>(a.conv_state);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float lo = 0.f, hi = 0.f;
+        if (st && col >= 0) {
+            lo = bf16_to_f32(st[((int64_t)nseq * a.ld_q + ch + 2 * q) * W + col]);
+            hi = bf16_to_f32(st[((int64_t)nseq * a.ld_q + ch + 2 * q + 1) * W + col]);
+        }
+        x[q] = make_float2(lo, hi);
+    }
+}
+
+// At the first chunk of a unit: the lane's taps and the raw rows c0-3 .. c0-1 before
+// the chunk (from x inside a sequence split into segments, else the conv state).
+__device__ __forceinline__ void conv_unit_start(const PrefillArgs& a, int n, int64_t c0, int ch,
+                                                const uint16_t* xp, float2 (&w2)[4][4], float2 (&win)[3][4]) {
+    conv_load_taps(a, ch, w2);
+    const int nseq = n / a.conv_seg;
+    const int64_t seq0 = a.conv_cu[nseq];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) conv_fetch(a, xp, ch, nseq, seq0, c0 - 3 + j, win[j]);
+}
+
+// Conv + SiLU in place over the 64 raw rows of one 16-byte column of a swizzled
+// bf16 box, with the arithmetic of the standalone conv (fp32 pairs, one-XU SiLU,
+// bf16 rounding). win comes in with the three raw rows before the box's first
+// row (oldest first) and leaves with its last three raw rows.
+__device__ __forceinline__ void conv_column(uint8_t* box, int c16, const float2 (&w2)[4][4],
+                                            float2 (&win)[3][4]) {
+#pragma unroll 4
+    for (int r = 0; r < kC; ++r) {
+        uint4* p = reinterpret_cast<uint4*>(box + sw128_off(r, c16));
+        const uint4 u = *p;
+        const uint32_t wi[4] = {u.x, u.y, u.z, u.w};
+        float2 xt[4];
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            unpack_bf16(wi[q], xt[q].x, xt[q].y);
+            float2 acc = __fmul2_rn(w2[0][q], win[0][q]);
+            acc = __ffma2_rn(w2[1][q], win[1][q], acc);
+            acc = __ffma2_rn(w2[2][q], win[2][q], acc);
+            acc = __ffma2_rn(w2[3][q], xt[q], acc);
+            o[q] = pack_bf16(silu_tanh(acc.x), silu_tanh(acc.y));
+        }
+        *p = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            win[0][q] = win[1][q];
+            win[1][q] = win[2][q];
+            win[2][q] = xt[q];
+        }
+    }
+}
+
 // Named barrier over `count` threads (warp multiple) with an OR-reduction.
 __device__ __forceinline__ bool group_any(int id, int count, bool pred) {
     uint32_t r;
@@ -395,6 +489,7 @@ __device__ __forceinline__ void issue_tiles(uint8_t* stage, uint64_t* bar, const
 // mbarriers (arrival count in parentheses; "commit" = tcgen05.commit).
 struct Bars {
     uint64_t full[kStages];      // tiles of a stage landed              (TMA bytes)
+    uint64_t conv_full[kStages];  // fused conv: tiles convolved          (warps 0 and 3, 1 each)
     uint64_t empty[kStages];     // tiles of a stage no longer read      (commit)
     uint64_t vfree[kStages];     // vector block of a stage no longer read (WG3, 1)
     uint64_t gready[kStages];    // gate vectors of a stage written      (gate warp, 1)
@@ -419,8 +514,10 @@ static_assert(sizeof(Bars) <= 512, "barrier block");
 
 // kUndecayed: each token reads the state before its own decay (row decay
 // gamma_{r-1} in A and W). A template parameter, so the default order's code is
-// not touched by the option.
-template <bool kUndecayed>
+// not touched by the option. kConv: the tiles are raw rows of the layer input,
+// convolved in shared memory by warp 0 (q, k) and the gate warp (v) before the
+// Gram MMA reads them.
+template <bool kUndecayed, bool kConv>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CUtensorMap map_q,
                   const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
@@ -456,6 +553,7 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&B.full[s], 1);
+            mbar_init(&B.conv_full[s], 2);
             mbar_init(&B.empty[s], 1);
             mbar_init(&B.vfree[s], 1);
             mbar_init(&B.gready[s], 1);
@@ -498,7 +596,70 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         }
     };
 
-    if (warp == kWarpTma) {
+    if (warp == kWarpTma && kConv) {
+        // ================================== producer + conv of the q, k tiles
+        // Lane 0 keeps the raw rows of chunk i and of the chunks after it whose
+        // stage is already free in flight; then the warp convolves chunk i in
+        // place (a lane per 16-byte column of the Q0, K0, Q1, K1 boxes) and hands
+        // the stage to the Gram MMA. The producer walk (lane 0) takes the units;
+        // the conv walk reads them from the ring like every other role.
+        if (lane == 0) {
+            prefetch_tmap(&map_q);
+            prefetch_tmap(&map_k);
+            prefetch_tmap(&map_v);
+        }
+        const UnitRing cring{ring.slot, ring.counter, ring.status, ring.abort_flag, ring.wlim, false};
+        Item pit, cit;
+        bool phave = lane == 0 && item_first(a, units, pit);
+        int pi = 0;                              // next chunk to load
+        uint32_t issued = 0, issued_par = 0;     // last load per stage, for the drain
+        const int bi = lane >> 3, c16 = lane & 7;  // box (Q0, K0, Q1, K1) and column
+        const bool is_k = (bi & 1) != 0;
+        const int off = 64 * (bi >> 1) + 8 * c16;  // channel within the head
+        float2 w2[4][4], win[3][4];
+        bool have = item_first(a, units, cit);
+        for (int i = 0; have; ++i, have = item_next(a, units, cit, cring)) {
+            const int s = i % kStages, k = i / kStages;
+            bool ok = true;
+            if (lane == 0) {
+                while (phave) {
+                    const int ps = pi % kStages, pk = pi / kStages;
+                    if (pi <= i) {  // chunk i itself: wait for its stage
+                        if (!mbar_wait_or_abort(&B.empty[ps], (pk & 1) ^ 1, abort_flag, wlim)) {
+                            ok = false;
+                            break;
+                        }
+                    } else if (pi >= i + kStages || !mbar_test_wait(&B.empty[ps], (pk & 1) ^ 1)) {
+                        break;
+                    }
+                    issue_tiles(stage(ps), &B.full[ps], &map_q, &map_k, &map_v, pit.U.h / group, pit.U.h,
+                                pit.c0);
+                    issued |= 1u << ps;
+                    issued_par = (issued_par & ~(1u << ps)) | ((uint32_t)(pk & 1) << ps);
+                    ++pi;
+                    phave = item_next(a, units, pit, ring);
+                }
+                if (ok) ok = mbar_wait_or_abort(&B.full[s], k & 1, abort_flag, wlim);
+            }
+            if (!__shfl_sync(0xffffffffu, (int)ok, 0)) {
+                if (lane == 0) fail();
+                break;
+            }
+            mbar_test_wait(&B.full[s], k & 1);  // each lane's own acquire of the landed rows
+            const int hk = cit.U.h / group;
+            const uint16_t* xp = static_cast<const uint16_t*>(is_k ? a.k : a.q) + hk * kD + off;
+            if (cit.first) conv_unit_start(a, cit.U.n, cit.c0, (is_k ? a.Hk * kD : 0) + hk * kD + off, xp, w2, win);
+            conv_column(stage(s) + bi * kBox, c16, w2, win);
+            fence_proxy_async();  // the tiles are read by the tensor cores
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.conv_full[s]);
+        }
+        // Every copy lands before the CTA exits, also those nobody consumed.
+        if (lane == 0)
+            for (int s = 0; s < kStages; ++s)
+                if ((issued >> s) & 1u) mbar_wait(&B.full[s], (issued_par >> s) & 1u, kDrainNs);
+        __syncwarp();
+    } else if (warp == kWarpTma) {
         // ============================================================ producer
         if (lane == 0) {
             prefetch_tmap(&map_q);
@@ -535,7 +696,8 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             // Gram of chunk ig: [Q;K] K^T -> R_G, once R_G has been read
             auto gram = [&]() -> bool {
                 const int s = ig % kStages, k = ig / kStages;
-                if (!mbar_wait_or_abort(&B.full[s], k & 1, abort_flag, wlim)) return false;
+                if (!mbar_wait_or_abort(kConv ? &B.conv_full[s] : &B.full[s], k & 1, abort_flag, wlim))
+                    return false;
                 if (ig > 0 && !mbar_wait_or_abort(&B.g_free, (ig - 1) & 1, abort_flag, wlim)) return false;
                 tc_fence_after();
                 const uint8_t* st = stage(s);
@@ -555,9 +717,15 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
                 have_g = item_next(a, units, git, ring);
             }
             // The next chunk's Gram goes out before this chunk's W, so the Gram
-            // epilogue of chunk i + 1 can follow the solve of chunk i at once.
+            // epilogue of chunk i + 1 can follow the solve of chunk i at once. With
+            // the fused conv it goes early only if that chunk is convolved already
+            // (else it follows W, which must not wait for the next chunk's conv).
             for (int i = 0; ok && have_w; ++i, have_w = item_next(a, units, wit, ring)) {
-                if (have_g) {
+                if (kConv && have_g && ig == i) {  // chunk i's own Gram, deferred
+                    if (!(ok = gram())) break;
+                    have_g = item_next(a, units, git, ring);
+                }
+                if (have_g && (!kConv || mbar_test_wait(&B.conv_full[ig % kStages], (ig / kStages) & 1))) {
                     if (!(ok = gram())) break;
                     have_g = item_next(a, units, git, ring);
                 }
@@ -651,6 +819,9 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
         __syncwarp();
     } else if (warp == kWarpGate) {
         // ============================================================== gates
+        // (and, with the fused conv, the conv of the v tiles: lanes 0-15, a
+        // 16-byte column of the V0, V1 boxes each)
+        float2 vw2[4][4], vwin[3][4];
         Item it;
         bool have = item_first(a, units, it);
         for (int i = 0; have; ++i, have = item_next(a, units, it, ring)) {
@@ -701,6 +872,23 @@ prefill_tc_kernel(const __grid_constant__ TcParams P, const __grid_constant__ CU
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&B.gready[s]);
+            if constexpr (kConv) {
+                const bool okc = lane != 0 || mbar_wait_or_abort(&B.full[s], k & 1, abort_flag, wlim);
+                if (!__shfl_sync(0xffffffffu, (int)okc, 0)) {
+                    if (lane == 0) fail();
+                    break;
+                }
+                mbar_test_wait(&B.full[s], k & 1);
+                if (a.conv_v && lane < 16) {
+                    const int off = 64 * (lane >> 3) + 8 * (lane & 7);
+                    const uint16_t* xp = static_cast<const uint16_t*>(a.v) + it.U.h * kD + off;
+                    if (it.first) conv_unit_start(a, it.U.n, it.c0, 2 * a.Hk * kD + it.U.h * kD + off, xp, vw2, vwin);
+                    conv_column(stage(s) + (4 + (lane >> 3)) * kBox, lane & 7, vw2, vwin);
+                }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&B.conv_full[s]);
+            }
         }
     } else if (warp < kWg2) {
         // ===================== WG1: Gram epilogue (P, A, k norms), solve, T export
@@ -1264,7 +1452,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t s, bool pdl) {
     if (!make_map(&mq, a.q, a.Hk, a.T_tot, a.ld_q) || !make_map(&mk, a.k, a.Hk, a.T_tot, a.ld_k) ||
         !make_map(&mv, a.v, a.H, a.T_tot, a.ld_v))
         return cudaErrorInvalidValue;
-    auto kernel = a.undecayed ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    auto kernel = a.conv_w ? (a.undecayed ? prefill_tc_kernel<true, true> : prefill_tc_kernel<false, true>)
+                           : (a.undecayed ? prefill_tc_kernel<true, false> : prefill_tc_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemAlloc);
     if (e != cudaSuccess) return e;

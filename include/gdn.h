@@ -9,6 +9,9 @@
  *                    rolling conv state.
  *   gdn_prefill      chunked gated delta rule over packed variable-length
  *                    sequences, optional initial state, fp32 final state.
+ *   gdn_prefill_layer  the whole mixer for a prefill: the conv and SiLU of
+ *                    the layer input fused into the chunked prefill, L2 norms,
+ *                    the rolling conv state and (optionally) the gated output.
  *   gdn_decode_step  one recurrent token per sequence, state updated in place.
  *   gdn_decode_layer_step  the whole mixer for one decode token: conv update
  *                    from the conv state, SiLU, L2 norm, the recurrent step
@@ -254,6 +257,53 @@ GDN_API gdn_status_t gdn_prefill_noalloc(const void* q, const void* k, const voi
 GDN_API size_t gdn_prefill_noalloc_max_scratch(void);
 
 /*
+ * The whole mixer for a prefill: gdn_conv_silu and gdn_prefill (or
+ * gdn_prefill_gated when z is given) as one call in which the conv never
+ * leaves the chip. [C] [R] [G] [P]
+ *
+ * x holds the fused projections [q | k | v] (C = 2*Hk*dk + H*dv channels,
+ * head-major inside each block) of packed sequences, before the conv. For
+ * each channel c and token t of sequence n (start s_n):
+ *   y[t, c] = SiLU( sum_{j<K} w[c, j] * x'[t - K + 1 + j, c] )
+ * with x'[p] = x[p] for p >= s_n and, before the sequence, the sequence's
+ * conv window: x'[s_n - K + 1 + j] = conv_state_in[n, c, j] (oldest first;
+ * zeros when conv_state_in is null). y's q, k, v channels then enter the
+ * recurrence exactly as gdn_prefill's q, k, v (L2 norms of q and k when
+ * qk_l2norm, query scale, undecayed order, h0 -> hT), and o is gated as in
+ * gdn_prefill_gated when z is given. conv_state_out[n, c, j] receives the
+ * window the next call continues from: the last K-1 inputs of sequence n
+ * (reaching back into conv_state_in for sequences shorter than K-1).
+ *
+ * The conv runs inside the tensor-core prefill: its producer warps load raw
+ * rows of x with the tile copies the plain prefill uses for q, k, v and
+ * convolve each tile in shared memory (with the chunk's three preceding rows)
+ * before the chunk's first matrix product, so y is never written to memory.
+ * Its arithmetic is gdn_conv_silu's (fp32, SiLU through tanh.approx, y rounded
+ * to bf16); the L2 norms are applied in the prefill after that rounding.
+ *
+ *   x               [T_tot, C]       bf16   layer input (pre-conv)
+ *   conv_w          [C, K]           bf16   depthwise taps, K in 1..4
+ *   conv_state_in   [N, C, K-1]      bf16   nullable: zeros
+ *   conv_state_out  [N, C, K-1]      bf16   nullable: not written; may equal
+ *                                           conv_state_in (updated in place)
+ *   g, beta, cu_seqlens, cu_seqlens_host, h0, hT, o, workspace: as gdn_prefill
+ *   z, norm_w, norm_eps: as gdn_prefill_gated; z nullable (no gate)
+ * Supported: bf16, dk = dv = 128 (the tensor-core kernel; chunk 64); any H / Hk.
+ * The workspace is gdn_prefill_workspace_size(N, T_tot, H, dk, dv, 64) bytes.
+ * No buffer may overlap another except conv_state_out == conv_state_in, and o
+ * must not overlap x. Errors as gdn_prefill, plus GDN_ERR_UNSUPPORTED for
+ * another dtype, head dims or K.
+ */
+GDN_API gdn_status_t gdn_prefill_layer(const void* x, const void* conv_w, int K, const void* conv_state_in,
+                                       void* conv_state_out, gdn_dtype_t dtype, const float* g,
+                                       const float* beta, const int32_t* cu_seqlens,
+                                       const int32_t* cu_seqlens_host, int N, int64_t T_tot, int H,
+                                       int Hk, int dk, int dv, float scale, int qk_l2norm, float eps,
+                                       int undecayed, const float* h0, float* hT, void* o,
+                                       const void* z, const float* norm_w, float norm_eps,
+                                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * The prefill kernel gdn_prefill would run for these arguments:
  * GDN_ALGO_SIMT or GDN_ALGO_TENSOR, or -1 if the combination is unsupported.
  */
@@ -399,7 +449,8 @@ GDN_API gdn_status_t gdn_check_device_status(void* stream);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH (0.2.0: q/k head count Hk,
  * the `undecayed` order, gdn_backward; 0.2.1: gdn_set_wait_limit_ns; 0.2.2:
- * gdn_prefill_gated; 0.2.3: gdn_backward_workspace_size_kept). Argument
+ * gdn_prefill_gated; 0.2.3: gdn_backward_workspace_size_kept; 0.2.4:
+ * gdn_prefill_layer). Argument
  * lists change between minor versions; a binding checks the version before
  * calling anything else. */
 GDN_API int gdn_version(void);

@@ -116,6 +116,33 @@ def test_prefill_empty_batch_is_noop(L):
     assert _prefill(L, N=0, T=0, q=None, k=None, v=None, o=None, cu=None) == 0
 
 
+def _prefill_layer(L, **kw):
+    args = dict(x=FAKE, cw=FAKE, K=4, si=None, so=None, dt=1, g=FAKE, beta=FAKE, cu=FAKE, cu_host=None,
+                N=2, T=100, H=16, Hk=0, dk=128, dv=128, scale=1.0, l2=1, eps=1e-6, und=0, h0=None,
+                hT=None, o=ctypes.c_void_p(1 << 21), z=None, nw=None, neps=1e-6, ws=None, ws_bytes=0,
+                stream=None)
+    args.update(kw)
+    return L.gdn_prefill_layer(*args.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dt=0), 2), (dict(dt=5), 1), (dict(dk=64), 2), (dict(dv=64), 2), (dict(K=0), 2),
+    (dict(K=5), 2), (dict(H=6, Hk=4), 1), (dict(Hk=-1), 1), (dict(N=-1), 1), (dict(x=None), 1),
+    (dict(cw=None), 1), (dict(x=ctypes.c_void_p((1 << 20) + 8)), 1),
+    (dict(si=ctypes.c_void_p((1 << 20) + 2)), 1), (dict(o=FAKE), 1),   # o must not alias x
+    (dict(z=FAKE), 1),                                                   # a gate needs norm_w
+    (dict(z=ctypes.c_void_p(1 << 22), nw=FAKE, neps=-1.0), 1),
+    (dict(und=2), 1), (dict(eps=float("nan")), 1),
+    (dict(), 3), (dict(ws=ctypes.c_void_p(1 << 23), ws_bytes=16), 3),  # valid: the workspace is missing
+])
+def test_prefill_layer_rejects_bad_arguments(L, kw, expect):
+    assert _prefill_layer(L, **kw) == expect
+
+
+def test_prefill_layer_empty_batch_is_noop(L):
+    assert _prefill_layer(L, N=0, T=0, x=None, cw=None, o=None, cu=None, g=None, beta=None) == 0
+
+
 def _conv(L, **kw):
     args = dict(x=FAKE, dt=1, w=FAKE, cu=FAKE, N=1, T=16, C=6144, K=4, si=None, so=None, l2=1,
                 nqk=4096, hd=128, eps=1e-6, y=ctypes.c_void_p(1 << 21), stream=None)

@@ -762,6 +762,137 @@ def test_layer_0p8b_conv_then_prefill():
     assert err(host(hT), h_ref) <= TOL_BF16
 
 
+def _layer_inputs(seed, lens, H, Hk, K, with_state, with_h0, gate, d=128):
+    """Seeded layer-prefill inputs: pre-conv x [T, C] bf16, taps, conv windows,
+    gates, initial state and the output gate."""
+    C = 2 * Hk * d + H * d
+    x, w, cu, st = gi.random_mixed(seed, lens, C, K=K, dtype="bf16", with_state=with_state)
+    r = np.random.default_rng(np.random.SeedSequence([3000, seed]))
+    T, N = int(cu[-1]), len(lens)
+    g = (-np.log1p(np.exp(r.normal(size=(T, H)) + 1.0))).astype(np.float32)
+    beta = (1.0 / (1.0 + np.exp(-r.normal(size=(T, H))))).astype(np.float32)
+    h0 = (r.normal(size=(N, H, d, d)) * 0.1).astype(np.float32) if with_h0 else None
+    z = gi.to_bf16_bits(r.normal(size=(T, H, d)).astype(np.float32)) if gate else None
+    nw = (1.0 + 0.1 * r.normal(size=d)).astype(np.float32) if gate else None
+    return dict(x=x, w=w, cu=cu, st=st, g=g, beta=beta, h0=h0, z=z, nw=nw, H=H, Hk=Hk, d=d)
+
+
+def _layer_oracle(L, undecayed=False):
+    """The oracle's conv + SiLU (fp64, unnormalised), then its recurrence with
+    the L2 norms of q and k, then the gate."""
+    H, Hk, d = L["H"], L["Hk"], L["d"]
+    y, st_out = oracle.conv_silu(L["x"], L["w"], L["cu"], dtype="bf16", state_in=L["st"])
+    T = y.shape[0]
+    q = y[:, :Hk * d].reshape(T, Hk, d)
+    k = y[:, Hk * d:2 * Hk * d].reshape(T, Hk, d)
+    v = y[:, 2 * Hk * d:].reshape(T, H, d)
+    o, hT = oracle.recurrence(q, k, v, L["g"], L["beta"], L["cu"], dtype="f64", h0=L["h0"],
+                              qk_l2norm=True, undecayed=undecayed)
+    if L["z"] is not None:
+        o = oracle.gated_rmsnorm(o, gi.bf16_bits_to_f32(L["z"]).astype(np.float64), L["nw"], dtype="f64")
+    return o, hT, st_out
+
+
+def _layer_gpu(L, undecayed=False, in_place_state=False, workspace=None):
+    cu = torch.from_numpy(L["cu"].astype(np.int32)).to(DEV)
+    st_in = None if L["st"] is None else dev_tensor(L["st"], "bf16")
+    K = L["w"].shape[1]
+    st_out = st_in if in_place_state else torch.empty((len(L["cu"]) - 1, L["x"].shape[1], K - 1),
+                                                      dtype=torch.bfloat16, device=DEV)
+    o, hT = gdn.prefill_layer(dev_tensor(L["x"], "bf16"), dev_tensor(L["w"], "bf16"),
+                              dev_tensor(L["g"], "f32"), dev_tensor(L["beta"], "f32"), cu,
+                              H=L["H"], Hk=L["Hk"], conv_state_in=st_in, conv_state_out=st_out,
+                              initial_state=None if L["h0"] is None else dev_tensor(L["h0"], "f32"),
+                              undecayed=undecayed,
+                              z=None if L["z"] is None else dev_tensor(L["z"], "bf16"),
+                              norm_w=None if L["nw"] is None else dev_tensor(L["nw"], "f32"),
+                              workspace=workspace)
+    gdn.check_device_status(DEV)
+    return host(o), host(hT), host(st_out)
+
+
+@pytest.mark.parametrize("lens,H,Hk,K,with_state,with_h0,gate,undecayed,in_place", [
+    ([130, 0, 64, 1, 200, 3], 2, 2, 4, True, True, True, False, False),
+    ([130, 0, 64, 1, 200, 3], 2, 2, 4, True, False, False, False, True),
+    ([70, 129, 5], 4, 2, 3, False, True, False, True, False),
+    ([70, 129, 5], 2, 1, 2, True, False, True, False, False),
+    ([100, 2], 2, 2, 1, False, False, False, False, False),
+])
+def test_prefill_layer_matches_oracle(lens, H, Hk, K, with_state, with_h0, gate, undecayed, in_place):
+    """The conv fused into the tensor-core prefill against the oracle's conv,
+    recurrence and gate: every element of o and hT, and the conv windows out
+    bit-exact (a copy of inputs). Ragged, empty and one-token sequences, conv
+    windows reaching into the caller's state, grouped heads, K = 1 .. 4, the
+    read-before-decay order and the conv state updated in place."""
+    L = _layer_inputs(70 + K + H, lens, H, Hk, K, with_state, with_h0, gate)
+    o, hT, st = _layer_gpu(L, undecayed=undecayed, in_place_state=in_place and with_state)
+    o_ref, h_ref, st_ref = _layer_oracle(L, undecayed=undecayed)
+    assert err(o, o_ref) <= TOL_BF16
+    assert err(hT, h_ref) <= TOL_BF16
+    if K > 1:
+        assert np.array_equal(st, gi.bf16_bits_to_f32(gi.to_bf16_bits(st_ref.astype(np.float32))))
+
+
+def test_prefill_layer_equals_conv_then_prefill():
+    """Fused and two-call layer (gdn_conv_silu without the norms, then
+    gdn_prefill with them on strided views of its output) agree to bf16
+    rounding of the conv output."""
+    L = _layer_inputs(81, [300, 17, 0, 96], 2, 2, 4, True, True, False)
+    o, hT, _ = _layer_gpu(L)
+    H, d = 2, 128
+    cu = torch.from_numpy(L["cu"].astype(np.int32)).to(DEV)
+    y, _ = gdn.conv_silu(dev_tensor(L["x"], "bf16"), dev_tensor(L["w"], "bf16"), cu,
+                         conv_state=dev_tensor(L["st"], "bf16"), qk_l2norm=False)
+    T = y.shape[0]
+    qkv = y.view(T, 3, H, d)
+    o2, h2 = gdn.prefill(qkv[:, 0], qkv[:, 1], qkv[:, 2], dev_tensor(L["g"], "f32"),
+                         dev_tensor(L["beta"], "f32"), cu, initial_state=dev_tensor(L["h0"], "f32"))
+    gdn.check_device_status(DEV)
+    assert err(o, host(o2)) <= 1e-2 and err(hT, host(h2)) <= 1e-2
+
+
+@pytest.mark.parametrize("lens,H,Hk,with_state", [
+    ([4096], 2, 2, True),
+    ([3000, 0, 5000], 2, 1, True),
+    ([2500, 700], 2, 2, False),
+])
+def test_prefill_layer_sequence_split(lens, H, Hk, with_state):
+    """Few units: the fused layer through the sequence split (segments that
+    start inside a sequence take their conv window from x, the v = 0 pass
+    leaves v unconvolved) against the oracle and against the plain launch."""
+    L = _layer_inputs(90 + len(lens), lens, H, Hk, 4, with_state, True, False)
+    N, T = len(lens), int(L["cu"][-1])
+    assert gdn.prefill_workspace_size(N, T, H, 128, 128) > 256 + (4 * N + 255) // 256 * 256
+    o, hT, st = _layer_gpu(L)
+    base_ws = torch.empty(256 + (4 * N + 255) // 256 * 256, dtype=torch.uint8, device=DEV)
+    o1, h1, _ = _layer_gpu(L, workspace=base_ws)
+    o_ref, h_ref, st_ref = _layer_oracle(L)
+    assert err(o, o_ref) <= TOL_BF16 and err(hT, h_ref) <= TOL_BF16
+    assert err(o1, o_ref) <= TOL_BF16 and err(h1, h_ref) <= TOL_BF16
+    assert np.array_equal(st, gi.bf16_bits_to_f32(gi.to_bf16_bits(st_ref.astype(np.float32))))
+
+
+def test_prefill_layer_more_units_than_sms():
+    """40 sequences x 4 heads (160 units on 148 SMs): CTAs move from unit to
+    unit, reloading taps and conv windows at each unit's first chunk."""
+    lens = [(37 * i) % 150 + 1 for i in range(40)]
+    L = _layer_inputs(95, lens, 4, 4, 4, True, False, False)
+    o, hT, _ = _layer_gpu(L)
+    o_ref, h_ref, _ = _layer_oracle(L)
+    assert err(o, o_ref) <= TOL_BF16 and err(hT, h_ref) <= TOL_BF16
+
+
+def test_layer_0p8b_fused():
+    """The 0.8B-shaped layer (T=4096, 16 heads of 128) through the fused call,
+    every element against the oracle."""
+    Lw = gi.layer_0p8b()
+    L = dict(x=Lw.mixed_qkv, w=Lw.conv_w, cu=np.asarray(Lw.cu_seqlens), st=None, g=Lw.g,
+             beta=Lw.beta, h0=None, z=None, nw=None, H=Lw.H, Hk=Lw.H, d=Lw.dk)
+    o, hT, _ = _layer_gpu(L)
+    o_ref, h_ref, _ = _layer_oracle(L)
+    assert err(o, o_ref) <= TOL_BF16 and err(hT, h_ref) <= TOL_BF16
+
+
 @pytest.mark.parametrize("lengths,H,Hk,undecayed,with_h0,in_place", [
     ([3000, 0, 1400, 4200], 2, 1, False, True, True),
     ([4096], 8, 8, True, False, False),
