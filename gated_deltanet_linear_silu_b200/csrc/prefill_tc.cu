@@ -350,8 +350,10 @@ __device__ __forceinline__ bool item_next(const PrefillArgs& a, int units, Item&
 // (8 channels) of a 64-channel box of the stage: channel ch of x, whose row p
 // starts at xp + p * ld.
 
-// Taps of channels ch .. ch+7, right-aligned into a 4-wide window: w2[j][p] holds
-// tap j of the channel pair p (y_t = sum_j w2[j] x_{t-3+j}; zero taps for K < 4).
+// Half the taps of channels ch .. ch+7, right-aligned into a 4-wide window: w2[j][p]
+// holds tap j of the channel pair p times 1/2, so the sum is h = y/2 of
+// y_t = sum_j w[j] x_{t-3+j} (zero taps for K < 4), SiLU's argument; scaling by a
+// power of two commutes with the rounding, so h is exactly half the fp32 sum.
 __device__ __forceinline__ void conv_load_taps(const PrefillArgs& a, int ch, float2 (&w2)[4][4]) {
     const uint16_t* w = static_cast<const uint16_t*>(a.conv_w);
     const int K = a.conv_K;
@@ -362,8 +364,8 @@ __device__ __forceinline__ void conv_load_taps(const PrefillArgs& a, int ch, flo
         for (int p = 0; p < 4; ++p) {
             float lo = 0.f, hi = 0.f;
             if (jj >= 0) {
-                lo = bf16_to_f32(w[(int64_t)(ch + 2 * p) * K + jj]);
-                hi = bf16_to_f32(w[(int64_t)(ch + 2 * p + 1) * K + jj]);
+                lo = 0.5f * bf16_to_f32(w[(int64_t)(ch + 2 * p) * K + jj]);
+                hi = 0.5f * bf16_to_f32(w[(int64_t)(ch + 2 * p + 1) * K + jj]);
             }
             w2[j][p] = make_float2(lo, hi);
         }
@@ -408,12 +410,14 @@ __device__ __forceinline__ void conv_unit_start(const PrefillArgs& a, int n, int
 }
 
 // Conv + SiLU in place over the 64 raw rows of one 16-byte column of a swizzled
-// bf16 box, with the arithmetic of the standalone conv (fp32 pairs, one-XU SiLU,
+// bf16 box, with the arithmetic of the standalone conv (fp32 pairs; SiLU(y) =
+// h + h tanh(h) with h = y/2 from the halved taps, one XU operation per element;
 // bf16 rounding). win comes in with the three raw rows before the box's first
-// row (oldest first) and leaves with its last three raw rows.
+// row (oldest first) and leaves with its last three raw rows. Unrolled by the
+// swizzle period (8 rows), so every row's offset is a constant.
 __device__ __forceinline__ void conv_column(uint8_t* box, int c16, const float2 (&w2)[4][4],
                                             float2 (&win)[3][4]) {
-#pragma unroll 4
+#pragma unroll 8
     for (int r = 0; r < kC; ++r) {
         uint4* p = reinterpret_cast<uint4*>(box + sw128_off(r, c16));
         const uint4 u = *p;
@@ -426,8 +430,12 @@ __device__ __forceinline__ void conv_column(uint8_t* box, int c16, const float2 
             float2 acc = __fmul2_rn(w2[0][q], win[0][q]);
             acc = __ffma2_rn(w2[1][q], win[1][q], acc);
             acc = __ffma2_rn(w2[2][q], win[2][q], acc);
-            acc = __ffma2_rn(w2[3][q], xt[q], acc);
-            o[q] = pack_bf16(silu_tanh(acc.x), silu_tanh(acc.y));
+            acc = __ffma2_rn(w2[3][q], xt[q], acc);  // h = y / 2
+            float2 t;
+            asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(acc.x));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(acc.y));
+            const float2 s = __ffma2_rn(acc, t, acc);
+            o[q] = pack_bf16(s.x, s.y);
         }
         *p = make_uint4(o[0], o[1], o[2], o[3]);
 #pragma unroll
