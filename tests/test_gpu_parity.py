@@ -851,22 +851,24 @@ def test_prefill_layer_equals_conv_then_prefill():
     assert err(o, host(o2)) <= 1e-2 and err(hT, host(h2)) <= 1e-2
 
 
-@pytest.mark.parametrize("lens,H,Hk,with_state", [
-    ([4096], 2, 2, True),
-    ([3000, 0, 5000], 2, 1, True),
-    ([2500, 700], 2, 2, False),
+@pytest.mark.parametrize("lens,H,Hk,with_state,undecayed,in_place", [
+    ([4096], 2, 2, True, False, True),
+    ([3000, 0, 5000], 2, 1, True, True, False),
+    ([2500, 700], 2, 2, False, False, False),
 ])
-def test_prefill_layer_sequence_split(lens, H, Hk, with_state):
+def test_prefill_layer_sequence_split(lens, H, Hk, with_state, undecayed, in_place):
     """Few units: the fused layer through the sequence split (segments that
     start inside a sequence take their conv window from x, the v = 0 pass
-    leaves v unconvolved) against the oracle and against the plain launch."""
+    leaves v unconvolved) against the oracle and against the plain launch;
+    with the conv state updated in place (read by all three passes first) and
+    the read-before-decay order."""
     L = _layer_inputs(90 + len(lens), lens, H, Hk, 4, with_state, True, False)
     N, T = len(lens), int(L["cu"][-1])
     assert gdn.prefill_workspace_size(N, T, H, 128, 128) > 256 + (4 * N + 255) // 256 * 256
-    o, hT, st = _layer_gpu(L)
+    o, hT, st = _layer_gpu(L, undecayed=undecayed, in_place_state=in_place)
     base_ws = torch.empty(256 + (4 * N + 255) // 256 * 256, dtype=torch.uint8, device=DEV)
-    o1, h1, _ = _layer_gpu(L, workspace=base_ws)
-    o_ref, h_ref, st_ref = _layer_oracle(L)
+    o1, h1, _ = _layer_gpu(L, undecayed=undecayed, workspace=base_ws)
+    o_ref, h_ref, st_ref = _layer_oracle(L, undecayed=undecayed)
     assert err(o, o_ref) <= TOL_BF16 and err(hT, h_ref) <= TOL_BF16
     assert err(o1, o_ref) <= TOL_BF16 and err(h1, h_ref) <= TOL_BF16
     assert np.array_equal(st, gi.bf16_bits_to_f32(gi.to_bf16_bits(st_ref.astype(np.float32))))
