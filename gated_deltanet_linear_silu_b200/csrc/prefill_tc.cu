@@ -413,36 +413,44 @@ __device__ __forceinline__ void conv_unit_start(const PrefillArgs& a, int n, int
 // bf16 box, with the arithmetic of the standalone conv (fp32 pairs; SiLU(y) =
 // h + h tanh(h) with h = y/2 from the halved taps, one XU operation per element;
 // bf16 rounding). win comes in with the three raw rows before the box's first
-// row (oldest first) and leaves with its last three raw rows. Unrolled by the
-// swizzle period (8 rows), so every row's offset is a constant.
+// row (oldest first) and leaves with its last three raw rows. Rows go in batches
+// of four: all four loads before the first store, since a store to a swizzled
+// address would otherwise hold back the next row's load (the compiler cannot
+// tell the rows apart) and chain all 64 rows end to end.
 __device__ __forceinline__ void conv_column(uint8_t* box, int c16, const float2 (&w2)[4][4],
                                             float2 (&win)[3][4]) {
-#pragma unroll 8
-    for (int r = 0; r < kC; ++r) {
-        uint4* p = reinterpret_cast<uint4*>(box + sw128_off(r, c16));
-        const uint4 u = *p;
-        const uint32_t wi[4] = {u.x, u.y, u.z, u.w};
-        float2 xt[4];
-        uint32_t o[4];
+#pragma unroll 1
+    for (int r0 = 0; r0 < kC; r0 += 4) {
+        uint8_t* rows = box + r0 * 128;
+        const int sw = r0 & 4;  // the rows' swizzle phase
+        uint4 raw[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            unpack_bf16(wi[q], xt[q].x, xt[q].y);
-            float2 acc = __fmul2_rn(w2[0][q], win[0][q]);
-            acc = __ffma2_rn(w2[1][q], win[1][q], acc);
-            acc = __ffma2_rn(w2[2][q], win[2][q], acc);
-            acc = __ffma2_rn(w2[3][q], xt[q], acc);  // h = y / 2
-            float2 t;
-            asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(acc.x));
-            asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(acc.y));
-            const float2 s = __ffma2_rn(acc, t, acc);
-            o[q] = pack_bf16(s.x, s.y);
-        }
-        *p = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int b = 0; b < 4; ++b) raw[b] = *reinterpret_cast<const uint4*>(rows + sw128_off(sw + b, c16) - sw * 128);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            win[0][q] = win[1][q];
-            win[1][q] = win[2][q];
-            win[2][q] = xt[q];
+        for (int b = 0; b < 4; ++b) {
+            const uint32_t wi[4] = {raw[b].x, raw[b].y, raw[b].z, raw[b].w};
+            float2 xt[4];
+            uint32_t o[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                unpack_bf16(wi[q], xt[q].x, xt[q].y);
+                float2 acc = __fmul2_rn(w2[0][q], win[0][q]);
+                acc = __ffma2_rn(w2[1][q], win[1][q], acc);
+                acc = __ffma2_rn(w2[2][q], win[2][q], acc);
+                acc = __ffma2_rn(w2[3][q], xt[q], acc);  // h = y / 2
+                float2 t;
+                asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(acc.x));
+                asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(acc.y));
+                const float2 s = __ffma2_rn(acc, t, acc);
+                o[q] = pack_bf16(s.x, s.y);
+            }
+            *reinterpret_cast<uint4*>(rows + sw128_off(sw + b, c16) - sw * 128) = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                win[0][q] = win[1][q];
+                win[1][q] = win[2][q];
+                win[2][q] = xt[q];
+            }
         }
     }
 }
