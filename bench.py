@@ -879,14 +879,19 @@ def bench_layer(args, dist, pk):
         gdn.prefill(q, k, v, g, beta, cu, final_state=hT, out=o, workspace=ws, qk_l2norm=False)
 
     st2 = torch.empty_like(st)
+    ws_layer = torch.empty(gdn.prefill_layer_workspace_size(1, T, H, H), dtype=torch.uint8, device=dev)
 
-    def fused():  # the conv inside the prefill kernel (gdn_prefill_layer)
+    def layer_call():  # gdn_prefill_layer with its own workspace: the split applies, so conv first
+        gdn.prefill_layer(x, w, g, beta, cu, H=H, conv_state_out=st2, final_state=hT, out=o,
+                          workspace=ws_layer)
+
+    def fused():  # the conv inside each of the split's three prefill passes
         gdn.prefill_layer(x, w, g, beta, cu, H=H, conv_state_out=st2, final_state=hT, out=o,
                           workspace=ws)
 
-    conv_ms, layer_ms, fused_ms = [], [], []
+    conv_ms, layer_ms, call_ms, fused_ms = [], [], [], []
     for rep in range(8):
-        for fn, acc in ((conv, conv_ms), (layer, layer_ms), (fused, fused_ms)):
+        for fn, acc in ((conv, conv_ms), (layer, layer_ms), (layer_call, call_ms), (fused, fused_ms)):
             flush.fill_(rep & 0xFF)  # L2 flush: the layer's inputs fit in L2
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record(stream)
@@ -895,18 +900,80 @@ def bench_layer(args, dist, pk):
             torch.cuda.synchronize()
             if rep >= 3:
                 acc.append(s.elapsed_time(e))
-    cms, lms, fms = (statistics.median(v) for v in (conv_ms, layer_ms, fused_ms))
+    cms, lms, ams, fms = (statistics.median(v) for v in (conv_ms, layer_ms, call_ms, fused_ms))
     conv_bytes = 2 * T * Lw.C * 2 + Lw.C * 4 * 2
     return {"value": T / (lms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": lms,
             "workload": "layer_0p8b_T4096_conv_then_prefill",
             "note": "two launches (conv, prefill); the prefill reads q, k, v as strided views of the conv output",
+            "prefill_layer": {"value": T / (ams * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": ams,
+                              "note": "gdn_prefill_layer, its own workspace: the prefill splits, so the "
+                                      "conv runs first into the workspace"},
             "fused": {"value": T / (fms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": fms,
-                      "note": "gdn_prefill_layer: the conv inside the tensor-core prefill (no y round trip)"},
+                      "note": "gdn_prefill_layer with the prefill's workspace: the conv inside each "
+                              "of the split's three passes (no y round trip)"},
             "conv": {"ms": cms, "roofline": {
                 "bound": "hbm", "achieved": conv_bytes / (cms * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": conv_bytes / (cms * 1e-3) / 1e9 / pk["hbm_gbs"],
                 "traffic": profiled_traffic("conv_silu_kernel", ["conv_silu.cu"], T),
                 "algorithmic_bytes": conv_bytes}}}
+
+
+def bench_layer_long(args, dist, pk):
+    """The layer prefill at the headline's size: the long-prefill workload's
+    q, k, v side by side as the pre-conv layer input x (8 x 16384 tokens,
+    C = 6144), conv taps ~ N(0, 0.5) bf16 (seeded), its gates. Conv then prefill
+    (two calls, y through HBM) against gdn_prefill_layer (the conv inside the
+    single-pass prefill), alternated; inputs larger than L2."""
+    import numpy as np
+    import torch
+    import gated_deltanet_linear_silu_b200 as gdn
+    import gdn_inputs as gi
+    dev = torch.device("cuda", dist.local)
+    P = gi.long_prefill(SEQS, SEQ_LEN, H, D)
+    T = P.T_tot
+    C = 3 * H * D
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    x = torch.cat([bf(P.q).view(T, -1), bf(P.k).view(T, -1), bf(P.v).view(T, -1)], dim=1).contiguous()
+    r = np.random.default_rng(11)
+    w = bf(gi.to_bf16_bits((0.5 * r.standard_normal((C, 4))).astype(np.float32)))
+    g, beta = torch.from_numpy(P.g).to(dev), torch.from_numpy(P.beta).to(dev)
+    cu = torch.from_numpy(P.cu_seqlens).to(dev)
+    del P
+    y = torch.empty_like(x)
+    st = torch.empty((SEQS, C, 3), dtype=torch.bfloat16, device=dev)
+    st2 = torch.empty_like(st)
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    hT = torch.empty((SEQS, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_layer_workspace_size(SEQS, T, H, H), dtype=torch.uint8, device=dev)
+    qkv = y.view(T, 3, H, D)
+    stream = torch.cuda.current_stream(dev)
+
+    def two():
+        gdn.conv_silu(x, w, cu, conv_state_out=st, out=y, n_qk_channels=2 * H * D, head_dim=D)
+        gdn.prefill(qkv[:, 0], qkv[:, 1], qkv[:, 2], g, beta, cu, final_state=hT, out=o, workspace=ws,
+                    qk_l2norm=False)
+
+    def fused():
+        gdn.prefill_layer(x, w, g, beta, cu, H=H, conv_state_out=st2, final_state=hT, out=o, workspace=ws)
+
+    times = {"two": [], "fused": []}
+    for rep in range(max(args.warmup, 3) + 5):
+        for name, fn in (("two", two), ("fused", fused)):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            torch.cuda.synchronize()
+            if rep >= max(args.warmup, 3):
+                times[name].append(s.elapsed_time(e))
+    gdn.check_device_status(dev)
+    tms, fms = statistics.median(times["two"]), statistics.median(times["fused"])
+    return {"value": T / (fms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": fms,
+            "workload": "layer_8x16384_h16_d128_bf16_conv_k4",
+            "note": "gdn_prefill_layer: conv + SiLU inside the single-pass tensor-core prefill",
+            "two_calls": {"value": T / (tms * 1e-3) * dist.world, "unit": UNIT, "ms_per_step": tms,
+                          "note": "gdn_conv_silu, then gdn_prefill on token-strided views of y"},
+            "gpu_launches": 2 * 5}
 
 
 def run_ours(args, dist: Dist):
@@ -933,6 +1000,7 @@ def run_ours(args, dist: Dist):
     if not args.no_extras:
         extras["decode"] = bench_decode(args, dist, pk)
         extras["layer"] = bench_layer(args, dist, pk)
+        extras["layer_long"] = bench_layer_long(args, dist, pk)
         extras["varlen"] = bench_varlen(args, dist, pk)
         extras["decode_layer"] = bench_decode_layer(args, dist, pk)
         extras["gated_rmsnorm"] = bench_gated_norm(args, dist, pk)
@@ -1018,6 +1086,12 @@ def summarize(line, extras):
         s["grouped"] = {k: obj(v) for k, v in extras["grouped"].items()}
     if "undecayed" in extras:
         s["undecayed"] = {k: obj(v) for k, v in extras["undecayed"].items()}
+    if "layer" in extras and "prefill_layer" in extras["layer"]:
+        s["layer"]["prefill_layer_ms"] = r(extras["layer"]["prefill_layer"]["ms_per_step"])
+        s["layer"]["fused_ms"] = r(extras["layer"]["fused"]["ms_per_step"])
+    if "layer_long" in extras:
+        s["layer_long"] = {"ms": r(extras["layer_long"]["ms_per_step"]),
+                           "two_calls_ms": r(extras["layer_long"]["two_calls"]["ms_per_step"])}
     return s
 
 
@@ -1060,7 +1134,7 @@ def main():
 ONLY = {"decode": bench_decode, "layer": bench_layer, "varlen": bench_varlen,
         "decode_layer": bench_decode_layer, "gated_rmsnorm": bench_gated_norm,
         "grouped": bench_grouped, "undecayed": bench_undecayed, "backward": bench_backward,
-        "prefill_gated": bench_prefill_gated}
+        "prefill_gated": bench_prefill_gated, "layer_long": bench_layer_long}
 
 if __name__ == "__main__":
     main()

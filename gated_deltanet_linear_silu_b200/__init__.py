@@ -26,7 +26,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
-ABI_VERSION = 204  # gdn_version() of the C ABI these argument lists describe
+ABI_VERSION = 205  # gdn_version() of the C ABI these argument lists describe
 
 GDN_F32, GDN_BF16 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tensor": 2}
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
                                         i32, i32, f32, i32, f32, i32, vp, vp, vp, vp, vp, f32, vp, sz,
                                         vp]
         L.gdn_prefill_layer.restype = i32
+        L.gdn_prefill_layer_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
+        L.gdn_prefill_layer_workspace_size.restype = sz
         L.gdn_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i32, f32, i32,
                                       f32, i32, vp, vp]
         L.gdn_decode_layer_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, f32, i32, i32,
@@ -251,6 +253,10 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, 
     return o, hT
 
 
+def prefill_layer_workspace_size(N: int, T_tot: int, H: int, Hk: int, dk: int = 128, dv: int = 128) -> int:
+    return int(lib().gdn_prefill_layer_workspace_size(N, T_tot, H, Hk, dk, dv))
+
+
 def prefill_layer(x: torch.Tensor, conv_w: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
                   cu_seqlens: torch.Tensor, *, H: int, Hk: Optional[int] = None, dk: int = 128,
                   dv: int = 128, conv_state_in: Optional[torch.Tensor] = None,
@@ -266,7 +272,10 @@ def prefill_layer(x: torch.Tensor, conv_w: torch.Tensor, g: torch.Tensor, beta: 
     prefill: x [T, C] bf16 fused [q | k | v] projections before the conv
     (C = 2 Hk dk + H dv), conv_w [C, K] bf16, conv windows [N, C, K-1] bf16 in
     (nullable: zeros) and out (nullable; may be conv_state_in), g, beta [T, H]
-    fp32, optional gate z [T, H, dv] with norm_w [dv] fp32. Returns (o, hT)."""
+    fp32, optional gate z [T, H, dv] with norm_w [dv] fp32. Returns (o, hT).
+    The default workspace (prefill_layer_workspace_size) lets a call whose
+    prefill runs as the sequence split convolve once into it instead of in
+    each pass; a workspace of prefill_workspace_size bytes keeps it fused."""
     Hk = H if Hk is None else Hk
     T, C = x.shape
     K = conv_w.shape[1]
@@ -277,9 +286,9 @@ def prefill_layer(x: torch.Tensor, conv_w: torch.Tensor, g: torch.Tensor, beta: 
     hT = final_state
     if hT is None and output_final_state:
         hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=x.device)
-    with _on(x.device):  # the workspace can depend on the device's SM count
-        ws_bytes = prefill_workspace_size(N, T, H, dk, dv, 64)
     if workspace is None:
+        with _on(x.device):  # the workspace can depend on the device's SM count
+            ws_bytes = prefill_layer_workspace_size(N, T, H, Hk, dk, dv)
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
     if z is not None and norm_w is None:
         raise ValueError("a gated prefill needs norm_w")

@@ -63,9 +63,10 @@ uint64_t wait_limit_ns() {
 
 extern "C" {
 
-// 0.2.4: gdn_prefill_layer; 0.2.3: gdn_backward_workspace_size_kept; 0.2.2: gdn_prefill_gated;
-// 0.2.1: gdn_set_wait_limit_ns; 0.2.0: Hk, undecayed, gdn_backward
-int gdn_version(void) { return 204; }
+// 0.2.5: gdn_prefill_layer_workspace_size; 0.2.4: gdn_prefill_layer; 0.2.3:
+// gdn_backward_workspace_size_kept; 0.2.2: gdn_prefill_gated; 0.2.1: gdn_set_wait_limit_ns;
+// 0.2.0: Hk, undecayed, gdn_backward
+int gdn_version(void) { return 205; }
 
 void gdn_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns < 0 ? -1 : ns, std::memory_order_relaxed); }
 
@@ -137,13 +138,18 @@ size_t gdn_prefill_workspace_size(int N, int64_t T_tot, int H, int dk, int dv, i
 
 namespace {
 
-// The layer input's conv, fused into the tensor-core prefill (gdn_prefill_layer).
+// The layer input's conv (gdn_prefill_layer): fused into the tensor-core
+// prefill, or (y != nullptr) run first into y, whose channels the prefill then
+// reads in place.
 struct ConvIn {
     const void* w;
     int K;
     const void* state_in;
     void* state_out;
+    void* y;  // [T_tot, C] in the workspace, or nullptr: fused
 };
+
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
 // gdn_prefill, gdn_prefill_gated (z == nullptr: no gate) and gdn_prefill_layer
 // (conv != nullptr: q, k, v are the channels of x, ld_q = ld_k = ld_v = C).
@@ -196,10 +202,22 @@ gdn_status_t prefill_impl(const void* q, const void* k, const void* v, gdn_dtype
     if (conv) {
         // only the tensor-core kernel convolves; without tokens there is nothing to convolve
         if (T_tot > 0 && !tc_ok) return GDN_ERR_UNSUPPORTED;
-        a.conv_w = conv->w;
-        a.conv_K = conv->K;
-        a.conv_state = conv->state_in;
-        a.conv_cu = cu_seqlens;
+        if (conv->y) {
+            // the conv (and the conv state) first, into y; the prefill reads y's channels
+            gdn::ConvArgs ca{q, 1, conv->w, cu_seqlens, N, T_tot, (int)ld_q, conv->K, conv->state_in,
+                             conv->state_out, 0, 0, 128, 0.f, conv->y, a.status};
+            if (gdn::launch_conv_silu(ca, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_CUDA;
+            const char* x0 = static_cast<const char*>(q);
+            const char* y0 = static_cast<const char*>(conv->y);
+            a.q = y0;
+            a.k = y0 + (static_cast<const char*>(k) - x0);
+            a.v = y0 + (static_cast<const char*>(v) - x0);
+        } else {
+            a.conv_w = conv->w;
+            a.conv_K = conv->K;
+            a.conv_state = conv->state_in;
+            a.conv_cu = cu_seqlens;
+        }
     }
     const bool use_tc = tc_ok && algo != GDN_ALGO_SIMT;
     if (!use_tc && gdn::prefill_simt_smem_bytes(chunk, dk, dv) > 227 * 1024) return GDN_ERR_UNSUPPORTED;
@@ -224,7 +242,7 @@ gdn_status_t prefill_impl(const void* q, const void* k, const void* v, gdn_dtype
         gdn::GatedNormArgs gn{o, z, norm_w, dtype == GDN_BF16, T_tot * H, dv, norm_eps, o};
         if ((e = gdn::launch_gated_rmsnorm(gn, s)) != cudaSuccess) return from_cuda(e);
     }
-    if (conv && conv->state_out) {
+    if (conv && !conv->y && conv->state_out) {
         // the conv windows the next call continues from (after every pass that read
         // conv->state_in, so the update may be in place)
         gdn::ConvArgs ca{q, 1, conv->w, cu_seqlens, N, T_tot, (int)ld_q, conv->K, conv->state_in,
@@ -289,10 +307,31 @@ gdn_status_t gdn_prefill_layer(const void* x, const void* conv_w, int K, const v
     const void* q = x;
     const void* k = xb ? xb + 2 * (int64_t)Hk * dk : nullptr;
     const void* v = xb ? xb + 4 * (int64_t)Hk * dk : nullptr;
-    const ConvIn conv{conv_w, K, conv_state_in, conv_state_out};
+    // Where the prefill runs as the sequence split, the fused conv would be redone in
+    // each of its three passes: there the conv goes first, into y at the end of the
+    // workspace, when the workspace holds it (gdn_prefill_layer_workspace_size).
+    void* y = nullptr;
+    size_t ws_prefill = ws_bytes;
+    if (N > 0 && T_tot > 0 && workspace && gdn::prefill_split_segments(N, T_tot, H, dk, dv, 64) > 1) {
+        const size_t y_off = round256(gdn_prefill_workspace_size(N, T_tot, H, dk, dv, 64));
+        if (ws_bytes >= y_off + (size_t)T_tot * C * 2) {
+            y = static_cast<char*>(workspace) + y_off;
+            ws_prefill = y_off;
+        }
+    }
+    const ConvIn conv{conv_w, K, conv_state_in, conv_state_out, y};
     return prefill_impl(q, k, v, dtype, g, beta, cu_seqlens, cu_seqlens_host, N, T_tot, H, Hk, dk, dv, C, C,
-                        C, scale, qk_l2norm, eps, undecayed, 64, h0, hT, o, workspace, ws_bytes,
+                        C, scale, qk_l2norm, eps, undecayed, 64, h0, hT, o, workspace, ws_prefill,
                         GDN_ALGO_AUTO, T_tot > 0 ? z : nullptr, norm_w, norm_eps, stream, &conv);
+}
+
+size_t gdn_prefill_layer_workspace_size(int N, int64_t T_tot, int H, int Hk, int dk, int dv) {
+    const size_t base = gdn_prefill_workspace_size(N, T_tot, H, dk, dv, 64);
+    if (Hk == 0) Hk = H;
+    if (N <= 0 || T_tot <= 0 || H <= 0 || Hk <= 0 || gdn::prefill_split_segments(N, T_tot, H, dk, dv, 64) <= 1)
+        return base;
+    const int64_t C = 2 * (int64_t)Hk * dk + (int64_t)H * dv;
+    return round256(base) + round256((size_t)T_tot * C * 2);
 }
 
 int gdn_prefill_selected_algo(gdn_dtype_t dtype, int dk, int dv, int chunk, gdn_algo_t algo) {

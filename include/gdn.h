@@ -274,12 +274,18 @@ GDN_API size_t gdn_prefill_noalloc_max_scratch(void);
  * window the next call continues from: the last K-1 inputs of sequence n
  * (reaching back into conv_state_in for sequences shorter than K-1).
  *
- * The conv runs inside the tensor-core prefill: its producer warps load raw
- * rows of x with the tile copies the plain prefill uses for q, k, v and
- * convolve each tile in shared memory (with the chunk's three preceding rows)
- * before the chunk's first matrix product, so y is never written to memory.
- * Its arithmetic is gdn_conv_silu's (fp32, SiLU through tanh.approx, y rounded
- * to bf16); the L2 norms are applied in the prefill after that rounding.
+ * Where the prefill runs in one pass, the conv runs inside the tensor-core
+ * prefill: its producer warps load raw rows of x with the tile copies the plain
+ * prefill uses for q, k, v and convolve each tile in shared memory (with the
+ * chunk's three preceding rows) before the chunk's first matrix product, so y
+ * is never written to memory. Where the prefill runs as the sequence split
+ * (few sequence-head units; see gdn_prefill_workspace_size), whose three passes
+ * would each convolve again, the call instead runs gdn_conv_silu's kernels into
+ * y at the end of the workspace and the split prefill on y -- when ws_bytes is
+ * at least gdn_prefill_layer_workspace_size (with only
+ * gdn_prefill_workspace_size bytes it stays fused). Either way the arithmetic
+ * is gdn_conv_silu's (fp32, SiLU through tanh.approx, y rounded to bf16) and
+ * the L2 norms are applied in the prefill after that rounding.
  *
  *   x               [T_tot, C]       bf16   layer input (pre-conv)
  *   conv_w          [C, K]           bf16   depthwise taps, K in 1..4
@@ -289,7 +295,8 @@ GDN_API size_t gdn_prefill_noalloc_max_scratch(void);
  *   g, beta, cu_seqlens, cu_seqlens_host, h0, hT, o, workspace: as gdn_prefill
  *   z, norm_w, norm_eps: as gdn_prefill_gated; z nullable (no gate)
  * Supported: bf16, dk = dv = 128 (the tensor-core kernel; chunk 64); any H / Hk.
- * The workspace is gdn_prefill_workspace_size(N, T_tot, H, dk, dv, 64) bytes.
+ * The workspace is gdn_prefill_layer_workspace_size bytes (at least
+ * gdn_prefill_workspace_size(N, T_tot, H, dk, dv, 64)).
  * No buffer may overlap another except conv_state_out == conv_state_in, and o
  * must not overlap x. Errors as gdn_prefill, plus GDN_ERR_UNSUPPORTED for
  * another dtype, head dims or K.
@@ -302,6 +309,15 @@ GDN_API gdn_status_t gdn_prefill_layer(const void* x, const void* conv_w, int K,
                                        int undecayed, const float* h0, float* hT, void* o,
                                        const void* z, const float* norm_w, float norm_eps,
                                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Bytes of device workspace for gdn_prefill_layer (a multiple of 256):
+ * gdn_prefill_workspace_size(N, T_tot, H, dk, dv, 64), plus T_tot * C * 2
+ * bytes for y (C = 2*Hk*dk + H*dv; Hk = 0: H) when the prefill runs as the
+ * sequence split. Depends on the current device's SM count, like
+ * gdn_prefill_workspace_size.
+ */
+GDN_API size_t gdn_prefill_layer_workspace_size(int N, int64_t T_tot, int H, int Hk, int dk, int dv);
 
 /*
  * The prefill kernel gdn_prefill would run for these arguments:
@@ -450,7 +466,7 @@ GDN_API gdn_status_t gdn_check_device_status(void* stream);
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH (0.2.0: q/k head count Hk,
  * the `undecayed` order, gdn_backward; 0.2.1: gdn_set_wait_limit_ns; 0.2.2:
  * gdn_prefill_gated; 0.2.3: gdn_backward_workspace_size_kept; 0.2.4:
- * gdn_prefill_layer). Argument
+ * gdn_prefill_layer; 0.2.5: gdn_prefill_layer_workspace_size). Argument
  * lists change between minor versions; a binding checks the version before
  * calling anything else. */
 GDN_API int gdn_version(void);

@@ -139,6 +139,22 @@ def test_prefill_layer_rejects_bad_arguments(L, kw, expect):
     assert _prefill_layer(L, **kw) == expect
 
 
+def test_prefill_layer_workspace_size(L):
+    """The layer workspace adds y (T * C bf16) only where the prefill splits."""
+    pre = L.gdn_prefill_workspace_size(1, 4096, 16, 128, 128, 64)
+    lay = L.gdn_prefill_layer_workspace_size(1, 4096, 16, 0, 128, 128)
+    if pre > 256 + 256:  # one 4096-token sequence on 16 heads splits (on >= 96 SMs)
+        assert lay == (pre + 255) // 256 * 256 + 4096 * 3 * 16 * 128 * 2
+        assert L.gdn_prefill_layer_workspace_size(1, 4096, 16, 8, 128, 128) == \
+            (pre + 255) // 256 * 256 + 4096 * (2 * 8 + 16) * 128 * 2
+    else:
+        assert lay == pre
+    # eight 16384-token sequences on 16 heads fill the GPU: no split, no y
+    assert L.gdn_prefill_layer_workspace_size(8, 131072, 16, 16, 128, 128) == \
+        L.gdn_prefill_workspace_size(8, 131072, 16, 128, 128, 64)
+    assert lay % 256 == 0
+
+
 def test_prefill_layer_empty_batch_is_noop(L):
     assert _prefill_layer(L, N=0, T=0, x=None, cw=None, o=None, cu=None, g=None, beta=None) == 0
 

@@ -857,21 +857,29 @@ def test_prefill_layer_equals_conv_then_prefill():
     ([2500, 700], 2, 2, False, False, False),
 ])
 def test_prefill_layer_sequence_split(lens, H, Hk, with_state, undecayed, in_place):
-    """Few units: the fused layer through the sequence split (segments that
-    start inside a sequence take their conv window from x, the v = 0 pass
-    leaves v unconvolved) against the oracle and against the plain launch;
-    with the conv state updated in place (read by all three passes first) and
-    the read-before-decay order."""
+    """Few units, so the prefill runs as the sequence split. With the layer
+    workspace the conv goes first into it (once) and the split prefill reads y;
+    with the prefill's workspace the conv stays fused into all three passes
+    (segments that start inside a sequence take their conv window from x, the
+    v = 0 pass leaves v unconvolved); with only the schedule's workspace the
+    fused prefill runs in one pass. All three against the oracle, with the conv
+    state updated in place (read before it is rewritten) and the
+    read-before-decay order."""
     L = _layer_inputs(90 + len(lens), lens, H, Hk, 4, with_state, True, False)
     N, T = len(lens), int(L["cu"][-1])
-    assert gdn.prefill_workspace_size(N, T, H, 128, 128) > 256 + (4 * N + 255) // 256 * 256
+    pre = gdn.prefill_workspace_size(N, T, H, 128, 128)
+    assert pre > 256 + (4 * N + 255) // 256 * 256  # the split applies
+    assert gdn.prefill_layer_workspace_size(N, T, H, Hk) >= pre + T * (2 * Hk + H) * 128 * 2
     o, hT, st = _layer_gpu(L, undecayed=undecayed, in_place_state=in_place)
+    o_f, h_f, st_f = _layer_gpu(L, undecayed=undecayed, in_place_state=in_place,
+                                workspace=torch.empty(pre, dtype=torch.uint8, device=DEV))
     base_ws = torch.empty(256 + (4 * N + 255) // 256 * 256, dtype=torch.uint8, device=DEV)
     o1, h1, _ = _layer_gpu(L, undecayed=undecayed, workspace=base_ws)
     o_ref, h_ref, st_ref = _layer_oracle(L, undecayed=undecayed)
-    assert err(o, o_ref) <= TOL_BF16 and err(hT, h_ref) <= TOL_BF16
-    assert err(o1, o_ref) <= TOL_BF16 and err(h1, h_ref) <= TOL_BF16
-    assert np.array_equal(st, gi.bf16_bits_to_f32(gi.to_bf16_bits(st_ref.astype(np.float32))))
+    st_bits = gi.bf16_bits_to_f32(gi.to_bf16_bits(st_ref.astype(np.float32)))
+    for oo, hh in ((o, hT), (o_f, h_f), (o1, h1)):
+        assert err(oo, o_ref) <= TOL_BF16 and err(hh, h_ref) <= TOL_BF16
+    assert np.array_equal(st, st_bits) and np.array_equal(st_f, st_bits)
 
 
 def test_prefill_layer_more_units_than_sms():
@@ -884,8 +892,9 @@ def test_prefill_layer_more_units_than_sms():
     assert err(o, o_ref) <= TOL_BF16 and err(hT, h_ref) <= TOL_BF16
 
 
-def test_layer_0p8b_fused():
-    """The 0.8B-shaped layer (T=4096, 16 heads of 128) through the fused call,
+def test_layer_0p8b_prefill_layer():
+    """The 0.8B-shaped layer (T=4096, 16 heads of 128) through gdn_prefill_layer
+    with its default workspace (the prefill splits, so the conv runs first, once),
     every element against the oracle."""
     Lw = gi.layer_0p8b()
     L = dict(x=Lw.mixed_qkv, w=Lw.conv_w, cu=np.asarray(Lw.cu_seqlens), st=None, g=Lw.g,
