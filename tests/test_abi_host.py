@@ -210,6 +210,16 @@ def test_binding_rejects_head_shapes_the_abi_cannot_see(shapes):
         gdn.backward(q, k, v, gg, gg, cu, torch.zeros(8, v.shape[1], 16))
 
 
+@pytest.mark.parametrize("C,H,Hk", [(768, 2, 2), (1024, 2, 1), (512, 3, 1)])
+def test_binding_rejects_layer_channel_counts(C, H, Hk):
+    """prefill_layer needs C = 2 Hk dk + H dv channels (before any device work)."""
+    x = torch.zeros(8, C, dtype=torch.bfloat16)
+    w = torch.zeros(C, 4, dtype=torch.bfloat16)
+    gg = torch.zeros(8, H)
+    with pytest.raises(ValueError, match="channels"):
+        gdn.prefill_layer(x, w, gg, gg, torch.tensor([0, 8], dtype=torch.int32), H=H, Hk=Hk, dk=64, dv=64)
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "absent.so"))
     monkeypatch.setattr(gdn, "_lib", None)
